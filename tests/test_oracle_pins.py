@@ -1,0 +1,447 @@
+"""Pins of the CPU oracle to things other than itself (no GPU needed).
+
+Each test ties one oracle function to a hand-derived fixture (tests/golden),
+brute force on tiny inputs, a closed form, an invariant, or an independent
+numpy / torch recomputation in float64, chosen so that a dropped term, a wrong
+sign or index, or a transposed operand fails at least one of them.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+from quantized_routed_expert_tc_b200 import synth, workloads as W
+from tests.conftest import read_golden
+
+pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
+
+
+def ints(s):
+    return [int(v) for v in s.split(",")]
+
+
+def floats(s):
+    return [float(v) for v in s.split(",")]
+
+
+def np_codes(q: np.ndarray, K: int, bits: int) -> np.ndarray:
+    """Independent numpy decode of packed rows (two's-complement fields)."""
+    q = q.astype(np.int32)
+    per = 8 // bits
+    fields = [(q >> (bits * i)) & ((1 << bits) - 1) for i in range(per)]
+    codes = np.stack(fields, axis=-1).reshape(q.shape[0], -1)[:, :K]
+    return np.where(codes >= (1 << (bits - 1)), codes - (1 << bits), codes).astype(np.int64)
+
+
+# --------------------------------------------------------------------------- packing
+def test_pack_fixture():
+    for fmt, codes, hexbytes in read_golden("pack_codes.txt"):
+        bits, codes = int(fmt), ints(codes)
+        want = bytes(int(h, 16) for h in hexbytes.split())
+        # pack through the quantiser: a row whose values are the codes and whose
+        # absmax equals qmax quantises to exactly those codes with scale 1
+        qmax = oracle._load().qo_qmax(bits)
+        row = np.array(codes + [qmax], dtype=np.float32)
+        pad = (-row.size) % (8 // bits)
+        row = np.concatenate([row, np.zeros(pad, np.float32)])
+        if np.abs(row).max() > qmax:   # codes at qmin: scale differs, test unpack only
+            continue
+        q, s = oracle.quantize_rows(row[None, :], bits)
+        assert s[0] == 1.0
+        assert bytes(q[0, :len(want)]) == want, (bits, codes)
+
+
+def test_unpack_fixture_and_exhaustive():
+    for fmt, codes, hexbytes in read_golden("pack_codes.txt"):
+        bits, codes = int(fmt), ints(codes)
+        b = np.array([[int(h, 16) for h in hexbytes.split()]], dtype=np.uint8)
+        got = oracle.unpack_rows(b, len(codes), bits)[0].tolist()
+        assert got == codes
+    allb = np.arange(256, dtype=np.uint8)[:, None]
+    for bits in (8, 4, 2):
+        K = 8 // bits
+        got = oracle.unpack_rows(allb, K, bits).astype(np.int64)
+        assert np.array_equal(got, np_codes(allb, K, bits))
+        lo, hi = -(1 << (bits - 1)), (1 << (bits - 1)) - 1
+        assert got.min() == lo and got.max() == hi
+        # every byte decodes to a distinct code tuple: the map is a bijection
+        assert len({tuple(r) for r in got.tolist()}) == 256
+
+
+def test_int4_is_bit_consistent_with_int8_container():
+    """README '已实现的功能': packing verified bit-consistent with the int8 container.
+    The same codes held as int4 and as int8 give identical integer block dots and
+    identical FFN outputs with the same scales."""
+    rng = np.random.default_rng(7)
+    K, rows = 128, 16
+    codes = rng.integers(-8, 8, size=(rows, K)).astype(np.int64)
+    q4 = np.zeros((rows, K // 2), np.uint8)
+    q4[:] = ((codes[:, 0::2] & 0xF) | ((codes[:, 1::2] & 0xF) << 4)).astype(np.uint8)
+    q8 = (codes & 0xFF).astype(np.uint8)
+    xq = rng.integers(-127, 128, size=K).astype(np.int8)
+    a4 = oracle.block_dots_q8(q4, K, 4, xq)
+    a8 = oracle.block_dots_q8(q8, K, 8, xq)
+    assert np.array_equal(a4, a8)
+    ref = (codes.reshape(rows, K // 32, 32) * xq.astype(np.int64).reshape(K // 32, 32)).sum(-1)
+    assert np.array_equal(a4, ref)
+    # FFN through both containers
+    wl = W.TINY.with_(hidden=K, inter=64, n_experts=1, n_group=1, topk_group=1, top_k=1, T=2)
+    g = rng.integers(-8, 8, size=(64, K)); u = rng.integers(-8, 8, size=(64, K))
+    d = rng.integers(-8, 8, size=(K, 64))
+
+    def pack(c, bits):
+        c = np.asarray(c)
+        if bits == 8:
+            return (c & 0xFF).astype(np.uint8)
+        return ((c[:, 0::2] & 0xF) | ((c[:, 1::2] & 0xF) << 4)).astype(np.uint8)
+    sc = lambda n: (rng.random(n).astype(np.float32) * 0.01 + 0.001)
+    gs, us, ds = sc(64), sc(64), sc(K)
+    x = rng.standard_normal((2, K)).astype(np.float32)
+    outs = []
+    for bits in (4, 8):
+        ex = oracle.Expert(pack(g, bits), gs, pack(u, bits), us, pack(d, bits), ds)
+        for af in (W.A_F32, W.A_Q8):
+            h, y = oracle.shared_ffn(wl.with_(wbits=bits, afmt=af), ex, x)
+            outs.append((bits, af, h, y))
+    for af in (W.A_F32, W.A_Q8):
+        r4 = [o for o in outs if o[0] == 4 and o[1] == af][0]
+        r8 = [o for o in outs if o[0] == 8 and o[1] == af][0]
+        assert np.array_equal(r4[2], r8[2]) and np.array_equal(r4[3], r8[3])
+
+
+# --------------------------------------------------------------------------- quantiser
+def test_quantize_fixture():
+    for fmt, wv, scale, codes in read_golden("quantize_rows.txt"):
+        bits = int(fmt)
+        w = np.array([floats(wv)], np.float32)
+        q, s = oracle.quantize_rows(w, bits)
+        assert s[0] == np.float32(float(scale))
+        assert oracle.unpack_rows(q, w.shape[1], bits)[0].tolist() == ints(codes)
+
+
+@pytest.mark.parametrize("bits", [8, 4, 2])
+def test_quantize_is_nearest_code(bits):
+    """Brute force: each code is the nearest of all codes in [qmin, qmax] to w/s
+    (halves away from zero), the scale maps absmax to qmax, qmin never emitted."""
+    w = synth.normal_f32(11, bits, 64 * 96, 0.0, 0.02).reshape(64, 96)
+    w[3] = 0.0
+    q, s = oracle.quantize_rows(w, bits)
+    codes = oracle.unpack_rows(q, 96, bits).astype(np.int64)
+    qmax = (1 << (bits - 1)) - 1
+    qmin = -(1 << (bits - 1))
+    absmax = np.abs(w).max(axis=1)
+    assert s[3] == 0 and not codes[3].any()
+    nz = absmax > 0
+    assert np.allclose(s[nz].astype(np.float64) * qmax, absmax[nz], rtol=1e-6)
+    cand = np.arange(qmin, qmax + 1)
+    for r in np.nonzero(nz)[0]:
+        v = (w[r] / s[r]).astype(np.float64)            # the f32 quotient, widened
+        dist = np.abs(v[:, None] - cand[None, :])
+        best = dist.min(axis=1)
+        ok = np.isclose(dist, best[:, None], rtol=0, atol=1e-12)
+        # among equally near codes, the one farther from zero
+        pick = np.array([cand[o][np.argmax(np.abs(cand[o]))] for o in ok])
+        assert np.array_equal(codes[r], pick)
+        assert codes[r].min() >= -qmax          # qmin is never emitted
+        # reconstruction error at most half a step
+        assert np.all(np.abs(w[r] - s[r] * codes[r]) <= s[r] * 0.5 * (1 + 1e-6))
+
+
+# --------------------------------------------------------------------------- Q8_0
+def test_q8_fixture():
+    for xs, d, qs in read_golden("q8_block.txt"):
+        x = np.array(floats(xs), np.float32)
+        q, dd = oracle.quantize_q8(x)
+        assert dd[0] == np.float32(float(d))
+        assert q.tolist() == ints(qs)
+
+
+def test_q8_properties():
+    x = synth.normal_f32(12, 1, 32 * 64, 0.0, 1.0).reshape(64, 32)
+    x[5] = 0.0
+    x[6, 3] = 1e-30
+    q, d = oracle.quantize_q8(x)
+    q = q.astype(np.int64)
+    for b in range(64):
+        amax = np.abs(x[b]).max()
+        if amax == 0:
+            assert d[b, 0] == 0 and not q[b].any()
+            continue
+        assert np.isclose(float(d[b, 0]) * 127, amax, rtol=1e-6)
+        assert np.abs(q[b]).max() == 127 and np.abs(q[b]).max() <= 127
+        assert np.all(np.abs(x[b] - d[b, 0] * q[b]) <= d[b, 0] * 0.5 * (1 + 1e-5))
+
+
+def test_block_dots_exact():
+    rng = np.random.default_rng(3)
+    for bits in (8, 4, 2):
+        K = 256
+        w = synth.normal_f32(13, bits, 8 * K, 0.0, 0.02).reshape(8, K)
+        q, _ = oracle.quantize_rows(w, bits)
+        xq = rng.integers(-127, 128, size=K).astype(np.int8)
+        acc = oracle.block_dots_q8(q, K, bits, xq)
+        codes = np_codes(q, K, bits)
+        ref = (codes.reshape(8, K // 32, 32) * xq.astype(np.int64).reshape(K // 32, 32)).sum(-1)
+        assert np.array_equal(acc, ref)
+
+
+def test_bf16_rounding_matches_torch():
+    torch = pytest.importorskip("torch")
+    v = np.concatenate([synth.normal_f32(14, 1, 4000), np.array(
+        [1.0, 1.00390625, 1.0 + 2**-8 + 2**-20, 1.0 + 2**-9, 1.0 + 3 * 2**-9, -2.5, 0.0, 65504.0,
+         3.0e38, 1e-40], np.float32)])
+    ours = oracle.f32_to_bf16(v)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+# --------------------------------------------------------------------------- router
+def _router_case(E, G, Gk, k, rsf, s, bias):
+    wl = W.TINY.with_(hidden=1, n_experts=E, n_group=G, topk_group=Gk, top_k=k, rsf=rsf, T=1)
+    s = np.array(s, np.float64)
+    Wr = np.log(s / (1 - s)).astype(np.float32)[:, None]
+    x = np.ones((1, 1), np.float32)
+    return wl, oracle.router(wl, x, Wr, np.array(bias, np.float32))
+
+
+def test_router_fixture():
+    for case, shape, sv, bias, idx, wv in read_golden("router_tiny.txt"):
+        E, G, Gk, k = ints(shape.rsplit(",", 1)[0])
+        rsf = float(shape.rsplit(",", 1)[1])
+        wl, r = _router_case(E, G, Gk, k, rsf, floats(sv), floats(bias))
+        assert r["idx"][0].tolist() == ints(idx), case
+        assert np.allclose(r["w"][0], floats(wv), rtol=0, atol=2e-6), case
+        assert r["ties"][0] == 0
+
+
+def _brute_router(sc, s, G, Gk, k, rsf):
+    """Enumerate every kept-group set and every k-subset of its experts."""
+    E = sc.size
+    gs = E // G
+    gscore = [np.sort(sc[g * gs:(g + 1) * gs])[::-1][:2].sum() for g in range(G)]
+    best_groups = max(itertools.combinations(range(G), Gk),
+                      key=lambda c: (sum(gscore[g] for g in c), [-g for g in c]))
+    cand = [e for e in range(E) if e // gs in best_groups]
+    best = max(itertools.combinations(cand, k), key=lambda c: (sum(sc[e] for e in c), [-e for e in c]))
+    chosen = sorted(best, key=lambda e: (-sc[e], e))
+    w = np.array([s[e] for e in chosen]) / sum(s[e] for e in chosen) * rsf
+    return chosen, w
+
+
+@pytest.mark.parametrize("E,G,Gk,k", [(16, 4, 2, 4), (12, 3, 2, 3), (8, 1, 1, 3), (8, 8, 4, 4),
+                                      (16, 2, 1, 5)])
+def test_router_brute_force(E, G, Gk, k):
+    H, T = 24, 24
+    wl = W.TINY.with_(hidden=H, n_experts=E, n_group=G, topk_group=Gk, top_k=k, T=T)
+    x = synth.normal_f32(21, E, T * H).reshape(T, H)
+    Wr = synth.normal_f32(22, E, E * H, 0, 0.3).reshape(E, H)
+    bias = synth.normal_f32(23, E, E, 0, 0.1)
+    r = oracle.router(wl, x, Wr, bias)
+    # logits: independent f64 matmul, rounded to f32
+    lg = (x.astype(np.float64) @ Wr.astype(np.float64).T).astype(np.float32)
+    assert np.array_equal(lg, r["logits"])
+    s = r["scores"].astype(np.float64)
+    assert np.allclose(s, 1 / (1 + np.exp(-lg.astype(np.float64))), rtol=1e-7, atol=0)
+    for t in range(T):
+        sc = (r["scores"][t] + bias).astype(np.float32).astype(np.float64)
+        chosen, w = _brute_router(sc, s[t], G, Gk, k, wl.rsf)
+        if r["ties"][t]:
+            continue
+        assert r["idx"][t].tolist() == chosen
+        assert np.allclose(r["w"][t], w, rtol=1e-6)
+        assert abs(float(r["w"][t].astype(np.float64).sum()) - wl.rsf) <= 1e-6 * wl.rsf
+
+
+def test_router_special_cases():
+    E, H, T, k = 16, 32, 16, 4
+    x = synth.normal_f32(31, 0, T * H).reshape(T, H)
+    Wr = synth.normal_f32(32, 0, E * H, 0, 0.3).reshape(E, H)
+    # one group: plain top-k of sc;  zero bias: top-k of logits (sigmoid is monotone)
+    wl = W.TINY.with_(hidden=H, n_experts=E, n_group=1, topk_group=1, top_k=k, T=T)
+    r = oracle.router(wl, x, Wr, np.zeros(E, np.float32))
+    lg = (x.astype(np.float64) @ Wr.astype(np.float64).T)
+    for t in range(T):
+        ref = sorted(range(E), key=lambda e: (-lg[t, e], e))[:k]
+        assert r["idx"][t].tolist() == ref
+    # G = Gk: group limiting keeps every group, same as one group
+    wl2 = wl.with_(n_group=4, topk_group=4)
+    r2 = oracle.router(wl2, x, Wr, np.zeros(E, np.float32))
+    assert np.array_equal(r["idx"], r2["idx"]) and np.array_equal(r["w"], r2["w"])
+    # the bias moves selection but never the weights' formula: weights are s/sum(s)*rsf
+    bias = synth.normal_f32(33, 0, E, 0, 0.5)
+    r3 = oracle.router(wl, x, Wr, bias)
+    for t in range(T):
+        s_sel = r3["scores"][t, r3["idx"][t]].astype(np.float64)
+        assert np.allclose(r3["w"][t], s_sel / s_sel.sum() * wl.rsf, rtol=1e-6)
+    # routed scaling factor scales the weights linearly
+    r4 = oracle.router(wl.with_(rsf=5.0), x, Wr, bias)
+    assert np.array_equal(r3["idx"], r4["idx"])
+    assert np.allclose(r4["w"], 2 * r3["w"], rtol=1e-6)
+
+
+def test_router_tie_flags():
+    # two candidates whose sc differ by 5e-6 straddle the k-th place
+    wl, r = _router_case(4, 1, 1, 1, 1.0, [0.6, 0.6, 0.1, 0.2], [0, 5e-6, 0, 0])
+    assert r["ties"][0] & 1
+    wl, r = _router_case(4, 1, 1, 1, 1.0, [0.6, 0.5, 0.1, 0.2], [0, 0, 0, 0])
+    assert r["ties"][0] == 0
+    # two groups whose scores differ by less than 1e-5
+    wl, r = _router_case(4, 2, 1, 1, 1.0, [0.6, 0.4, 0.5, 0.5], [0, 0, 0, 2e-6])
+    assert r["ties"][0] & 2
+
+
+def test_router_bf16_input():
+    E, H, T = 16, 64, 4
+    xb = synth.normal_bf16(41, 0, T * H).reshape(T, H)
+    Wr = synth.normal_f32(42, 0, E * H, 0, 0.3).reshape(E, H)
+    wl = W.TINY.with_(hidden=H, afmt=W.A_BF16, T=T)
+    r = oracle.router(wl, xb, Wr, np.zeros(E, np.float32))
+    xf = synth.bf16_bits_to_f32(xb)
+    r2 = oracle.router(wl.with_(afmt=W.A_F32), xf, Wr, np.zeros(E, np.float32))
+    assert np.array_equal(r["logits"], r2["logits"]) and np.array_equal(r["idx"], r2["idx"])
+
+
+# --------------------------------------------------------------------------- permutation
+def test_permute_fixture():
+    rows = {r[0]: r[1] for r in read_golden("permute_tiny.txt")}
+    E, k = int(rows["E"]), int(rows["k"])
+    idx = np.array(ints(rows["idx"]), np.int32).reshape(-1, k)
+    p = oracle.permute(idx, E)
+    for key in ("counts", "offsets", "sorted", "inv"):
+        assert p[key].tolist() == ints(rows[key]), key
+    assert p["union_ids"].tolist() == ints(rows["union"])
+
+
+def test_permute_against_numpy():
+    rng = np.random.default_rng(5)
+    for T, k, E in [(1, 8, 256), (37, 4, 16), (512, 8, 256), (64, 2, 3)]:
+        idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
+        p = oracle.permute(idx, E)
+        flat = idx.ravel()
+        assert np.array_equal(p["counts"], np.bincount(flat, minlength=E))
+        assert p["counts"].sum() == T * k
+        assert np.array_equal(p["sorted"], np.argsort(flat, kind="stable"))
+        assert np.array_equal(p["inv"][p["sorted"]], np.arange(T * k))
+        assert np.array_equal(p["union_ids"], np.unique(flat))
+        assert np.array_equal(p["offsets"], np.concatenate([[0], np.cumsum(p["counts"])]))
+
+
+# --------------------------------------------------------------------------- FFN
+def _tiny_layer(bits=4, afmt=W.A_F32, T=6, H=64, I=32, E=8, k=2):
+    wl = W.TINY.with_(hidden=H, inter=I, n_experts=E, n_group=2, topk_group=1, top_k=k, T=T,
+                      wbits=bits, afmt=afmt)
+    ex = {}
+    for e in range(E + 1):
+        g = synth.normal_f32(51, W.stream(W.K_GATE, e), I * H, 0, 0.02).reshape(I, H)
+        u = synth.normal_f32(51, W.stream(W.K_UP, e), I * H, 0, 0.02).reshape(I, H)
+        d = synth.normal_f32(51, W.stream(W.K_DOWN, e), H * I, 0, 0.02).reshape(H, I)
+        ex[e] = oracle.quantize_expert(g, u, d, bits)
+    shared = ex.pop(E)
+    if afmt == W.A_BF16:
+        x = synth.normal_bf16(52, 0, T * H).reshape(T, H)
+    else:
+        x = synth.normal_f32(52, 0, T * H).reshape(T, H)
+    Wr = synth.normal_f32(53, 0, E * H, 0, 0.1).reshape(E, H)
+    bias = synth.normal_f32(54, 0, E, 0, 0.1)
+    return wl, ex, shared, x, Wr, bias
+
+
+def _deq(q, s, K, bits):
+    return np_codes(q, K, bits).astype(np.float64) * s.astype(np.float64)[:, None]
+
+
+def _np_bf16(v):
+    torch = pytest.importorskip("torch")
+    import torch as T_
+    b = T_.from_numpy(np.ascontiguousarray(v, np.float32)).to(T_.bfloat16).to(T_.float32)
+    return b.numpy().astype(np.float64)
+
+
+def _dense_ffn(wl, ex, xrow):
+    """Independent f64 dense dequantised reference of one token through one expert,
+    with the f32 roundings the definition states (g, u, h stored as f32)."""
+    H, I, bits = wl.hidden, wl.inter, wl.wbits
+    Wg, Wu, Wd = _deq(ex.gate_q, ex.gate_s, H, bits), _deq(ex.up_q, ex.up_s, H, bits), \
+        _deq(ex.down_q, ex.down_s, I, bits)
+    if wl.afmt == W.A_Q8:
+        xq, xd = oracle.quantize_q8(xrow.astype(np.float32))
+        xv = (xq.astype(np.float64).reshape(-1, 32) * xd.astype(np.float64)[:, None]).ravel()
+    elif wl.afmt == W.A_BF16:
+        xv = synth.bf16_bits_to_f32(xrow).astype(np.float64)
+    else:
+        xv = xrow.astype(np.float64)
+    g = (Wg @ xv).astype(np.float32).astype(np.float64)
+    u = (Wu @ xv).astype(np.float32).astype(np.float64)
+    h = (g / (1 + np.exp(-g)) * u).astype(np.float32)
+    if wl.afmt == W.A_Q8:
+        hq, hd = oracle.quantize_q8(h)
+        hv = (hq.astype(np.float64).reshape(-1, 32) * hd.astype(np.float64)[:, None]).ravel()
+    elif wl.afmt == W.A_BF16:
+        hv = _np_bf16(h)
+    else:
+        hv = h.astype(np.float64)
+    y = (Wd @ hv).astype(np.float32)
+    return h, y
+
+
+@pytest.mark.parametrize("bits,afmt", [(4, W.A_F32), (8, W.A_F32), (2, W.A_F32), (4, W.A_Q8),
+                                       (2, W.A_Q8), (8, W.A_Q8), (4, W.A_BF16)])
+def test_ffn_against_dense_f64(bits, afmt):
+    wl, ex, shared, x, Wr, bias = _tiny_layer(bits, afmt)
+    for t in range(wl.T):
+        for e in (0, 3):
+            h, y = oracle.ffn_token(wl, ex[e], x, t)
+            hr, yr = _dense_ffn(wl, ex[e], x[t])
+            assert np.allclose(h, hr, rtol=2.5e-7, atol=1e-30)
+            assert np.allclose(y, yr, rtol=2.5e-7, atol=1e-9 * np.abs(yr).max())
+
+
+def test_ffn_zero_cases():
+    wl, ex, shared, x, Wr, bias = _tiny_layer()
+    h, y = oracle.ffn_token(wl, ex[0], np.zeros_like(x), 0)
+    assert not h.any() and not y.any()
+    z = oracle.Expert(np.zeros_like(ex[0].gate_q), ex[0].gate_s, ex[0].up_q, ex[0].up_s,
+                      ex[0].down_q, ex[0].down_s)
+    h, y = oracle.ffn_token(wl, z, x, 0)
+    assert not h.any() and not y.any()
+
+
+@pytest.mark.parametrize("afmt", [W.A_F32, W.A_Q8, W.A_BF16])
+def test_union_equals_per_token(afmt):
+    wl, ex, shared, x, Wr, bias = _tiny_layer(afmt=afmt, T=9)
+    r = oracle.router(wl, x, Wr, bias)
+    p = oracle.permute(r["idx"], wl.n_experts)
+    h_u, y_u = oracle.expert_ffn(wl, ex, p, x)
+    y_t = oracle.expert_ffn_per_token(wl, ex, r["idx"], p, x)
+    assert np.array_equal(y_u, y_t)
+    y_d = oracle.expert_down(wl, ex, p, h_u)
+    assert np.array_equal(y_d, y_u)
+
+
+def test_combine_and_layer():
+    wl, ex, shared, x, Wr, bias = _tiny_layer(T=7)
+    idx, wt, out = oracle.moe_forward(wl, x, Wr, bias, ex, shared)
+    r = oracle.router(wl, x, Wr, bias)
+    assert np.array_equal(idx, r["idx"]) and np.array_equal(wt, r["w"])
+    p = oracle.permute(idx, wl.n_experts)
+    _, ys = oracle.expert_ffn(wl, ex, p, x)
+    _, ysh = oracle.shared_ffn(wl, shared, x)
+    # combine against numpy f64
+    ref = ysh.astype(np.float64).copy()
+    for t in range(wl.T):
+        for j in range(wl.top_k):
+            ref[t] += float(wt[t, j]) * ys[p["inv"][t * wl.top_k + j]].astype(np.float64)
+    assert np.allclose(out, ref.astype(np.float32), rtol=2.5e-7, atol=1e-12)
+    # layer through per-token dense references
+    for t in range(wl.T):
+        acc = _dense_ffn(wl, shared, x[t])[1].astype(np.float64)
+        for j in range(wl.top_k):
+            acc += float(wt[t, j]) * _dense_ffn(wl, ex[idx[t, j]], x[t])[1].astype(np.float64)
+        assert np.allclose(out[t], acc, rtol=1e-6, atol=1e-7 * np.abs(acc).max())
+    # doubling rsf doubles the routed part exactly up to rounding
+    _, wt2, out2 = oracle.moe_forward(wl.with_(rsf=2 * wl.rsf), x, Wr, bias, ex, shared)
+    assert np.allclose(out2 - ysh, 2 * (out - ysh), rtol=1e-5, atol=1e-6 * np.abs(out).max())
+    # x = 0: every expert output is 0, so the layer output is 0
+    _, _, out0 = oracle.moe_forward(wl, np.zeros_like(x), Wr, bias, ex, shared)
+    assert not out0.any()
