@@ -1,0 +1,379 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-MoE layer forward on B200.
+
+Default workload: the GLM-5.2-shaped MoE layer (hidden 6144, 256 routed experts
+plus one shared expert, intermediate 2048, sigmoid group-limited top-8 router),
+one decode token per step, packed int4 experts with per-row f32 scales, f32
+activations.  A step is one full layer forward (route, permute, gate/up +
+SwiGLU, down, combine) through the C ABI on one batch of synthetic input that
+is already resident in HBM.  Inputs rotate through distinct token batches and
+L2 is flushed between steps outside the timed events.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl qrx|reference]
+
+--impl reference times the CPU oracle (the plain reference implementation) on
+the host cores on the same workload.  N > 1: one process per GPU under
+torchrun, each an independent replica (the layer does not shard), value =
+tokens of all ranks / max over ranks of the per-step time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed-MoE layer tokens/s; int4 expert-weight GB/s vs HBM peak"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["qrx", "reference"], default="qrx")
+    ap.add_argument("--workload", default="glm_decode_t1_int4_f32")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="budget of the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    """Hash of the GEMV kernel source: traffic figures apply only to this version."""
+    h = hashlib.sha256()
+    for f in ("k_ffn_gemv.cuh", "qrx_dev.cuh"):
+        with open(os.path.join(ROOT, "quantized_routed_expert_tc_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    rec = d.get(kernel, {}).get(workload)
+    if not rec or rec.get("source_sha") != kernel_source_hash():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                p = [v.strip() for v in line.split(",")]
+                if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                    rows.append(p)
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, wl):
+    """The CPU oracle on the host cores: one decode token per step."""
+    import numpy as np
+    import oracle
+    from quantized_routed_expert_tc_b200.layer import activations, expert_f32, router_weights
+
+    Wr, bias = router_weights(wl)
+    npool = min(max(args.steps, 1), 4)
+    xs = [activations(wl, batch=b) for b in range(npool)]
+    needed = set()
+    for x in xs:
+        r = oracle.router(wl, x, Wr, bias)
+        needed.update(int(e) for e in np.unique(r["idx"]))
+    experts = {e: oracle.quantize_expert(*expert_f32(wl, e), wl.wbits) for e in sorted(needed)}
+    shared = oracle.quantize_expert(*expert_f32(wl, wl.n_experts), wl.wbits)
+    for i in range(args.warmup if args.warmup < 2 else 1):
+        oracle.moe_forward(wl, xs[i % npool], Wr, bias, experts, shared)
+    times = []
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.moe_forward(wl, xs[i % npool], Wr, bias, experts, shared)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = wl.T / (ms / 1e3)
+    cores = oracle.max_threads()
+    sample = f"{npool} distinct {wl.T}-token batches cycled over {args.steps} steps"
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": workload_config(wl),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }))
+
+
+def workload_config(wl):
+    from quantized_routed_expert_tc_b200 import workloads as W
+    return {"workload": wl.name, "tokens_per_step": wl.T, "hidden": wl.hidden,
+            "routed_experts": wl.n_experts, "shared_experts": 1, "inter": wl.inter,
+            "top_k": wl.top_k, "n_group": wl.n_group, "topk_group": wl.topk_group,
+            "weights": f"int{wl.wbits} per-row f32 scale",
+            "activations": W.AFMT_NAMES[wl.afmt], "parallelism": "replicas",
+            "l2": "flushed between steps (256 MiB write outside the timed events); "
+                  "inputs rotate over distinct token batches"}
+
+
+# ----------------------------------------------------------------------------- CPU baseline
+def cpu_baseline(wl, seconds: float):
+    import numpy as np
+    import oracle
+    from quantized_routed_expert_tc_b200.layer import activations, expert_f32, router_weights
+
+    Wr, bias = router_weights(wl)
+    xs = [activations(wl, batch=1000 + b) for b in range(2)]
+    needed = set()
+    for x in xs:
+        needed.update(int(e) for e in np.unique(oracle.router(wl, x, Wr, bias)["idx"]))
+    experts = {e: oracle.quantize_expert(*expert_f32(wl, e), wl.wbits) for e in sorted(needed)}
+    shared = oracle.quantize_expert(*expert_f32(wl, wl.n_experts), wl.wbits)
+    n, t_total = 0, 0.0
+    while t_total < seconds or n < 2:
+        t0 = time.perf_counter()
+        oracle.moe_forward(wl, xs[n % 2], Wr, bias, experts, shared)
+        t_total += time.perf_counter() - t0
+        n += 1
+        if n >= 200:
+            break
+    return {"value": n * wl.T / t_total, "unit": "tokens/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"{n} layer forwards of {wl.T} token(s) over 2 distinct batches "
+                      f"({t_total:.1f} s of CPU time)"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_qrx(args, wl, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from quantized_routed_expert_tc_b200 import build as qbuild, qrx
+    from quantized_routed_expert_tc_b200.layer import GpuLayer, activations, to_device_act
+
+    qbuild.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    glay = GpuLayer(wl, device=dev)
+    cfg = qrx.cfg_of(wl)
+    T, H, k = wl.T, wl.hidden, wl.top_k
+    npool = 16
+    xs_np = [activations(wl, batch=rank * 1000 + b) for b in range(npool)]
+    xs = [to_device_act(wl, x, dev) for x in xs_np]
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    ws = qrx.workspace(cfg, T, dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB > L2
+    stream = torch.cuda.current_stream(dev)
+
+    # union size per pool batch (for the algorithmic bytes of each step)
+    unions = []
+    for x in xs:
+        qrx.qrx_moe_forward(cfg, x, glay.Wr, glay.bias, glay.routed[wl.wbits],
+                            glay.shared[wl.wbits], idx, w, out, ws)
+        unions.append(int(torch.unique(idx).numel()))
+    torch.cuda.synchronize(dev)
+    rc = qrx.qrx_last_error()
+    if rc != qrx.QRX_OK:
+        raise RuntimeError(f"device error before timing: {qrx.qrx_strerror(rc)}")
+
+    def step(i, evs):
+        flush.zero_()
+        qrx.qrx_moe_forward_profiled(cfg, xs[i % npool], glay.Wr, glay.bias,
+                                     glay.routed[wl.wbits], glay.shared[wl.wbits], idx, w, out,
+                                     ws, evs, stream)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    warm_evs = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+    for i in range(args.warmup):
+        step(i, warm_evs)
+    t_settle = time.perf_counter()
+    i = 0
+    while time.perf_counter() - t_settle < 1.0:          # clocks settle under load
+        step(i, warm_evs)
+        i += 1
+        if i % 64 == 0:
+            torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        step(i, evs[i])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(6)]
+                    for i in range(args.steps)])          # ms per stage per step
+    total = per.sum(axis=1)
+    ms_step = float(total.mean())
+    if world > 1:
+        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    rc = qrx.qrx_last_error()
+    if rc != qrx.QRX_OK:
+        raise RuntimeError(f"device error during timing: {qrx.qrx_strerror(rc)}")
+
+    # algorithmic bytes: each union expert and the shared expert read once
+    nu = np.array([unions[i % npool] for i in range(args.steps)], dtype=np.float64)
+    exp_bytes = wl.expert_bytes()
+    I, b = wl.inter, wl.wbits
+    gateup_bytes = (nu + 1) * (2 * I * (H * b // 8 + 4))
+    layer_bytes = (nu + 1) * exp_bytes
+    gu_ms = per[:, 3]
+    achieved = float((gateup_bytes / (gu_ms / 1e3)).mean() / 1e9)
+    peak, peak_kind = peaks()
+    weight_gbs = float((layer_bytes.mean()) / (ms_step / 1e3) / 1e9)
+    traffic = recorded_traffic("k_ffn_gemv_gateup", wl.name)
+
+    e2e = None
+    if not args.no_e2e:
+        xh = [torch.from_numpy(x).pin_memory() if wl.afmt != 2 else
+              torch.from_numpy(x.view(np.int16)).pin_memory() for x in xs_np]
+        oh = torch.empty((T, H), dtype=torch.float32).pin_memory()
+        es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for i in range(min(args.warmup, 3)):
+            qrx.qrx_moe_forward_hostio(cfg, xh[i % npool], glay.Wr, glay.bias,
+                                       glay.routed[wl.wbits], glay.shared[wl.wbits], oh, ws, stream)
+        for i in range(args.steps):
+            flush.zero_()
+            es[i][0].record(stream)
+            qrx.qrx_moe_forward_hostio(cfg, xh[i % npool], glay.Wr, glay.bias,
+                                       glay.routed[wl.wbits], glay.shared[wl.wbits], oh, ws, stream)
+            es[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = float(np.mean([a.elapsed_time(z) for a, z in es]))
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        xbytes = T * H * (2 if wl.afmt == 2 else 4)
+        e2e = {"value": T * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": xbytes,
+               "d2h_bytes_per_step": T * H * 4, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_seconds)
+
+    if rank == 0:
+        stages = ["router", "permute", "act_quant", "gateup", "down", "combine"]
+        launches_per_step = 6 + (1 if wl.afmt == 1 else 0)
+        line = {
+            "metric": METRIC, "value": T * world / (ms_step / 1e3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int32",
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights quantised by the "
+                    "library; no trained weights)",
+            "config": workload_config(wl),
+            "weight_gbs": weight_gbs,
+            "weight_gbs_frac_of_measured_hbm": weight_gbs / peak,
+            "weight_gbs_frac_of_8tbs": weight_gbs / SPEC_HBM_GBS,
+            "n_union_mean": float(nu.mean()),
+            "stage_us": {s: float(per[:, j].mean() * 1e3) for j, s in enumerate(stages)},
+            "roofline": {"kernel": "k_ffn_gemv (gate/up + SwiGLU)", "bound": "hbm",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "traffic": traffic,
+                         "algorithmic_bytes_per_launch": float(gateup_bytes.mean())},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line))
+
+
+def main():
+    args = parse()
+    from quantized_routed_expert_tc_b200 import workloads as W
+    wl = W.ALL[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, wl)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_qrx(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

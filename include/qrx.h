@@ -1,0 +1,244 @@
+/*
+ * qrx.h -- C ABI of libqrx: the routed-MoE layer forward over packed low-bit
+ * expert weights, on one NVIDIA B200 (sm_100a).
+ *
+ * The operation is the MoE layer of GLM-5.2 as the colibri pages describe it:
+ *   - colibri README ("JustVugg/colibri"), section "已实现的功能" (implemented
+ *     features): DeepSeek-V3-like sigmoid router (noaux_tc,
+ *     routed_scaling_factor), a shared expert, Q8_0-style int8-activation
+ *     integer dot kernels, int8 / packed int4 / packed int2 weights with
+ *     per-row scales dequantised on use, and the batch-union MoE (each unique
+ *     expert of a batch read once, applied to every position routed to it);
+ *   - blog "GLM-5.2 on slow computers", section "让它变得可以忍受的那些装置":
+ *     the same expert in a batch is read only once; int4 container with
+ *     per-row scale, dequant-on-use.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller (for
+ *     example torch tensors' data_ptr()), except where a call says "host".
+ *     The library never frees or keeps them.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on that stream and never synchronise
+ *     the host, except qrx_last_error, qrx_moe_forward_hostio and the
+ *     query functions.
+ *   - Argument checks are synchronous and happen before any launch; a
+ *     failing check returns a negative QRX_E* code and launches nothing.
+ *   - Kernels that detect a bad value at run time (an expert index out of
+ *     range, an exhausted bounded wait) set a sticky device flag;
+ *     qrx_last_error() synchronises the device and reports it.
+ *   - Calls are not thread-safe with respect to the same workspace.
+ *
+ * Tensor layouts (row-major, C order):
+ *   x        [T][H]      f32 (QRX_A_F32, QRX_A_Q8_0) or bf16 (QRX_A_BF16)
+ *   W_router [E][H]      f32;  bias [E] f32 (score-correction bias)
+ *   topk_idx [T][k]      int32; topk_w [T][k] f32
+ *   Expert weights, `n` experts back to back (n = E routed, 1 shared):
+ *     w13 [n][2I][H*b/8] uint8: row 2i is gate row i, row 2i+1 is up row i
+ *     s13 [n][2I]        f32 row scales of w13
+ *     w2  [n][H][I*b/8]  uint8: down projection rows
+ *     s2  [n][H]         f32 row scales of w2
+ *     (b = 8, 4 or 2 bits; packed fields as in the README: int4 low nibble
+ *     first, int2 lowest bit pair first, two's-complement codes.)
+ *   Assignment a = t*k + j.  Sorted order groups assignments by expert,
+ *   stable in a; position p indexes that order; h and y rows are positions.
+ */
+#ifndef QRX_H
+#define QRX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define QRX_OK 0
+#define QRX_EINVAL (-1)        /* NULL pointer, bad size, T <= 0, ... */
+#define QRX_EUNSUPPORTED (-2)  /* configuration outside what the kernels handle */
+#define QRX_ECUDA (-3)         /* a CUDA runtime call failed */
+#define QRX_ETIMEOUT (-4)      /* a bounded device wait gave up */
+#define QRX_EDEVICE (-5)       /* a kernel saw an invalid value (sticky flag) */
+#define QRX_ENOSPACE (-6)      /* workspace smaller than qrx_workspace_bytes */
+
+typedef enum { QRX_W_INT8 = 8, QRX_W_INT4 = 4, QRX_W_INT2 = 2 } qrx_wfmt;
+typedef enum { QRX_A_F32 = 0, QRX_A_Q8_0 = 1, QRX_A_BF16 = 2 } qrx_afmt;
+
+/* Layer configuration (the README's router knobs plus sizes and formats). */
+typedef struct {
+    int32_t hidden;                /* H */
+    int32_t n_experts;             /* E routed experts */
+    int32_t inter;                 /* I expert intermediate size */
+    int32_t n_group;               /* G expert groups (contiguous, E/G each) */
+    int32_t topk_group;            /* Gk groups kept per token */
+    int32_t top_k;                 /* k experts per token */
+    float routed_scaling_factor;   /* rsf */
+    int32_t wfmt;                  /* qrx_wfmt of routed and shared experts */
+    int32_t afmt;                  /* qrx_afmt of the activations */
+} qrx_cfg;
+
+/* Packed experts (see layout above).  All device pointers. */
+typedef struct {
+    const uint8_t *w13;
+    const float *s13;
+    const uint8_t *w2;
+    const float *s2;
+} qrx_experts;
+
+/* Batch-union permutation buffers (device, int32):
+ *   counts[E], offsets[E+1], sorted[T*k] (value a), inv[T*k] (value p),
+ *   union_ids[E] (first *n_union valid, ascending), n_union[1]. */
+typedef struct {
+    int32_t *counts;
+    int32_t *offsets;
+    int32_t *sorted;
+    int32_t *inv;
+    int32_t *union_ids;
+    int32_t *n_union;
+} qrx_perm;
+
+/* Activations handed to the expert FFN.
+ *   QRX_A_F32:  x = f32 [T][H];        xq, xd unused.
+ *   QRX_A_BF16: x = bf16 [T][H];       xq, xd unused.
+ *   QRX_A_Q8_0: xq = int8 [T][H] and xd = f32 [T][H/32] from
+ *               qrx_quantize_act_q8;   x unused. */
+typedef struct {
+    const void *x;
+    const int8_t *xq;
+    const float *xd;
+} qrx_act;
+
+/* ---- queries (host only, synchronous) ---------------------------------- */
+
+/* Check a configuration.  QRX_EINVAL for non-positive sizes or a bad enum;
+ * QRX_EUNSUPPORTED when: E % G != 0, Gk > G, Gk*E/G < k, k > 32, E > 1024,
+ * H or I not a multiple of 64, or a row of H or I codes is not a supported
+ * number of 16-byte chunks (1, 2, 4, 8, 16, 32, 64, 96, 128, 192 or 384). */
+int qrx_validate(const qrx_cfg *cfg);
+
+/* Bytes of scratch the calls below need for T tokens (a multiple of 256). */
+size_t qrx_workspace_bytes(const qrx_cfg *cfg, int32_t T);
+
+/* Sticky device status: synchronises the current device, returns QRX_OK,
+ * QRX_EDEVICE or QRX_ETIMEOUT (and clears the flag), or QRX_ECUDA if the
+ * context reported an error. */
+int qrx_last_error(void);
+const char *qrx_strerror(int code);
+
+/* ---- quantisation ------------------------------------------------------ */
+
+/* Per-row symmetric quantisation of f32 rows into packed codes
+ * (README "已实现的功能": per-row scale; tiny-layer workload: scale =
+ * absmax/7 for int4, codes in [-8, 7], two per byte low nibble first).
+ * scale_r = absmax_r / qmax (qmax = 127, 7, 1 for 8, 4, 2 bits), one f32
+ * division; code = clamp(round-half-away(w / scale_r), qmin, qmax); a zero
+ * row gets scale 0 and codes 0.
+ *   w      [rows][K] f32 (device)
+ *   q      output: row r at q + r*ldq bytes, K*wbits/8 bytes per row
+ *   scale  output: scale of row r at scale[r*lds]
+ * K must be a multiple of 32.  Bit-exact with the CPU reference. */
+int qrx_quantize_weights(const float *w, int64_t rows, int64_t K, int32_t wbits,
+                         uint8_t *q, int64_t ldq, float *scale, int64_t lds, void *stream);
+
+/* Q8_0-style activations (README "已实现的功能": integer dot with Q8_0-style
+ * int8 activations; blocks of 32 with an f32 absmax scale):
+ * d = amax/127, q = clamp(round-half-away(x * (127/amax)), -127, 127), a zero
+ * block gives d = 0, q = 0.  x [T][H] f32 -> xq [T][H] int8, xd [T][H/32] f32.
+ * H must be a multiple of 32.  Bit-exact with the CPU reference. */
+int qrx_quantize_act_q8(const float *x, int64_t T, int64_t H, int8_t *xq, float *xd,
+                        void *stream);
+
+/* Exact int32 block accumulators acc[r][b] = sum over the 32-element block b
+ * of code(r, i) * xq[i], through the same unpack and dp4a path as the FFN
+ * kernels (the integer part of a Q8_0 dot; compared bit for bit in tests).
+ *   q [rows][K*wbits/8], xq [K] int8, acc [rows][K/32] int32. */
+int qrx_block_dots_q8(int32_t wbits, const uint8_t *q, int64_t rows, int64_t K,
+                      const int8_t *xq, int32_t *acc, void *stream);
+
+/* ---- the layer, step by step ------------------------------------------ */
+
+/* Router (README "已实现的功能": DeepSeek-V3-like sigmoid router, noaux_tc,
+ * routed_scaling_factor): logit = x . W_router[e] (f64 accumulation, rounded
+ * to f32), s = sigmoid(logit), sc = s + bias (selection only); groups of E/G
+ * contiguous experts scored by the sum of their two largest sc; the Gk best
+ * groups kept (ties to the lower group); the k largest sc among their
+ * experts (ties to the lower id) in descending order; weights
+ * w_j = s_j / sum(s) * rsf.  x per cfg->afmt (f32 for F32 and Q8_0, bf16 for
+ * BF16).  ws: at least qrx_workspace_bytes(cfg, T) bytes. */
+int qrx_route(const qrx_cfg *cfg, const void *x, int32_t T, const float *W_router,
+              const float *bias, int32_t *topk_idx, float *topk_w, void *ws,
+              size_t ws_bytes, void *stream);
+
+/* Batch-union permutation (README "已实现的功能": batch-union MoE; blog:
+ * same expert read once per batch): a stable counting sort of the T*k
+ * assignments by expert.  Deterministic.  Sets the device error flag if an
+ * index is outside [0, E). */
+int qrx_permute(const qrx_cfg *cfg, const int32_t *topk_idx, int32_t T,
+                const qrx_perm *perm, void *stream);
+
+/* Routed experts' SwiGLU FFN over the batch union: for each expert of the
+ * union, its gate/up rows are read once for all of its positions:
+ * h = silu(s_g (Q_g x)) * (s_u (Q_u x)), then y = s_d (Q_d h') where h' is h
+ * (F32), h rounded to bf16 (BF16) or h re-quantised to Q8_0 (Q8_0).
+ *   h_sorted: [T*k][I] f32 output (may be NULL: workspace is used)
+ *   y_sorted: [T*k][H] f32 output, rows in sorted order. */
+int qrx_expert_ffn(const qrx_cfg *cfg, const qrx_experts *routed, const qrx_perm *perm,
+                   const qrx_act *act, int32_t T, float *h_sorted, float *y_sorted,
+                   void *ws, size_t ws_bytes, void *stream);
+
+/* Down projection alone, from a given h_sorted [T*k][I] f32 (stage
+ * isolation: lets a test feed the reference's h). */
+int qrx_expert_down(const qrx_cfg *cfg, const qrx_experts *routed, const qrx_perm *perm,
+                    const float *h_sorted, int32_t T, float *y_sorted, void *ws,
+                    size_t ws_bytes, void *stream);
+
+/* Shared expert (README "已实现的功能"): the same FFN on every token, weight
+ * 1, ungated.  h_sh [T][I] (may be NULL), y_sh [T][H] f32. */
+int qrx_shared_ffn(const qrx_cfg *cfg, const qrx_experts *shared, const qrx_act *act,
+                   int32_t T, float *h_sh, float *y_sh, void *ws, size_t ws_bytes,
+                   void *stream);
+
+/* Weighted combine: out[t] = y_sh[t] + sum_j topk_w[t][j] * y_sorted[inv[t*k+j]]
+ * in fixed j order.  y_sh may be NULL (no shared term).  out [T][H] f32. */
+int qrx_combine(const qrx_cfg *cfg, const float *y_sorted, const float *y_sh,
+                const float *topk_w, const int32_t *inv, int32_t T, float *out,
+                void *stream);
+
+/* ---- the whole layer --------------------------------------------------- */
+
+/* route -> permute -> (Q8_0 quantise) -> routed + shared FFN -> combine, all
+ * on `stream` with no host synchronisation (capturable in a CUDA graph).
+ * shared may be NULL.  topk_idx, topk_w: outputs [T][k].  out [T][H] f32. */
+int qrx_moe_forward(const qrx_cfg *cfg, const void *x, int32_t T, const float *W_router,
+                    const float *bias, const qrx_experts *routed, const qrx_experts *shared,
+                    int32_t *topk_idx, float *topk_w, float *out, void *ws,
+                    size_t ws_bytes, void *stream);
+
+/* qrx_moe_forward with stage timing: events[0..6] are cudaEvent_t handles
+ * (passed as void*) recorded on `stream` before the router, after the
+ * router, after the permutation, after the Q8_0 activation quantiser (right
+ * after the permutation when there is none), after the gate/up kernel, after
+ * the down kernel and after the combine.  n_events must be 7.  Everything
+ * else is as qrx_moe_forward. */
+int qrx_moe_forward_profiled(const qrx_cfg *cfg, const void *x, int32_t T,
+                             const float *W_router, const float *bias,
+                             const qrx_experts *routed, const qrx_experts *shared,
+                             int32_t *topk_idx, float *topk_w, float *out, void *ws,
+                             size_t ws_bytes, void *const *events, int32_t n_events,
+                             void *stream);
+
+/* The same layer with HOST input and output: copies x_host (pinned or
+ * pageable, T*H elements of the activation type) to the device, runs
+ * qrx_moe_forward and copies the result to out_host [T][H] f32, then
+ * synchronises `stream`.  ws must also hold the device copies:
+ * qrx_workspace_bytes(cfg, T) covers them. */
+int qrx_moe_forward_hostio(const qrx_cfg *cfg, const void *x_host, int32_t T,
+                           const float *W_router, const float *bias,
+                           const qrx_experts *routed, const qrx_experts *shared,
+                           float *out_host, void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QRX_H */

@@ -1,0 +1,70 @@
+// qrx_internal.h -- launchers shared between the qrx .cu files (not public).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/qrx.h"
+
+namespace qrx {
+
+// device status flag (one per device, in k_quant.cu)
+cudaError_t read_and_clear_device_flag(int *flag);
+
+cudaError_t launch_quantize_weights(const float *w, int64_t rows, int64_t K, int wbits,
+                                    uint8_t *q, int64_t ldq, float *scale, int64_t lds,
+                                    cudaStream_t st);
+cudaError_t launch_quantize_act_q8(const float *x, int64_t nblocks, int8_t *xq, float *xd,
+                                   cudaStream_t st);
+cudaError_t launch_block_dots_q8(int wbits, const uint8_t *q, int64_t rows, int64_t K,
+                                 const int8_t *xq, int32_t *acc, cudaStream_t st);
+
+// router: partial dots then selection
+struct RouterArgs {
+    const void *x;          // f32 or bf16 [T][H]
+    int x_bf16;
+    const float *Wr;        // [E][H]
+    const float *bias;      // [E]
+    int T, H, E, G, Gk, k;
+    float rsf;
+    double *partial;        // [KS][T][E]
+    int KS;
+    int32_t *idx;           // [T][k]
+    float *w;               // [T][k]
+};
+int router_ksplit(int T, int H, int E, int num_sms);
+cudaError_t launch_router(const RouterArgs &a, cudaStream_t st);
+
+cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const qrx_perm &p,
+                           cudaStream_t st);
+
+// expert FFN over the union (GEMV-shaped kernels)
+struct FfnArgs {
+    int wbits, afmt;
+    int H, I, E, k, T;
+    // routed experts (may be null if !routed), shared expert (may be null)
+    const uint8_t *w13, *w2;
+    const float *s13, *s2;
+    const uint8_t *w13_sh, *w2_sh;
+    const float *s13_sh, *s2_sh;
+    int routed, shared;
+    const int32_t *offsets, *sorted, *union_ids, *n_union;
+    // activations
+    const void *x;          // f32 / bf16 [T][H]
+    const int8_t *xq;       // Q8 [T][H]
+    const float *xd;        // Q8 [T][H/32]
+    // positions: routed p in [0, T*k), shared p = T*k + t
+    float *h;               // [P][I] intermediate (gate/up output, down input)
+    float *y;               // [P][H]
+    int64_t h_ld, y_ld;     // row strides (elements)
+    // where the shared expert's rows live: h + sh_h_off*h_ld, y + sh_y_off*y_ld
+    int64_t sh_h_row0, sh_y_row0;
+};
+cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st);
+cudaError_t launch_ffn_down(const FfnArgs &a, int num_sms, cudaStream_t st);
+
+cudaError_t launch_combine(const float *y_sorted, const float *y_sh, const float *w,
+                           const int32_t *inv, int T, int k, int H, float *out,
+                           cudaStream_t st);
+
+}  // namespace qrx

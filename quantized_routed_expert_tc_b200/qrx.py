@@ -1,0 +1,302 @@
+"""Thin Python binding of libqrx (include/qrx.h): argument marshalling only.
+
+Every function named ``qrx_*`` here calls the C entry point of the same name
+with the tensors' device pointers and the current torch CUDA stream.  Every
+step of the layer runs in the library's CUDA kernels; there is no Python or
+CPU fallback: if libqrx.so is missing or a call fails, a QrxError is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+
+import torch
+
+from . import build as _build
+
+QRX_OK, QRX_EINVAL, QRX_EUNSUPPORTED, QRX_ECUDA, QRX_ETIMEOUT, QRX_EDEVICE, QRX_ENOSPACE = \
+    0, -1, -2, -3, -4, -5, -6
+W_INT8, W_INT4, W_INT2 = 8, 4, 2
+A_F32, A_Q8_0, A_BF16 = 0, 1, 2
+
+HEADER = os.path.join(os.path.dirname(_build.HERE), "include", "qrx.h")
+
+
+class QrxError(RuntimeError):
+    def __init__(self, name: str, code: int, detail: str | None = None):
+        self.code = code
+        super().__init__(f"{name}: {detail or qrx_strerror(code)} ({code})")
+
+
+class Cfg(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+                ("inter", ctypes.c_int32), ("n_group", ctypes.c_int32),
+                ("topk_group", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_float), ("wfmt", ctypes.c_int32),
+                ("afmt", ctypes.c_int32)]
+
+
+class CExperts(ctypes.Structure):
+    _fields_ = [("w13", ctypes.c_void_p), ("s13", ctypes.c_void_p), ("w2", ctypes.c_void_p),
+                ("s2", ctypes.c_void_p)]
+
+
+class CPerm(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("counts", "offsets", "sorted", "inv", "union_ids", "n_union")]
+
+
+class CAct(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("xq", ctypes.c_void_p), ("xd", ctypes.c_void_p)]
+
+
+_lib = None
+vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+P = ctypes.POINTER
+
+_SIGS = {
+    "qrx_validate": ([P(Cfg)], ctypes.c_int),
+    "qrx_workspace_bytes": ([P(Cfg), i32], sz),
+    "qrx_last_error": ([], ctypes.c_int),
+    "qrx_strerror": ([ctypes.c_int], ctypes.c_char_p),
+    "qrx_quantize_weights": ([vp, i64, i64, i32, vp, i64, vp, i64, vp], ctypes.c_int),
+    "qrx_quantize_act_q8": ([vp, i64, i64, vp, vp, vp], ctypes.c_int),
+    "qrx_block_dots_q8": ([i32, vp, i64, i64, vp, vp, vp], ctypes.c_int),
+    "qrx_route": ([P(Cfg), vp, i32, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+    "qrx_permute": ([P(Cfg), vp, i32, P(CPerm), vp], ctypes.c_int),
+    "qrx_expert_ffn": ([P(Cfg), P(CExperts), P(CPerm), P(CAct), i32, vp, vp, vp, sz, vp],
+                       ctypes.c_int),
+    "qrx_expert_down": ([P(Cfg), P(CExperts), P(CPerm), vp, i32, vp, vp, sz, vp], ctypes.c_int),
+    "qrx_shared_ffn": ([P(Cfg), P(CExperts), P(CAct), i32, vp, vp, vp, sz, vp], ctypes.c_int),
+    "qrx_combine": ([P(Cfg), vp, vp, vp, vp, i32, vp, vp], ctypes.c_int),
+    "qrx_moe_forward": ([P(Cfg), vp, i32, vp, vp, P(CExperts), P(CExperts), vp, vp, vp, vp, sz,
+                         vp], ctypes.c_int),
+    "qrx_moe_forward_hostio": ([P(Cfg), vp, i32, vp, vp, P(CExperts), P(CExperts), vp, vp, sz,
+                                vp], ctypes.c_int),
+    "qrx_moe_forward_profiled": ([P(Cfg), vp, i32, vp, vp, P(CExperts), P(CExperts), vp, vp, vp,
+                                  vp, sz, ctypes.POINTER(vp), i32, vp], ctypes.c_int),
+}
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def lib():
+    """Load libqrx.so (built in-tree by build()).  Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        path = lib_path()
+        if not os.path.exists(path):
+            raise QrxError("load", QRX_ECUDA,
+                           f"{path} is missing: build it with "
+                           "quantized_routed_expert_tc_b200.build.build()")
+        L = ctypes.CDLL(path)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def header_symbols() -> list[str]:
+    """Names of the functions include/qrx.h declares."""
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(qrx_\w+)\s*\(", txt, re.M)))
+
+
+# ------------------------------------------------------------------ marshalling helpers
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _st(stream):
+    if stream is not None:
+        return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(name: str, rc: int):
+    if rc != QRX_OK:
+        raise QrxError(name, rc)
+
+
+def cfg_of(w) -> Cfg:
+    """qrx_cfg from a workload-like object (hidden, n_experts, ..., wbits, afmt)."""
+    return Cfg(w.hidden, w.n_experts, w.inter, w.n_group, w.topk_group, w.top_k, w.rsf,
+               w.wbits, w.afmt)
+
+
+@dataclass
+class Experts:
+    """Packed experts on the device (layout of include/qrx.h)."""
+    w13: torch.Tensor    # [n, 2I, H*b/8] uint8
+    s13: torch.Tensor    # [n, 2I] f32
+    w2: torch.Tensor     # [n, H, I*b/8] uint8
+    s2: torch.Tensor     # [n, H] f32
+
+    def c(self) -> CExperts:
+        return CExperts(_p(self.w13), _p(self.s13), _p(self.w2), _p(self.s2))
+
+    @staticmethod
+    def empty(n: int, H: int, I: int, wbits: int, device="cuda") -> "Experts":
+        return Experts(torch.empty((n, 2 * I, H * wbits // 8), dtype=torch.uint8, device=device),
+                       torch.empty((n, 2 * I), dtype=torch.float32, device=device),
+                       torch.empty((n, H, I * wbits // 8), dtype=torch.uint8, device=device),
+                       torch.empty((n, H), dtype=torch.float32, device=device))
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.w13, self.s13, self.w2, self.s2))
+
+
+@dataclass
+class Perm:
+    counts: torch.Tensor
+    offsets: torch.Tensor
+    sorted: torch.Tensor
+    inv: torch.Tensor
+    union_ids: torch.Tensor
+    n_union: torch.Tensor
+
+    def c(self) -> CPerm:
+        return CPerm(*(_p(t) for t in (self.counts, self.offsets, self.sorted, self.inv,
+                                        self.union_ids, self.n_union)))
+
+    @staticmethod
+    def empty(T: int, k: int, E: int, device="cuda") -> "Perm":
+        z = lambda n: torch.empty(n, dtype=torch.int32, device=device)
+        return Perm(z(E), z(E + 1), z(T * k), z(T * k), z(E), z(1))
+
+
+def workspace(cfg: Cfg, T: int, device="cuda") -> torch.Tensor:
+    n = qrx_workspace_bytes(cfg, T)
+    if n == 0:
+        raise QrxError("qrx_workspace_bytes", QRX_EINVAL)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ C entry points
+def qrx_validate(cfg: Cfg) -> int:
+    return lib().qrx_validate(ctypes.byref(cfg))
+
+
+def qrx_workspace_bytes(cfg: Cfg, T: int) -> int:
+    return lib().qrx_workspace_bytes(ctypes.byref(cfg), T)
+
+
+def qrx_last_error() -> int:
+    return lib().qrx_last_error()
+
+
+def qrx_strerror(code: int) -> str:
+    if _lib is None and not os.path.exists(lib_path()):
+        return f"error {code}"
+    return lib().qrx_strerror(code).decode()
+
+
+def qrx_quantize_weights(w, wbits, q, ldq, scale, lds, stream=None):
+    rows, K = w.shape
+    _check("qrx_quantize_weights", lib().qrx_quantize_weights(
+        _p(w), rows, K, wbits, _p(q), ldq, _p(scale), lds, _st(stream)))
+
+
+def qrx_quantize_act_q8(x, xq, xd, stream=None):
+    T, H = x.shape
+    _check("qrx_quantize_act_q8", lib().qrx_quantize_act_q8(_p(x), T, H, _p(xq), _p(xd),
+                                                            _st(stream)))
+
+
+def qrx_block_dots_q8(wbits, q, K, xq, acc, stream=None):
+    _check("qrx_block_dots_q8", lib().qrx_block_dots_q8(wbits, _p(q), q.shape[0], K, _p(xq),
+                                                        _p(acc), _st(stream)))
+
+
+def qrx_route(cfg, x, Wr, bias, topk_idx, topk_w, ws, stream=None):
+    _check("qrx_route", lib().qrx_route(ctypes.byref(cfg), _p(x), x.shape[0], _p(Wr), _p(bias),
+                                        _p(topk_idx), _p(topk_w), _p(ws), ws.numel(), _st(stream)))
+
+
+def qrx_permute(cfg, topk_idx, perm: Perm, stream=None):
+    _check("qrx_permute", lib().qrx_permute(ctypes.byref(cfg), _p(topk_idx), topk_idx.shape[0],
+                                            ctypes.byref(perm.c()), _st(stream)))
+
+
+def _act(cfg, x=None, xq=None, xd=None) -> CAct:
+    return CAct(_p(x), _p(xq), _p(xd))
+
+
+def qrx_expert_ffn(cfg, routed: Experts, perm: Perm, T, y_sorted, ws, x=None, xq=None, xd=None,
+                   h_sorted=None, stream=None):
+    _check("qrx_expert_ffn", lib().qrx_expert_ffn(
+        ctypes.byref(cfg), ctypes.byref(routed.c()), ctypes.byref(perm.c()),
+        ctypes.byref(_act(cfg, x, xq, xd)), T, _p(h_sorted), _p(y_sorted), _p(ws), ws.numel(),
+        _st(stream)))
+
+
+def qrx_expert_down(cfg, routed: Experts, perm: Perm, h_sorted, T, y_sorted, ws, stream=None):
+    _check("qrx_expert_down", lib().qrx_expert_down(
+        ctypes.byref(cfg), ctypes.byref(routed.c()), ctypes.byref(perm.c()), _p(h_sorted), T,
+        _p(y_sorted), _p(ws), ws.numel(), _st(stream)))
+
+
+def qrx_shared_ffn(cfg, shared: Experts, T, y_sh, ws, x=None, xq=None, xd=None, h_sh=None,
+                   stream=None):
+    _check("qrx_shared_ffn", lib().qrx_shared_ffn(
+        ctypes.byref(cfg), ctypes.byref(shared.c()), ctypes.byref(_act(cfg, x, xq, xd)), T,
+        _p(h_sh), _p(y_sh), _p(ws), ws.numel(), _st(stream)))
+
+
+def qrx_combine(cfg, y_sorted, y_sh, topk_w, inv, out, stream=None):
+    _check("qrx_combine", lib().qrx_combine(ctypes.byref(cfg), _p(y_sorted), _p(y_sh),
+                                            _p(topk_w), _p(inv), topk_w.shape[0], _p(out),
+                                            _st(stream)))
+
+
+def qrx_moe_forward(cfg, x, Wr, bias, routed: Experts, shared: Experts | None, topk_idx, topk_w,
+                    out, ws, stream=None):
+    sh = ctypes.byref(shared.c()) if shared is not None else None
+    _check("qrx_moe_forward", lib().qrx_moe_forward(
+        ctypes.byref(cfg), _p(x), x.shape[0], _p(Wr), _p(bias), ctypes.byref(routed.c()), sh,
+        _p(topk_idx), _p(topk_w), _p(out), _p(ws), ws.numel(), _st(stream)))
+
+
+def qrx_moe_forward_profiled(cfg, x, Wr, bias, routed: Experts, shared: Experts | None,
+                             topk_idx, topk_w, out, ws, events, stream=None):
+    """qrx_moe_forward recording 7 torch.cuda.Event objects between its stages."""
+    sh = ctypes.byref(shared.c()) if shared is not None else None
+    arr = (vp * 7)(*[ev.cuda_event for ev in events])
+    _check("qrx_moe_forward_profiled", lib().qrx_moe_forward_profiled(
+        ctypes.byref(cfg), _p(x), x.shape[0], _p(Wr), _p(bias), ctypes.byref(routed.c()), sh,
+        _p(topk_idx), _p(topk_w), _p(out), _p(ws), ws.numel(), arr, len(events), _st(stream)))
+
+
+def qrx_moe_forward_hostio(cfg, x_host, Wr, bias, routed: Experts, shared: Experts | None,
+                           out_host, ws, stream=None):
+    sh = ctypes.byref(shared.c()) if shared is not None else None
+    _check("qrx_moe_forward_hostio", lib().qrx_moe_forward_hostio(
+        ctypes.byref(cfg), _p(x_host), x_host.shape[0], _p(Wr), _p(bias),
+        ctypes.byref(routed.c()), sh, _p(out_host), _p(ws), ws.numel(), _st(stream)))
+
+
+# ------------------------------------------------------------------ weight packing
+def quantize_expert_into(ex: Experts, e: int, gate: torch.Tensor, up: torch.Tensor,
+                         down: torch.Tensor, wbits: int, stream=None) -> None:
+    """Quantise one expert's f32 gate [I,H], up [I,H], down [H,I] (device tensors)
+    into slot e of `ex`: gate rows to the even rows of w13, up rows to the odd rows."""
+    I, H = gate.shape
+    rb13 = ex.w13.shape[2]
+    w13 = ex.w13[e]
+    s13 = ex.s13[e]
+    qrx_quantize_weights(gate, wbits, w13.data_ptr(), 2 * rb13, s13.data_ptr(), 2, stream)
+    qrx_quantize_weights(up, wbits, w13.data_ptr() + rb13, 2 * rb13, s13.data_ptr() + 4, 2, stream)
+    qrx_quantize_weights(down, wbits, ex.w2[e].data_ptr(), ex.w2.shape[2], ex.s2[e].data_ptr(), 1,
+                         stream)

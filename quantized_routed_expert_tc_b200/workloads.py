@@ -13,8 +13,13 @@ Input recipe (every array is a pure function of (seed, stream, index); see
   - router weight Wr [E][H]: f32 N(0, 0.02);
   - score-correction bias [E]: f32 N(0, bias_std);
   - activations x [T][H]: N(0, 1), f32 or bf16;
-  - seed = 1000 + workload id; batch b of a workload draws x from stream
-    (X, b), so a benchmark can rotate through distinct batches.
+  - weights and router: drawn from the layer seed -- 1000 for the tiny layer,
+    1001 for the GLM-shaped layer, which every GLM-shaped workload shares (the
+    decode, verify/prefill and format-sweep workloads all run "the same
+    GLM-shaped layer");
+  - bias and activations: drawn from the workload seed 1000 + workload id;
+    batch b of a workload draws x from stream (X, b), so a benchmark can
+    rotate through distinct batches.
 """
 from __future__ import annotations
 
@@ -50,7 +55,13 @@ class Workload:
 
     @property
     def seed(self) -> int:
+        """Seed of the bias and the activations."""
         return 1000 + self.wid
+
+    @property
+    def layer_seed(self) -> int:
+        """Seed of the expert weights and the router weight."""
+        return 1000 if self.hidden == 256 else 1001
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)

@@ -1,0 +1,375 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Rules: integer, index and byte results bit-exact (expert indices up to counted
+near-ties, where the oracle's selection is then fed to the later stages); f32
+outputs max|gpu - oracle| <= 1e-3 * max|oracle|.  Sizes span the tiny layer
+(every format and activation mode, ragged T) and the full GLM-shaped layer
+(decode, Q8_0 decode batch, verify and prefill batches, the format sweep), at
+full size on sampled tokens the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_routed_expert_tc_b200 import build as qbuild, qrx, synth, workloads as W
+from quantized_routed_expert_tc_b200.layer import (GpuLayer, activations, router_weights,
+                                                   to_device_act)
+from tests.harness import TOL, OracleLayer, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="session")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    qbuild.build()
+    torch.cuda.set_device(0)
+    assert qrx.qrx_last_error() == qrx.QRX_OK
+    return torch.device("cuda:0")
+
+
+@pytest.fixture(scope="session")
+def tiny(dev):
+    return GpuLayer(W.TINY, formats=(8, 4, 2)), OracleLayer(W.TINY)
+
+
+@pytest.fixture(scope="session")
+def glm(dev):
+    return GpuLayer(W.GLM_DECODE_T1, formats=(4, 8, 2)), OracleLayer(W.GLM_DECODE_T1)
+
+
+def cu(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def np_(t):
+    return t.detach().cpu().numpy()
+
+
+def check_routing(r, idx_gpu, w_gpu):
+    """Expert indices bit-exact except counted near-ties; weights of matching tokens."""
+    idx_gpu, w_gpu = np.asarray(idx_gpu), np.asarray(w_gpu)
+    ties = []
+    for t in range(idx_gpu.shape[0]):
+        if np.array_equal(idx_gpu[t], r["idx"][t]):
+            assert np.allclose(w_gpu[t], r["w"][t], rtol=2e-7, atol=0), t
+        else:
+            assert r["ties"][t] != 0, f"token {t}: selection differs without a near-tie"
+            ties.append(t)
+    return ties
+
+
+def gpu_layer(glay, wl, x_np, bias=None, bits=None):
+    """Whole layer through qrx_moe_forward; returns (idx, w, out) on the host."""
+    bits = wl.wbits if bits is None else bits
+    cfg = qrx.cfg_of(wl.with_(wbits=bits))
+    T = x_np.shape[0]
+    x = to_device_act(wl, x_np)
+    idx = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+    out = torch.empty((T, wl.hidden), dtype=torch.float32, device="cuda")
+    ws = qrx.workspace(cfg, T)
+    qrx.qrx_moe_forward(cfg, x, glay.Wr, glay.bias if bias is None else bias,
+                        glay.routed[bits], glay.shared[bits], idx, w, out, ws)
+    torch.cuda.synchronize()
+    assert qrx.qrx_last_error() == qrx.QRX_OK
+    return np_(idx), np_(w), np_(out)
+
+
+def gpu_staged(glay, wl, x_np, idx_np, w_np, bits=None):
+    """The layer by stages from a given selection (used to resolve near-ties)."""
+    bits = wl.wbits if bits is None else bits
+    c = qrx.cfg_of(wl.with_(wbits=bits))
+    T = x_np.shape[0]
+    ws = qrx.workspace(c, T)
+    perm = qrx.Perm.empty(T, wl.top_k, wl.n_experts)
+    qrx.qrx_permute(c, cu(idx_np.astype(np.int32)), perm)
+    x = to_device_act(wl, x_np)
+    kw = dict(x=x)
+    if wl.afmt == W.A_Q8:
+        xq = torch.empty((T, wl.hidden), dtype=torch.int8, device="cuda")
+        xd = torch.empty((T, wl.hidden // 32), dtype=torch.float32, device="cuda")
+        qrx.qrx_quantize_act_q8(x, xq, xd)
+        kw = dict(xq=xq, xd=xd)
+    A = T * wl.top_k
+    ys = torch.empty((A, wl.hidden), dtype=torch.float32, device="cuda")
+    ysh = torch.empty((T, wl.hidden), dtype=torch.float32, device="cuda")
+    qrx.qrx_expert_ffn(c, glay.routed[bits], perm, T, ys, ws, **kw)
+    qrx.qrx_shared_ffn(c, glay.shared[bits], T, ysh, ws, **kw)
+    out = torch.empty((T, wl.hidden), dtype=torch.float32, device="cuda")
+    qrx.qrx_combine(c, ys, ysh, cu(w_np.astype(np.float32)), perm.inv, out)
+    torch.cuda.synchronize()
+    assert qrx.qrx_last_error() == qrx.QRX_OK
+    return np_(out)
+
+
+def check_layer(glay, olay, wl, x_np, tokens, bits=None, bias_np=None):
+    """Whole-layer parity on the listed tokens (near-ties resolved by the oracle)."""
+    bits = wl.wbits if bits is None else bits
+    wlb = wl.with_(wbits=bits)
+    bias_np = router_weights(wl)[1] if bias_np is None else bias_np
+    idx, w, out = gpu_layer(glay, wlb, x_np, bias=cu(bias_np), bits=bits)
+    r, ref = olay.forward_tokens(wlb, x_np, tokens, bias=bias_np)
+    ties = check_routing(r, idx, w)
+    got = out[list(tokens)]
+    if ties:
+        staged = gpu_staged(glay, wlb, x_np, r["idx"], r["w"], bits)
+        got = staged[list(tokens)]
+    e = rel_err(got, ref)
+    assert e <= TOL, f"{wl.name} int{bits}: rel err {e:.3g}"
+    return dict(rel_err=e, ties=len(ties), idx=idx, out=out)
+
+
+# ------------------------------------------------------------------ bit-exact kernels
+@pytest.mark.parametrize("bits", [8, 4, 2])
+def test_quantize_weights_bitexact(dev, bits):
+    for K in (256, 6144):
+        w = synth.normal_f32(71, bits, 40 * K, 0.0, 0.02).reshape(40, K)
+        w[1] = 0.0
+        w[2] = (np.arange(K) % 16 - 7.5).astype(np.float32) * 2 ** -4   # exact halves
+        w[3, :] = 1e-30
+        w[3, 5] = -3e-30
+        q_ref, s_ref = oracle.quantize_rows(w, bits)
+        q = torch.zeros((40, K * bits // 8), dtype=torch.uint8, device="cuda")
+        s = torch.zeros(40, dtype=torch.float32, device="cuda")
+        qrx.qrx_quantize_weights(cu(w), bits, q, K * bits // 8, s, 1)
+        torch.cuda.synchronize()
+        assert np.array_equal(np_(q), q_ref)
+        assert np.array_equal(np_(s).view(np.uint32), s_ref.view(np.uint32))
+
+
+def test_quantize_act_q8_bitexact(dev):
+    T, H = 33, 6144
+    x = synth.normal_f32(72, 0, T * H).reshape(T, H)
+    x[0, :32] = 0.0
+    x[1, 32:64] = 1e-38
+    x[2, :32] = np.arange(32, dtype=np.float32) * 0.0625 - 1.0    # exact multiples
+    q_ref, d_ref = oracle.quantize_q8(x)
+    xq = torch.empty((T, H), dtype=torch.int8, device="cuda")
+    xd = torch.empty((T, H // 32), dtype=torch.float32, device="cuda")
+    qrx.qrx_quantize_act_q8(cu(x), xq, xd)
+    torch.cuda.synchronize()
+    assert np.array_equal(np_(xq), q_ref)
+    assert np.array_equal(np_(xd).view(np.uint32), d_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("bits", [8, 4, 2])
+def test_block_dots_bitexact(dev, bits):
+    rng = np.random.default_rng(bits)
+    for K in (256, 2048, 6144):
+        w = synth.normal_f32(73, bits, 24 * K, 0.0, 0.02).reshape(24, K)
+        q_ref, _ = oracle.quantize_rows(w, bits)
+        xq = rng.integers(-127, 128, size=K).astype(np.int8)
+        acc_ref = oracle.block_dots_q8(q_ref, K, bits, xq)
+        acc = torch.empty((24, K // 32), dtype=torch.int32, device="cuda")
+        qrx.qrx_block_dots_q8(bits, cu(q_ref), K, cu(xq), acc)
+        torch.cuda.synchronize()
+        assert np.array_equal(np_(acc), acc_ref)
+
+
+# ------------------------------------------------------------------ router and permutation
+def _route_gpu(glay, wl, x_np, bias_np):
+    c = qrx.cfg_of(wl)
+    T = x_np.shape[0]
+    idx = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+    ws = qrx.workspace(c, T)
+    qrx.qrx_route(c, to_device_act(wl, x_np), glay.Wr, cu(bias_np), idx, w, ws)
+    torch.cuda.synchronize()
+    return np_(idx), np_(w)
+
+
+def test_route_tiny(tiny):
+    glay, olay = tiny
+    for T in (1, 5, 8, 64):
+        wl = W.TINY.with_(T=T)
+        x = activations(wl, T)
+        _, bias = router_weights(wl)
+        idx, w = _route_gpu(glay, wl, x, bias)
+        check_routing(oracle.router(wl, x, olay.Wr, bias), idx, w)
+
+
+@pytest.mark.parametrize("wl", [W.GLM_DECODE_T1, W.GLM_DECODE_T32_Q8, W.GLM_VERIFY_T4_BF16,
+                                W.GLM_PREFILL_T2048_BF16], ids=lambda w: w.name)
+def test_route_glm(glm, wl):
+    glay, olay = glm
+    x = activations(wl)
+    _, bias = router_weights(wl)
+    idx, w = _route_gpu(glay, wl, x, bias)
+    r = oracle.router(wl, x, olay.Wr, bias)
+    ties = check_routing(r, idx, w)
+    assert len(ties) <= max(2, wl.T // 50)
+
+
+def _perm_gpu(idx_np, E):
+    T, k = idx_np.shape
+    wl = W.TINY.with_(n_experts=E, n_group=1, topk_group=1, top_k=k)
+    perm = qrx.Perm.empty(T, k, E)
+    qrx.qrx_permute(qrx.cfg_of(wl), cu(idx_np.astype(np.int32)), perm)
+    torch.cuda.synchronize()
+    return {k_: np_(getattr(perm, k_)) for k_ in ("counts", "offsets", "sorted", "inv",
+                                                  "union_ids", "n_union")}
+
+
+def test_permute_bitexact(dev):
+    rng = np.random.default_rng(9)
+    for T, k, E in [(1, 8, 256), (7, 4, 16), (64, 8, 256), (2048, 8, 256), (33, 3, 1024),
+                    (5, 1, 2)]:
+        idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
+        if T == 2048:
+            idx = (rng.zipf(1.5, size=(T, k)) % E).astype(np.int32)   # skewed load
+        ref = oracle.permute(idx, E)
+        got = _perm_gpu(idx, E)
+        for key in ("counts", "offsets", "sorted", "inv"):
+            assert np.array_equal(got[key], ref[key]), (T, k, E, key)
+        n = int(got["n_union"][0])
+        assert n == ref["n_union"]
+        assert np.array_equal(got["union_ids"][:n], ref["union_ids"])
+
+
+def test_permute_bad_index_sets_device_flag(dev):
+    idx = np.array([[0, 3], [16, 1]], dtype=np.int32)        # 16 is outside [0, 16)
+    _perm_gpu(idx, 16)
+    assert qrx.qrx_last_error() == qrx.QRX_EDEVICE
+    assert qrx.qrx_last_error() == qrx.QRX_OK                # the flag was cleared
+
+
+# ------------------------------------------------------------------ FFN stages, tiny layer
+@pytest.mark.parametrize("bits", [8, 4, 2])
+@pytest.mark.parametrize("afmt", [W.A_F32, W.A_Q8, W.A_BF16], ids=["f32", "q8", "bf16"])
+@pytest.mark.parametrize("T", [1, 5, 8])
+def test_stages_tiny(tiny, bits, afmt, T):
+    glay, olay = tiny
+    wl = W.TINY.with_(wbits=bits, afmt=afmt, T=T)
+    x = activations(wl, T)
+    _, bias = router_weights(wl)
+    r = oracle.router(wl, x, olay.Wr, bias)
+    p = oracle.permute(r["idx"], wl.n_experts)
+    ex = olay.experts(r["idx"].ravel(), bits)
+    h_o, y_o = oracle.expert_ffn(wl, ex, p, x)
+    hsh_o, ysh_o = oracle.shared_ffn(wl, olay.shared(bits), x)
+    out_o = oracle.combine(wl, y_o, ysh_o, r["w"], p["inv"])
+
+    c = qrx.cfg_of(wl)
+    ws = qrx.workspace(c, T)
+    perm = qrx.Perm.empty(T, wl.top_k, wl.n_experts)
+    qrx.qrx_permute(c, cu(r["idx"]), perm)
+    xt = to_device_act(wl, x)
+    kw = dict(x=xt)
+    if afmt == W.A_Q8:
+        xq = torch.empty((T, wl.hidden), dtype=torch.int8, device="cuda")
+        xd = torch.empty((T, wl.hidden // 32), dtype=torch.float32, device="cuda")
+        qrx.qrx_quantize_act_q8(xt, xq, xd)
+        q_ref, d_ref = oracle.quantize_q8(x)
+        torch.cuda.synchronize()
+        assert np.array_equal(np_(xq), q_ref) and np.array_equal(np_(xd), d_ref)
+        kw = dict(xq=xq, xd=xd)
+    A = T * wl.top_k
+    hs = torch.empty((A, wl.inter), dtype=torch.float32, device="cuda")
+    ys = torch.empty((A, wl.hidden), dtype=torch.float32, device="cuda")
+    qrx.qrx_expert_ffn(c, glay.routed[bits], perm, T, ys, ws, h_sorted=hs, **kw)
+    hsh = torch.empty((T, wl.inter), dtype=torch.float32, device="cuda")
+    ysh = torch.empty((T, wl.hidden), dtype=torch.float32, device="cuda")
+    qrx.qrx_shared_ffn(c, glay.shared[bits], T, ysh, ws, h_sh=hsh, **kw)
+    # down stage fed the oracle's h
+    yd = torch.empty((A, wl.hidden), dtype=torch.float32, device="cuda")
+    qrx.qrx_expert_down(c, glay.routed[bits], perm, cu(h_o), T, yd, ws)
+    # combine fed the oracle's expert outputs
+    oc = torch.empty((T, wl.hidden), dtype=torch.float32, device="cuda")
+    qrx.qrx_combine(c, cu(y_o), cu(ysh_o), cu(r["w"]), perm.inv, oc)
+    torch.cuda.synchronize()
+    assert qrx.qrx_last_error() == qrx.QRX_OK
+    assert np.array_equal(np_(perm.sorted), p["sorted"])
+    for name, got, ref in [("h", hs, h_o), ("y", ys, y_o), ("h_sh", hsh, hsh_o),
+                           ("y_sh", ysh, ysh_o), ("down(h_oracle)", yd, y_o)]:
+        assert rel_err(np_(got), ref) <= TOL, name
+    assert rel_err(np_(oc), out_o) <= 1e-6
+    # the whole layer
+    check_layer(glay, olay, wl, x, range(T), bits)
+
+
+def test_tiny_zero_input_gives_zero(tiny):
+    glay, _ = tiny
+    wl = W.TINY
+    _, _, out = gpu_layer(glay, wl, np.zeros((8, wl.hidden), np.float32))
+    assert not out.any()
+
+
+def test_tiny_large_batch_many_token_groups(tiny):
+    """T = 300 tokens at the tiny size: every expert serves many tokens."""
+    glay, olay = tiny
+    for afmt in (W.A_F32, W.A_Q8):
+        wl = W.TINY.with_(T=300, afmt=afmt)
+        x = activations(wl, 300, batch=3)
+        check_layer(glay, olay, wl, x, [0, 77, 299])
+
+
+# ------------------------------------------------------------------ GLM-shaped layer, full size
+def test_glm_decode_t1(glm):
+    glay, olay = glm
+    wl = W.GLM_DECODE_T1
+    for b in range(3):
+        check_layer(glay, olay, wl, activations(wl, 1, batch=b), [0])
+
+
+def test_glm_decode_t32_q8(glm):
+    glay, olay = glm
+    wl = W.GLM_DECODE_T32_Q8
+    res = check_layer(glay, olay, wl, activations(wl), [0, 13, 31])
+    n_union = len(np.unique(res["idx"]))
+    assert n_union < 256                       # skewed bias: the union is below E
+
+
+def test_glm_verify_t4_bf16(glm):
+    glay, olay = glm
+    wl = W.GLM_VERIFY_T4_BF16
+    check_layer(glay, olay, wl, activations(wl), range(4))
+
+
+def test_glm_prefill_t2048_bf16(glm):
+    glay, olay = glm
+    wl = W.GLM_PREFILL_T2048_BF16
+    check_layer(glay, olay, wl, activations(wl), [0, 1031, 2047])
+
+
+@pytest.mark.parametrize("wl", W.sweep(), ids=lambda w: w.name)
+def test_glm_sweep(glm, wl):
+    glay, olay = glm
+    toks = [0] if wl.T == 1 else [0, wl.T - 1]
+    check_layer(glay, olay, wl, activations(wl), toks, bits=wl.wbits)
+
+
+def test_glm_all_tokens_one_expert_set(glm):
+    """Degenerate routing: a bias that sends all 64 tokens to experts 0..7 (union = 8)."""
+    glay, olay = glm
+    wl = W.GLM_DECODE_T1.with_(T=64)
+    bias = np.zeros(wl.n_experts, np.float32)
+    bias[:8] = 10.0
+    x = activations(wl, 64, batch=5)
+    res = check_layer(glay, olay, wl, x, [0, 63], bias_np=bias)
+    assert sorted(np.unique(res["idx"]).tolist()) == list(range(8))
+
+
+def test_glm_deterministic(glm):
+    glay, _ = glm
+    wl = W.GLM_DECODE_T32_Q8
+    x = activations(wl)
+    bias = cu(router_weights(wl)[1])
+    a = gpu_layer(glay, wl, x, bias=bias)[2]
+    b = gpu_layer(glay, wl, x, bias=bias)[2]
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+def test_hostio_matches_device_call(glm):
+    glay, _ = glm
+    wl = W.GLM_DECODE_T1
+    x = activations(wl, 1, batch=7)
+    _, _, out = gpu_layer(glay, wl, x)
+    c = qrx.cfg_of(wl)
+    xh = torch.from_numpy(x).pin_memory()
+    oh = torch.empty((1, wl.hidden), dtype=torch.float32).pin_memory()
+    ws = qrx.workspace(c, 1)
+    qrx.qrx_moe_forward_hostio(c, xh, glay.Wr, glay.bias, glay.routed[4], glay.shared[4], oh, ws)
+    assert np.array_equal(oh.numpy(), out)
