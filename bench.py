@@ -47,6 +47,10 @@ def parse():
                     help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="profiling case: fewer routed experts (same per-launch work at T=1)")
+    ap.add_argument("--no-settle", action="store_true",
+                    help="skip the 1 s clock-settle loop (for ncu launch counting)")
     return ap.parse_args()
 
 
@@ -252,7 +256,7 @@ def run_qrx(args, wl, rank, world, local_rank):
         step(i, warm_evs)
     t_settle = time.perf_counter()
     i = 0
-    while time.perf_counter() - t_settle < 1.0:          # clocks settle under load
+    while not args.no_settle and time.perf_counter() - t_settle < 1.0:   # clocks settle
         step(i, warm_evs)
         i += 1
         if i % 64 == 0:
@@ -261,9 +265,11 @@ def run_qrx(args, wl, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_push("timed")
     for i in range(args.steps):
         step(i, evs[i])
     torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_pop()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -354,6 +360,8 @@ def main():
     args = parse()
     from quantized_routed_expert_tc_b200 import workloads as W
     wl = W.ALL[args.workload]
+    if args.experts:
+        wl = wl.with_(name=f"{wl.name}_e{args.experts}", n_experts=args.experts)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -176,7 +176,9 @@ void qo_unpack_rows(const uint8_t *q, int64_t rows, int64_t K, int bits, int8_t 
  * activations.  Workload definition: blocks of 32, f32 absmax scale.
  * [reading] d = amax/127 (f32 division); q = clamp(round-half-away(x * f),
  * -127, 127) with f = 127/amax (one f32 division, one f32 multiply per
- * element); a zero block has d = 0 and q = 0. */
+ * element); the clamp applies to the f32 product (so a block whose amax is
+ * below 127/FLT_MAX, where f overflows, still maps to +-127 and 0); a zero
+ * block has d = 0 and q = 0. */
 void qo_quantize_q8(const float *x, int64_t n, int8_t *q, float *d)
 {
     for (int64_t b = 0; b < n / 32; ++b) {
@@ -192,12 +194,16 @@ void qo_quantize_q8(const float *x, int64_t n, int8_t *q, float *d)
             continue;
         }
         d[b] = amax / 127.0f;
-        float f = 127.0f / amax;
+        float f = 127.0f / amax;      /* +inf when amax < 127/FLT_MAX */
         for (int i = 0; i < 32; ++i) {
+            /* the clamp is taken on the product, so an infinite factor still
+             * gives +-127, and 0 * inf (a zero beside a tiny amax) gives 0 */
             float v = xb[i] * f;
-            int c = (int)roundf(v);
-            if (c > 127) c = 127;
-            if (c < -127) c = -127;
+            int c;
+            if (v != v) c = 0;
+            else if (v >= 127.0f) c = 127;
+            else if (v <= -127.0f) c = -127;
+            else c = (int)roundf(v);
             q[b * 32 + i] = (int8_t)c;
         }
     }

@@ -205,10 +205,7 @@ __global__ void __launch_bounds__(GV_NT, 1) k_ffn_gemv(const GemvP p)
                         const float v = p.hin[row * p.hin_ld + elem];
                         const float amax = warp_max(fabsf(v));
                         if (amax != 0.f) {
-                            const float f = __fdiv_rn(127.f, amax);
-                            int q = (int)roundf(__fmul_rn(v, f));
-                            q = q > 127 ? 127 : (q < -127 ? -127 : q);
-                            d[0] = (int8_t)q;
+                            d[0] = (int8_t)q8_code(v, __fdiv_rn(127.f, amax));
                             sig = __fdiv_rn(amax, 127.f);
                         }
                     }

@@ -69,9 +69,7 @@ __global__ void __launch_bounds__(256) k_quantize_act_q8(const float *__restrict
     const float amax = warp_max(fabsf(v));
     int c = 0;
     if (amax != 0.f) {
-        const float f = __fdiv_rn(127.f, amax);
-        c = (int)roundf(__fmul_rn(v, f));
-        c = c > 127 ? 127 : (c < -127 ? -127 : c);
+        c = q8_code(v, __fdiv_rn(127.f, amax));
     }
     xq[b * 32 + lane] = (int8_t)c;
     if (lane == 0) xd[b] = amax != 0.f ? __fdiv_rn(amax, 127.f) : 0.f;

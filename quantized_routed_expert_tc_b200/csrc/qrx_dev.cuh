@@ -134,6 +134,18 @@ __device__ __forceinline__ float warp_max(float v)
     return v;
 }
 
+// Q8_0 code of x given f = 127/amax: round-half-away of the f32 product,
+// clamped to [-127, 127] on the product (an infinite f from a tiny amax still
+// gives +-127; 0 * inf gives 0).
+__device__ __forceinline__ int q8_code(float x, float f)
+{
+    const float v = __fmul_rn(x, f);
+    if (v != v) return 0;
+    if (v >= 127.f) return 127;
+    if (v <= -127.f) return -127;
+    return (int)roundf(v);
+}
+
 __device__ __forceinline__ float silu_mul(float g, float u)
 {
     return g / (1.0f + expf(-g)) * u;

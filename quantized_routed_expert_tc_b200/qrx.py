@@ -273,6 +273,9 @@ def qrx_moe_forward_profiled(cfg, x, Wr, bias, routed: Experts, shared: Experts 
                              topk_idx, topk_w, out, ws, events, stream=None):
     """qrx_moe_forward recording 7 torch.cuda.Event objects between its stages."""
     sh = ctypes.byref(shared.c()) if shared is not None else None
+    for ev in events:                     # torch creates the CUDA event on first record
+        if not ev.cuda_event:
+            ev.record(stream)
     arr = (vp * 7)(*[ev.cuda_event for ev in events])
     _check("qrx_moe_forward_profiled", lib().qrx_moe_forward_profiled(
         ctypes.byref(cfg), _p(x), x.shape[0], _p(Wr), _p(bias), ctypes.byref(routed.c()), sh,

@@ -161,6 +161,8 @@ def test_q8_properties():
     x = synth.normal_f32(12, 1, 32 * 64, 0.0, 1.0).reshape(64, 32)
     x[5] = 0.0
     x[6, 3] = 1e-30
+    x[7] = 0.0
+    x[7, :3] = [1e-38, -5e-39, 2e-39]   # amax below 127/FLT_MAX: 127/amax overflows
     q, d = oracle.quantize_q8(x)
     q = q.astype(np.int64)
     for b in range(64):
