@@ -204,6 +204,31 @@ int qrx_combine(const qrx_cfg *cfg, const float *y_sorted, const float *y_sh,
                 const float *topk_w, const int32_t *inv, int32_t T, float *out,
                 void *stream);
 
+/* qrx_expert_ffn without any caller workspace, for callers that cannot
+ * allocate device memory when they call in: for example a host whose memory
+ * allocator owns the whole device budget and hands out nothing after start-up,
+ * or a plug-in loaded into another runtime that gives it no allocator and no
+ * workspace.  There is no counterpart of this call on the colibri pages; it is
+ * the routed FFN of qrx_expert_ffn with its one scratch buffer (the gate/up
+ * output h, T*k*I f32 values) held in a fixed 4 MiB array inside the library.
+ *   - Limit: T*top_k*inter*4 bytes must fit 4 MiB (for I = 2048, k = 8:
+ *     T <= 64); larger T returns QRX_ENOSPACE before any launch.  Only the
+ *     GEMV path of qrx_expert_ffn is used.
+ *   - The array is a file-scope device variable: every GPU that loads the
+ *     library holds its 4 MiB until the process exits.  The first call on a
+ *     device looks up the array's device address (cudaGetSymbolAddress) with
+ *     that device current; make that first call before any stream capture.
+ *   - The array is shared by all calls on a device and keeps the last call's
+ *     contents; nothing in it needs clearing, because every row of h that the
+ *     down projection reads is written by the same call's gate/up step first.
+ *     Calls that overlap on the GPU (on different streams, or from different
+ *     host threads) race on the array: serialise them.
+ *   - The call allocates nothing (no cudaMalloc, no library allocation).
+ * Arguments and results are as qrx_expert_ffn, minus h_sorted and ws. */
+int qrx_expert_ffn_noalloc(const qrx_cfg *cfg, const qrx_experts *routed,
+                           const qrx_perm *perm, const qrx_act *act, int32_t T,
+                           float *y_sorted, void *stream);
+
 /* ---- the whole layer --------------------------------------------------- */
 
 /* route -> permute -> (Q8_0 quantise) -> routed + shared FFN -> combine, all

@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "qrx_internal.h"
 #include "qrx_dev.cuh"
@@ -486,3 +487,65 @@ int qrx_moe_forward_hostio(const qrx_cfg *c, const void *x_host, int32_t T, cons
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free routed FFN: its scratch (h) lives in a fixed device array.
+// Callers that cannot allocate device memory when they call in use this entry
+// point instead of qrx_expert_ffn.  The array's name is only a host-side
+// handle in host code; its device address comes from cudaGetSymbolAddress,
+// looked up once per device with that device current.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;   // 4 MiB per device
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[kMaxDevices] = {nullptr};
+
+int noalloc_scratch(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QRX_ECUDA;
+    if (dev < 0 || dev >= kMaxDevices) return QRX_EUNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QRX_ECUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return QRX_OK;
+}
+
+}  // namespace
+
+extern "C" int qrx_expert_ffn_noalloc(const qrx_cfg *c, const qrx_experts *routed,
+                                      const qrx_perm *perm, const qrx_act *act, int32_t T,
+                                      float *y_sorted, void *stream)
+{
+    int v = check_common(c, T);
+    if (v) return v;
+    if ((v = check_experts(routed)) || (v = check_perm(perm)) || (v = check_act(c, act))) return v;
+    if (!y_sorted) return QRX_EINVAL;
+    const size_t need = (size_t)T * c->top_k * c->inter * sizeof(float);
+    if (need > kNoAllocScratchBytes) return QRX_ENOSPACE;
+    void *scratch = nullptr;
+    if ((v = noalloc_scratch(&scratch))) return v;
+    FfnArgs a = ffn_args(c, T);
+    set_act(a, act);
+    set_routed(a, routed, perm);
+    a.h = static_cast<float *>(scratch);
+    a.h_ld = c->inter;
+    a.y = y_sorted;
+    a.y_ld = c->hidden;
+    const int sms = num_sms_current();
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = launch_ffn_gateup(a, sms, st);
+    if (e == cudaSuccess) e = launch_ffn_down(a, sms, st);
+    return cuda_code(e);
+}

@@ -68,6 +68,8 @@ _SIGS = {
     "qrx_permute": ([P(Cfg), vp, i32, P(CPerm), vp], ctypes.c_int),
     "qrx_expert_ffn": ([P(Cfg), P(CExperts), P(CPerm), P(CAct), i32, vp, vp, vp, sz, vp],
                        ctypes.c_int),
+    "qrx_expert_ffn_noalloc": ([P(Cfg), P(CExperts), P(CPerm), P(CAct), i32, vp, vp],
+                               ctypes.c_int),
     "qrx_expert_down": ([P(Cfg), P(CExperts), P(CPerm), vp, i32, vp, vp, sz, vp], ctypes.c_int),
     "qrx_shared_ffn": ([P(Cfg), P(CExperts), P(CAct), i32, vp, vp, vp, sz, vp], ctypes.c_int),
     "qrx_combine": ([P(Cfg), vp, vp, vp, vp, i32, vp, vp], ctypes.c_int),
@@ -240,6 +242,14 @@ def qrx_expert_ffn(cfg, routed: Experts, perm: Perm, T, y_sorted, ws, x=None, xq
         ctypes.byref(cfg), ctypes.byref(routed.c()), ctypes.byref(perm.c()),
         ctypes.byref(_act(cfg, x, xq, xd)), T, _p(h_sorted), _p(y_sorted), _p(ws), ws.numel(),
         _st(stream)))
+
+
+def qrx_expert_ffn_noalloc(cfg, routed: Experts, perm: Perm, T, y_sorted, x=None, xq=None,
+                           xd=None, stream=None):
+    """qrx_expert_ffn with no caller workspace (the library's fixed 4 MiB array)."""
+    _check("qrx_expert_ffn_noalloc", lib().qrx_expert_ffn_noalloc(
+        ctypes.byref(cfg), ctypes.byref(routed.c()), ctypes.byref(perm.c()),
+        ctypes.byref(_act(cfg, x, xq, xd)), T, _p(y_sorted), _st(stream)))
 
 
 def qrx_expert_down(cfg, routed: Experts, perm: Perm, h_sorted, T, y_sorted, ws, stream=None):
