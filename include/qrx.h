@@ -77,7 +77,7 @@ typedef struct {
     int32_t afmt;                  /* qrx_afmt of the activations */
 } qrx_cfg;
 
-/* Packed experts (see layout above).  All device pointers. */
+/* Packed experts (see layout above).  All device pointers, 16-byte aligned. */
 typedef struct {
     const uint8_t *w13;
     const float *s13;
@@ -209,20 +209,24 @@ int qrx_combine(const qrx_cfg *cfg, const float *y_sorted, const float *y_sh,
  * allocator owns the whole device budget and hands out nothing after start-up,
  * or a plug-in loaded into another runtime that gives it no allocator and no
  * workspace.  There is no counterpart of this call on the colibri pages; it is
- * the routed FFN of qrx_expert_ffn with its one scratch buffer (the gate/up
- * output h, T*k*I f32 values) held in a fixed 4 MiB array inside the library.
- *   - Limit: T*top_k*inter*4 bytes must fit 4 MiB (for I = 2048, k = 8:
- *     T <= 64); larger T returns QRX_ENOSPACE before any launch.  Only the
- *     GEMV path of qrx_expert_ffn is used.
+ * the routed FFN of qrx_expert_ffn with its scratch (the gate/up output h,
+ * T*k*I f32 values, and the digit records of the activations and of h) held
+ * in a fixed 8 MiB array inside the library.
+ *   - Limit: the 256-byte-aligned T*top_k*inter*4 bytes of h, plus T records
+ *     of the activations and T*top_k records of h must fit 8 MiB.  A record of
+ *     a row of length K takes 3*K + 16*(K/32) bytes (f32, bf16) or
+ *     K + 8*(K/32) bytes (Q8_0).  For the GLM shape (H = 6144, I = 2048,
+ *     k = 8) that is T <= 58 with f32 or bf16 activations.  Larger T returns
+ *     QRX_ENOSPACE before any launch.
  *   - The array is a file-scope device variable: every GPU that loads the
- *     library holds its 4 MiB until the process exits.  The first call on a
+ *     library holds its 8 MiB until the process exits.  The first call on a
  *     device looks up the array's device address (cudaGetSymbolAddress) with
  *     that device current; make that first call before any stream capture.
  *   - The array is shared by all calls on a device and keeps the last call's
- *     contents; nothing in it needs clearing, because every row of h that the
- *     down projection reads is written by the same call's gate/up step first.
- *     Calls that overlap on the GPU (on different streams, or from different
- *     host threads) race on the array: serialise them.
+ *     contents; nothing in it needs clearing, because every record and every
+ *     row of h that a kernel reads is written by the same call first.  Calls
+ *     that overlap on the GPU (on different streams, or from different host
+ *     threads) race on the array: serialise them.
  *   - The call allocates nothing (no cudaMalloc, no library allocation).
  * Arguments and results are as qrx_expert_ffn, minus h_sorted and ws. */
 int qrx_expert_ffn_noalloc(const qrx_cfg *cfg, const qrx_experts *routed,
@@ -231,8 +235,11 @@ int qrx_expert_ffn_noalloc(const qrx_cfg *cfg, const qrx_experts *routed,
 
 /* ---- the whole layer --------------------------------------------------- */
 
-/* route -> permute -> (Q8_0 quantise) -> routed + shared FFN -> combine, all
- * on `stream` with no host synchronisation (capturable in a CUDA graph).
+/* activation records -> route -> permute -> routed + shared FFN -> combine,
+ * all on `stream` with no host synchronisation (capturable in a CUDA graph).
+ * The kernels after the first are chained with programmatic dependent launch:
+ * each may start while its predecessor drains and waits for it only where it
+ * reads its output (the down kernel starts streaming its weights first).
  * shared may be NULL.  topk_idx, topk_w: outputs [T][k].  out [T][H] f32. */
 int qrx_moe_forward(const qrx_cfg *cfg, const void *x, int32_t T, const float *W_router,
                     const float *bias, const qrx_experts *routed, const qrx_experts *shared,
@@ -240,11 +247,13 @@ int qrx_moe_forward(const qrx_cfg *cfg, const void *x, int32_t T, const float *W
                     size_t ws_bytes, void *stream);
 
 /* qrx_moe_forward with stage timing: events[0..6] are cudaEvent_t handles
- * (passed as void*) recorded on `stream` before the router, after the
- * router, after the permutation, after the Q8_0 activation quantiser (right
- * after the permutation when there is none), after the gate/up kernel, after
- * the down kernel and after the combine.  n_events must be 7.  Everything
- * else is as qrx_moe_forward. */
+ * (passed as void*) recorded on `stream` before the activation-record
+ * kernel, after it, after the router, after the permutation, after the
+ * gate/up kernel, after the down kernel and after the combine.  n_events must
+ * be 7.  The events separate the kernels, so the launch overlap that
+ * qrx_moe_forward gets from programmatic dependent launch is lost here: the
+ * stage times add up to more than a plain call takes.  Everything else is as
+ * qrx_moe_forward. */
 int qrx_moe_forward_profiled(const qrx_cfg *cfg, const void *x, int32_t T,
                              const float *W_router, const float *bias,
                              const qrx_experts *routed, const qrx_experts *shared,

@@ -13,6 +13,8 @@ __global__ void __launch_bounds__(256) k_combine(const float *__restrict__ y, co
                                                  const int32_t *__restrict__ inv, int T, int k, int H,
                                                  float *__restrict__ out)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int hq = H / 4;
     if (id >= (int64_t)T * hq) return;
@@ -37,8 +39,8 @@ cudaError_t launch_combine(const float *y_sorted, const float *y_sh, const float
                            const int32_t *inv, int T, int k, int H, float *out, cudaStream_t st)
 {
     const int64_t n = (int64_t)T * (H / 4);
-    k_combine<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(y_sorted, y_sh, w, inv, T, k, H, out);
-    return cudaGetLastError();
+    return launch_k(k_combine, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, y_sorted, y_sh, w,
+                    inv, T, k, H, out);
 }
 
 }  // namespace qrx

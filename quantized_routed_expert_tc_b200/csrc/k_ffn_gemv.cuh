@@ -8,29 +8,260 @@
 // expert is a SwiGLU FFN: h = silu(s_g Q_g x) * (s_u Q_u x), y = s_d Q_d h.
 //
 // Work decomposition.  A "slot" is one expert of the union (or the shared
-// expert) with the list of token positions routed to it, cut into token
-// groups of at most TS tokens.  Each slot's matrix is cut into blocks of RB
-// rows; the (slot, group, block) units are split into contiguous ranges of
-// equal estimated cost (weight streaming plus per-token dot work), one range
-// per CTA (one CTA per SM).  Inside a CTA, a "team" of CPR threads covers
-// one row (thread c loads 16-byte chunk c of the row), and each team handles R
-// consecutive rows of a block.  The slot's activations are staged once into
-// shared memory as digit planes (see qrx_dev.cuh) for up to TS tokens; each
-// thread keeps its R weight chunks in registers and runs every staged token
-// over them, so a weight byte is read from HBM once per slot.  For gate/up
-// the matrix rows are interleaved (gate row i, up row i) so the SwiGLU is
-// applied where both rows' sums meet.  Reductions are fixed-order (warp
-// butterflies, then warp partials in index order): results are deterministic.
+// expert) with the token positions routed to it, cut into token groups of at
+// most TS tokens.  Each slot's matrix is cut into blocks of RB rows (always
+// 48 KB: 384 threads x 8 rows x 16 bytes); the (slot, group, block) units are
+// split into contiguous ranges of equal estimated cost (weight streaming plus
+// per-token dot work), one range per CTA, one CTA per SM.
+//
+// Memory pipeline.  Thread 0 streams the CTA's blocks with cp.async.bulk into
+// a ring of 3-4 shared-memory stages (mbarrier completion, bounded waits), so
+// up to 144-192 KB per SM are in flight while the CTA computes.  Inside a CTA
+// a "team" of CPR threads covers one row (thread c reads 16-byte chunk c) and
+// handles R = 8 consecutive rows of a block.  Activations enter as digit
+// planes (qrx_dev.cuh) prepared once per row by k_act_digits (tokens, for
+// gate/up) and k_h_digits (h rows, for down).  With one token per slot each
+// thread loads its chunk's digits straight from that record; with more, the
+// slot's token group is staged in shared memory.  Reductions
+// are fixed-order (warp butterflies, then warp partials in index order), so
+// results are deterministic.  For gate/up the matrix rows are interleaved
+// (gate row i, up row i) so the SwiGLU is applied where both sums meet.
 #pragma once
 #include "qrx_dev.cuh"
 
 namespace qrx {
 
-constexpr int GV_NT = 384;   // threads per CTA (12 warps)
-constexpr int GV_R = 8;      // rows per team per block
+constexpr int GV_BLK = 48 * 1024;             // bytes per block: NT threads x R rows x 16 B
+
+// Threads per CTA (12 warps, 8 rows per thread).
+template <int WB, int NDIG> struct GvShape {
+    static constexpr int NT = 384;
+    static constexpr int R = GV_BLK / (NT * 16);
+};
+constexpr int GV_SMEM_MAX = 227 * 1024;       // dynamic shared memory per CTA
+constexpr long long GV_WAIT_CAP = 1ll << 22;  // mbarrier polls before giving up
+
+// ---------------------------------------------------------------- records
+// Digit record of one activation row of length K (per token or per h row):
+//   planes [NDIG][K] bytes, chunk-permuted for the weight format (digit_slot)
+//   scales [K/32] f32      (sigma_b: 2^-s for 22-bit fixed point, d_b for Q8_0)
+//   corr   [K/32][NDIG] i32 (-OFF * sum of the block's digits, per plane)
+__host__ __device__ constexpr int align16(int v) { return (v + 15) & ~15; }
+
+struct RecLayout {
+    int scales, corr, bytes;
+};
+
+__host__ __device__ inline RecLayout rec_layout(int ndig, int K)
+{
+    RecLayout L;
+    L.scales = ndig * K;
+    L.corr = L.scales + align16((K / 32) * 4);
+    L.bytes = L.corr + align16((K / 32) * ndig * 4);
+    return L;
+}
+
+// 2^s as f32 for -126 <= s <= 127, else via ldexpf.
+__device__ __forceinline__ float pow2f(int s)
+{
+    return (s >= -126 && s <= 127) ? __int_as_float((s + 127) << 23) : ldexpf(1.f, s);
+}
+
+// Convert one 32-element block (lane = element) into the record `rec`:
+// NDIG = 3: f32 value -> 3 digits of a 22-bit fixed point; NDIG = 1: Q8_0
+// quantisation of the f32 value.  The caller rounds to bf16 first when the
+// activations are bf16.  All 32 lanes of the warp must call.
+template <int WB, int NDIG>
+__device__ __forceinline__ void stage_block(unsigned char *rec, const RecLayout &L, int cpr, int b,
+                                            int lane, float v)
+{
+    using F = Fmt<WB>;
+    const float amax = warp_max(fabsf(v));
+    int8_t d[3] = {0, 0, 0};
+    float sig = 0.f;
+    if constexpr (NDIG == 1) {
+        if (amax != 0.f) {
+            d[0] = (int8_t)q8_code(v, __fdiv_rn(127.f, amax));
+            sig = __fdiv_rn(amax, 127.f);
+        }
+    } else {
+        if (amax != 0.f) {
+            const int sh = fixed_shift(amax);
+            const float scaled = (sh >= -126 && sh <= 127) ? __fmul_rn(v, pow2f(sh)) : ldexpf(v, sh);
+            split3(__float2int_rn(scaled), d[0], d[1], d[2]);
+            sig = pow2f(-sh);
+        }
+    }
+    const int elem = b * 32 + lane;
+    const int cc = elem / F::EPC, l = elem % F::EPC;
+    int wd, by;
+    digit_slot<WB>(l, wd, by);
+    const int K = cpr * F::EPC;
+#pragma unroll
+    for (int pl = 0; pl < NDIG; ++pl) {
+        rec[(size_t)pl * K + ((size_t)cc * F::DW + wd) * 4 + by] = (unsigned char)d[pl];
+        int sum = d[pl];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) reinterpret_cast<int *>(rec + L.corr)[b * NDIG + pl] = -F::OFF * sum;
+    }
+    if (lane == 0) reinterpret_cast<float *>(rec + L.scales)[b] = sig;
+}
+
+// Q8_0 codes and scales already computed (qrx_quantize_act_q8): permute only.
+template <int WB>
+__device__ __forceinline__ void stage_block_q8(unsigned char *rec, const RecLayout &L, int cpr, int b,
+                                               int lane, int8_t q, float dq)
+{
+    using F = Fmt<WB>;
+    const int elem = b * 32 + lane;
+    const int cc = elem / F::EPC, l = elem % F::EPC;
+    int wd, by;
+    digit_slot<WB>(l, wd, by);
+    rec[((size_t)cc * F::DW + wd) * 4 + by] = (unsigned char)q;
+    int sum = q;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) {
+        reinterpret_cast<int *>(rec + L.corr)[b] = -F::OFF * sum;
+        reinterpret_cast<float *>(rec + L.scales)[b] = dq;
+    }
+}
+
+// Activation rows -> digit records in global memory, one warp per block of 32.
+// Q8_0: from precomputed codes (xq, xd) or, when xq is null, from f32 x.
+template <int WB, int NDIG>
+__global__ void __launch_bounds__(256) k_act_digits(const void *__restrict__ x,
+                                                    const int8_t *__restrict__ xq,
+                                                    const float *__restrict__ xd, int afmt, int T,
+                                                    int K, unsigned char *__restrict__ out)
+{
+    const int lane = threadIdx.x & 31;
+    const int nb = K / 32;
+    pdl_wait();
+    pdl_trigger();
+    const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (gw >= (int64_t)T * nb) return;
+    const int t = (int)(gw / nb), b = (int)(gw % nb);
+    const RecLayout L = rec_layout(NDIG, K);
+    unsigned char *rec = out + (size_t)t * L.bytes;
+    const int cpr = K / Fmt<WB>::EPC;
+    const int64_t e = (int64_t)t * K + b * 32 + lane;
+    if constexpr (NDIG == 1) {
+        if (xq)          // codes and scales from qrx_quantize_act_q8
+            stage_block_q8<WB>(rec, L, cpr, b, lane, xq[e], xd[(int64_t)t * nb + b]);
+        else             // quantise the f32 activations here (same Q8_0 formula)
+            stage_block<WB, 1>(rec, L, cpr, b, lane, reinterpret_cast<const float *>(x)[e]);
+    } else {
+        const float v = afmt == QRX_A_BF16
+                            ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(x)[e])
+                            : reinterpret_cast<const float *>(x)[e];
+        stage_block<WB, NDIG>(rec, L, cpr, b, lane, v);
+    }
+}
+
+// h rows (f32, row stride ld) -> digit records, one warp per block of 32; for
+// bf16 activations h is rounded to bf16 first (the down projection's input).
+template <int WB, int NDIG>
+__global__ void __launch_bounds__(256) k_h_digits(const float *__restrict__ h, int64_t ld, int rows,
+                                                  int K, int afmt, unsigned char *__restrict__ out)
+{
+    const int lane = threadIdx.x & 31;
+    const int nb = K / 32;
+    pdl_wait();
+    pdl_trigger();
+    const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (gw >= (int64_t)rows * nb) return;
+    const int r = (int)(gw / nb), b = (int)(gw % nb);
+    const RecLayout L = rec_layout(NDIG, K);
+    float v = h[(int64_t)r * ld + b * 32 + lane];
+    if (afmt == QRX_A_BF16) v = __bfloat162float(__float2bfloat16_rn(v));
+    stage_block<WB, NDIG>(out + (size_t)r * L.bytes, L, K / Fmt<WB>::EPC, b, lane, v);
+}
+
+// ---------------------------------------------------------------- mbarrier / bulk copy
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// One bulk copy completing on `mbar` (its bytes were announced by expect_tx).
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes, uint32_t mbar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst), "l"(src), "r"(bytes), "r"(mbar)
+        : "memory");
+}
+
+// Bounded wait for phase `parity` of an mbarrier; false if it gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity)
+{
+    for (long long it = 0; it < GV_WAIT_CAP; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(mbar), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+// ---------------------------------------------------------------- kernel
+struct GvSmem {
+    int stage_bytes, scales_off, mbar, cnt, abort, dig, red, red_stage, tin, tout, pre, total;
+};
+
+// Shared memory: `stages` ring stages (weights, then the block's row scales),
+// their mbarriers and arrival counters, the token group's digit records,
+// per-stage partial sums [ts][tpc][wpt][R], token rows, the slot cost prefix.
+__host__ __device__ inline GvSmem gv_smem(int stages, int ts, int recb, int rb, int tpc, int wpt,
+                                          int R, int maxslots)
+{
+    GvSmem m;
+    m.scales_off = GV_BLK;
+    m.stage_bytes = GV_BLK + align16(rb * 4);
+    int o = stages * m.stage_bytes;
+    m.mbar = o;
+    o += stages * 8;
+    m.cnt = o;
+    o += stages * 4;
+    m.abort = o;
+    o = align16(o + 4);
+    m.dig = o;
+    o += ts * recb;
+    m.red = o;
+    m.red_stage = ts * tpc * wpt * R;         // floats
+    o += stages * m.red_stage * 4;
+    m.tin = o;
+    o += ts * 4;
+    m.tout = o;
+    o += ts * 4;
+    o = (o + 7) & ~7;
+    m.pre = o;
+    o += (maxslots + 2) * 8;
+    m.total = o;
+    return m;
+}
 
 struct GemvP {
-    int K, rows, row_bytes, cpr, tpc, rb, nblk, ts, wpt, redn;
+    int K, rows, row_bytes, cpr, tpc, rb, nblk, ts, wpt, stages, maxslots, nthreads;
+    RecLayout rec;
+    GvSmem sm;
     const uint8_t *w;
     int64_t w_stride;        // bytes between experts' matrices
     const float *s;
@@ -41,11 +272,8 @@ struct GemvP {
     const int32_t *offsets, *sorted, *union_ids, *n_union;
     int E, k, T;
     int afmt;
-    const void *x;           // gate/up input rows (token index)
-    const int8_t *xq;
-    const float *xd;
-    const float *hin;        // down input rows
-    int64_t hin_ld, sh_in_row0;
+    const unsigned char *xrec;   // digit records of the input rows (tokens, or h rows)
+    int64_t sh_in_row0;          // down: record row of the shared expert's first h row
     float *out;
     int64_t out_ld, sh_out_row0;
 };
@@ -85,30 +313,197 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
-template <int WB, int NDIG, int TP, bool GATEUP>
-__global__ void __launch_bounds__(GV_NT, 1) k_ffn_gemv(const GemvP p)
+// A lane's view of one activation row: its chunk's digit words, block scales
+// and offset corrections.
+template <int WB, int NDIG>
+struct LaneDig {
+    static constexpr int NBC = WB == 2 ? 2 : 1;     // scale blocks touched by a chunk
+    uint32_t w[NDIG][Fmt<WB>::DW];
+    float sig[NBC];
+    int corr[NBC][NDIG];
+
+    __device__ __forceinline__ void load(const unsigned char *rec, const RecLayout &L, int c, int K)
+    {
+        constexpr int DW = Fmt<WB>::DW;
+#pragma unroll
+        for (int pl = 0; pl < NDIG; ++pl) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(rec + (size_t)pl * K + (size_t)c * DW * 4);
+#pragma unroll
+            for (int q = 0; q < DW / 4; ++q) {
+                const uint4 v4 = src[q];
+                w[pl][4 * q + 0] = v4.x;
+                w[pl][4 * q + 1] = v4.y;
+                w[pl][4 * q + 2] = v4.z;
+                w[pl][4 * q + 3] = v4.w;
+            }
+        }
+        const float *sc = reinterpret_cast<const float *>(rec + L.scales);
+        const int *co = reinterpret_cast<const int *>(rec + L.corr);
+#pragma unroll
+        for (int bc = 0; bc < NBC; ++bc) {
+            const int sb = WB == 8 ? (c >> 1) : (WB == 4 ? c : 2 * c + bc);
+            sig[bc] = sc[sb];
+#pragma unroll
+            for (int pl = 0; pl < NDIG; ++pl) corr[bc][pl] = WB == 8 ? 0 : co[sb * NDIG + pl];
+        }
+    }
+
+    // The lane's share of one row's dot product: exact int32 per block, then f32.
+    // Each plane keeps two partial accumulators (even and odd weight words) so
+    // the dp4a chains are half as deep.
+    __device__ __forceinline__ float dot(const uint4 &wv) const
+    {
+        int acc[NBC][NDIG][2];
+#pragma unroll
+        for (int bc = 0; bc < NBC; ++bc)
+#pragma unroll
+            for (int pl = 0; pl < NDIG; ++pl) {
+                acc[bc][pl][0] = corr[bc][pl];
+                acc[bc][pl][1] = 0;
+            }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t u[Fmt<WB>::UPW];
+            unpack_word<WB>(word_of(wv, i), u);
+            const int bc = WB == 2 ? (i >> 1) : 0;
+#pragma unroll
+            for (int j = 0; j < Fmt<WB>::UPW; ++j)
+#pragma unroll
+                for (int pl = 0; pl < NDIG; ++pl)
+                    acc[bc][pl][i & 1] = dp4a(u[j], w[pl][i * Fmt<WB>::UPW + j], acc[bc][pl][i & 1]);
+        }
+        float v = 0.f;
+#pragma unroll
+        for (int bc = 0; bc < NBC; ++bc) {
+            float cv;
+            if constexpr (NDIG == 3)
+                cv = fmaf(__int2float_rn(acc[bc][2][0] + acc[bc][2][1]), 65536.f,
+                          __int2float_rn((acc[bc][0][0] + acc[bc][0][1]) +
+                                         256 * (acc[bc][1][0] + acc[bc][1][1])));
+            else
+                cv = __int2float_rn(acc[bc][0][0] + acc[bc][0][1]);
+            v = fmaf(sig[bc], cv, v);
+        }
+        return v;
+    }
+};
+
+// Iterator over the CTA's (slot, token group, block) units, in order.
+struct Units {
+    const int64_t *pre;
+    int nslots, nu, nblk, ts;
+    int64_t c0, c1, bwu;
+    int s, j, ntok, nt;
+    int64_t b, bend;
+    bool valid;
+    const uint8_t *W;        // the slot's weights and row scales, looked up once per slot
+    const float *S;
+};
+
+__device__ __forceinline__ int slot_ntok(const GemvP &p, int s, int nu)
 {
-    using F = Fmt<WB>;
-    constexpr int R = GV_R, V = R * TP, LV = Log2<V>::value;
-    constexpr int NBC = WB == 2 ? 2 : 1;              // scale blocks touched by a chunk
-    extern __shared__ __align__(16) unsigned char smem[];
-    const int K = p.K, nb = K / 32, cpr = p.cpr;
-    uint32_t *dig = reinterpret_cast<uint32_t *>(smem);
-    float *bsc = reinterpret_cast<float *>(smem + (size_t)p.ts * NDIG * K);
-    float *red = bsc + (size_t)p.ts * nb;
-    int *tin = reinterpret_cast<int *>(red + 2 * p.redn);
-    int *tout = tin + p.ts;
-    int64_t *pre = reinterpret_cast<int64_t *>(tout + p.ts);   // [nslots + 1], 8-aligned
+    if (s < nu) {
+        const int e = p.union_ids[s];
+        return (e >= 0 && e < p.E) ? p.offsets[e + 1] - p.offsets[e] : 0;
+    }
+    return p.T;
+}
+
+__device__ __forceinline__ const uint8_t *slot_weights(const GemvP &p, int s, int nu);
+__device__ __forceinline__ const float *slot_scales(const GemvP &p, int s, int nu);
+
+// Enter slot s: token count and the slot's weight / scale base pointers.
+__device__ __forceinline__ void units_enter_slot(Units &u, const GemvP &p, int s)
+{
+    u.s = s;
+    u.j = -1;
+    if (s < u.nslots) {
+        u.ntok = slot_ntok(p, s, u.nu);
+        u.W = slot_weights(p, s, u.nu);
+        u.S = slot_scales(p, s, u.nu);
+    }
+}
+
+__device__ void units_advance(Units &u, const GemvP &p)
+{
+    if (u.valid && ++u.b < u.bend) return;
+    u.valid = false;
+    for (;;) {
+        if (u.s >= u.nslots || u.pre[u.s] >= u.c1) return;
+        ++u.j;
+        if ((int64_t)u.j * u.ts >= u.ntok) {
+            units_enter_slot(u, p, u.s + 1);
+            continue;
+        }
+        const int nt = min(u.ts, u.ntok - u.j * u.ts);
+        const int64_t gstart = u.pre[u.s] + (int64_t)u.nblk * u.j * (u.bwu + u.ts);
+        const int64_t cb = u.bwu + nt;
+        int64_t bf = u.c0 > gstart ? (u.c0 - gstart + cb - 1) / cb : 0;
+        int64_t be = u.c1 > gstart ? (u.c1 - gstart + cb - 1) / cb : 0;
+        if (be > u.nblk) be = u.nblk;
+        if (bf < be) {
+            u.b = bf;
+            u.bend = be;
+            u.nt = nt;
+            u.valid = true;
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ const float *slot_scales(const GemvP &p, int s, int nu)
+{
+    if (s < nu) {
+        int e = p.union_ids[s];
+        e = (e >= 0 && e < p.E) ? e : 0;
+        return p.s + (int64_t)e * p.s_stride;
+    }
+    return p.s_sh;
+}
+
+__device__ __forceinline__ const uint8_t *slot_weights(const GemvP &p, int s, int nu)
+{
+    if (s < nu) {
+        int e = p.union_ids[s];
+        e = (e >= 0 && e < p.E) ? e : 0;     // a bad index was flagged when the slot was costed
+        return p.w + (int64_t)e * p.w_stride;
+    }
+    return p.w_sh;
+}
+
+template <int WB, int NDIG, int TP, bool GATEUP>
+__global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const GemvP p)
+{
+    using LD = LaneDig<WB, NDIG>;
+    constexpr int NT = GvShape<WB, NDIG>::NT;
+    constexpr int R = GvShape<WB, NDIG>::R, V = R * TP, LV = Log2<V>::value;
+    constexpr int NWARPS = NT / 32;
+    constexpr int64_t BWU = NDIG == 1 ? 8 : 3;       // cost of streaming a block, in tokens
+    extern __shared__ __align__(128) unsigned char smem[];
+    const GvSmem M = p.sm;
+    unsigned char *ring = smem;
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + M.mbar);
+    int *cnt = reinterpret_cast<int *>(smem + M.cnt);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + M.abort);
+    unsigned char *dig = smem + M.dig;
+    float *red = reinterpret_cast<float *>(smem + M.red);
+    int *tin = reinterpret_cast<int *>(smem + M.tin);
+    int *tout = reinterpret_cast<int *>(smem + M.tout);
+    int64_t *pre = reinterpret_cast<int64_t *>(smem + M.pre);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int K = p.K, cpr = p.cpr;
     const int c = tid % cpr, team = tid / cpr, wit = c >> 5;
+    const RecLayout RL = p.rec;
 
-    // ---- cost-weighted partition of (slot, token group, row block) work units.
-    // A unit costs BWU (streaming its weights) + its token count (dot work);
-    // slot s has ceil(ntok/TS) groups, all full but the last, so its cost is
-    // nblk * (BWU * groups + ntok).  pre[] holds the prefix over slots; each
-    // CTA owns the units whose cost start falls in its equal share.
-    constexpr int64_t BWU = NDIG == 1 ? 8 : 3;
+    // gate/up reads the permutation and the activation records of the kernels
+    // before it; down only needs h after its weight stream has started.
+    if constexpr (GATEUP) {
+        pdl_wait();
+        pdl_trigger();
+    }
+    // ---- cost prefix over slots: a unit costs BWU + its token count; slot s
+    // has ceil(ntok/TS) groups (all full but the last): nblk * (BWU*groups + ntok).
     const int nu = p.routed ? *p.n_union : 0;
     const int nslots = nu + (p.shared ? 1 : 0);
     if (tid < 32) {
@@ -117,261 +512,252 @@ __global__ void __launch_bounds__(GV_NT, 1) k_ffn_gemv(const GemvP p)
             const int s = s0 + lane;
             int64_t cost = 0;
             if (s < nslots) {
-                int ntok = p.T;
                 if (s < nu) {
                     const int e = p.union_ids[s];
-                    ntok = (e >= 0 && e < p.E) ? p.offsets[e + 1] - p.offsets[e] : 0;
+                    if (e < 0 || e >= p.E) raise_status(DERR_BADIDX);
                 }
-                const int groups = (ntok + p.ts - 1) / p.ts;
-                cost = (int64_t)p.nblk * (BWU * groups + ntok);
+                const int ntok = slot_ntok(p, s, nu);
+                cost = (int64_t)p.nblk * (BWU * ((ntok + p.ts - 1) / p.ts) + ntok);
             }
             int64_t inc = cost;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int64_t n = __shfl_up_sync(0xffffffffu, inc, o);
-                if (lane >= o) inc += n;
+                const int64_t nb = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += nb;
             }
             if (s < nslots) pre[s] = run + inc - cost;
             run += __shfl_sync(0xffffffffu, inc, 31);
         }
         if (lane == 0) pre[nslots] = run;
     }
+    if (tid == 0) {
+        for (int st = 0; st < p.stages; ++st) {
+            mbar_init(smem_u32(&mbar[st]), 1);
+            cnt[st] = 0;
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
     __syncthreads();
     const int64_t Ctot = pre[nslots];
-    const int64_t c0 = Ctot * blockIdx.x / gridDim.x, c1 = Ctot * (blockIdx.x + 1) / gridDim.x;
-    int sfirst = 0;
+    Units cu;
+    cu.pre = pre;
+    cu.nslots = nslots;
+    cu.nu = nu;
+    cu.nblk = p.nblk;
+    cu.ts = p.ts;
+    cu.bwu = BWU;
+    cu.c0 = Ctot * blockIdx.x / gridDim.x;
+    cu.c1 = Ctot * (blockIdx.x + 1) / gridDim.x;
     {   // last slot whose prefix is <= c0
         int lo = 0, hi = nslots;
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (pre[mid] <= c0) lo = mid; else hi = mid;
+            if (pre[mid] <= cu.c0) lo = mid; else hi = mid;
         }
-        sfirst = lo;
+        cu.s = lo;
     }
-    int pass = 0;
+    cu.ntok = 0;
+    cu.W = nullptr;
+    cu.S = nullptr;
+    units_enter_slot(cu, p, cu.s);
+    cu.nt = 0;
+    cu.b = cu.bend = 0;
+    cu.valid = false;
+    units_advance(cu, p);
 
-    for (int s = sfirst; s < nslots && pre[s] < c1; ++s) {
-        int p0, ntok;
-        const uint8_t *W;
-        const float *S;
-        const bool is_routed = s < nu;
-        if (is_routed) {
-            const int e = p.union_ids[s];
-            if (e < 0 || e >= p.E) { if (tid == 0) raise_status(DERR_BADIDX); return; }
-            p0 = p.offsets[e];
-            ntok = p.offsets[e + 1] - p0;
-            W = p.w + (int64_t)e * p.w_stride;
-            S = p.s + (int64_t)e * p.s_stride;
-        } else {
-            p0 = 0;
-            ntok = p.T;
-            W = p.w_sh;
-            S = p.s_sh;
-        }
-        for (int tg = 0, j = 0; tg < ntok; tg += p.ts, ++j) {
-            const int nt = min(p.ts, ntok - tg);
-            const int64_t gstart = pre[s] + (int64_t)p.nblk * j * (BWU + p.ts);
-            const int64_t cb = BWU + nt;
-            int64_t bfirst = c0 > gstart ? (c0 - gstart + cb - 1) / cb : 0;
-            int64_t bend = c1 > gstart ? (c1 - gstart + cb - 1) / cb : 0;
-            if (bend > p.nblk) bend = p.nblk;
-            if (bfirst >= bend) continue;
-            __syncthreads();                       // previous group's readers are done
-            if (tid < nt) {
-                const int i = tg + tid;
+    // Every thread keeps a producer iterator `stages` units ahead of its own
+    // consumer iterator; the last warp to finish unit n refills its stage with
+    // unit n + stages.  Thread 0 issues the first `stages` units.
+    auto issue = [&](const Units &u, int stage) {
+        const int64_t row0 = u.b * (int64_t)p.rb;
+        const int64_t nrows = min((int64_t)p.rb, (int64_t)p.rows - row0);
+        const uint8_t *src = u.W + row0 * p.row_bytes;
+        const float *ssrc = u.S + row0;
+        unsigned char *dst = ring + (size_t)stage * M.stage_bytes;
+        const uint32_t mb = smem_u32(&mbar[stage]);
+        const uint32_t wbytes = (uint32_t)(nrows * p.row_bytes), sbytes = (uint32_t)(nrows * 4);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb),
+                     "r"(wbytes + sbytes)
+                     : "memory");
+        bulk_copy(smem_u32(dst), src, wbytes, mb);
+        bulk_copy(smem_u32(dst + M.scales_off), ssrc, sbytes, mb);
+    };
+    Units pu = cu;
+    for (int st = 0; st < p.stages && pu.valid; ++st) {
+        if (tid == 0) issue(pu, st);
+        units_advance(pu, p);
+    }
+    if constexpr (!GATEUP) {     // the weights are on their way; now wait for h
+        pdl_wait();
+        pdl_trigger();
+    }
+
+    int n = 0, cur_s = -1, cur_j = -1;
+    int p0 = 0, tout1 = 0;
+    bool is_routed = false;
+    LD dreg;
+    while (cu.valid) {
+        const int nt = cu.nt;
+        if (cu.s != cur_s || cu.j != cur_j) {
+            if (cu.s != cur_s) {
+                is_routed = cu.s < nu;
                 if (is_routed) {
-                    const int pos = p0 + i;
-                    tin[tid] = GATEUP ? p.sorted[pos] / p.k : pos;
-                    tout[tid] = pos;
+                    int e = p.union_ids[cu.s];
+                    e = (e >= 0 && e < p.E) ? e : 0;
+                    p0 = p.offsets[e];
                 } else {
-                    tin[tid] = GATEUP ? i : (int)p.sh_in_row0 + i;
-                    tout[tid] = (int)p.sh_out_row0 + i;
+                    p0 = 0;
                 }
             }
-            __syncthreads();
-            // ---- stage the tokens' activations as digit planes
-            unsigned char *digb = reinterpret_cast<unsigned char *>(dig);
-            for (int blk = warp; blk < nt * nb; blk += GV_NT / 32) {
-                const int i = blk / nb, bb = blk % nb;
-                const int elem = bb * 32 + lane;
-                const int64_t row = tin[i];
-                int8_t d[3] = {0, 0, 0};
-                float sig = 0.f;
-                if constexpr (NDIG == 1) {
-                    if constexpr (GATEUP) {
-                        d[0] = p.xq[row * K + elem];
-                        sig = p.xd[row * nb + bb];
+            const int tg = cu.j * p.ts;
+            if constexpr (TP == 1) {               // one token: its record straight from global
+                int row_in;
+                if (is_routed) {
+                    const int pos = p0 + tg;
+                    row_in = GATEUP ? p.sorted[pos] / p.k : pos;
+                    tout1 = pos;
+                } else {
+                    row_in = GATEUP ? tg : (int)p.sh_in_row0 + tg;
+                    tout1 = (int)p.sh_out_row0 + tg;
+                }
+                dreg.load(p.xrec + (size_t)row_in * RL.bytes, RL, c, K);
+            } else {
+                __syncthreads();                   // earlier readers of dig, tin, tout are done
+                if (*abort_flag) break;
+                if (tid < nt) {
+                    const int i = tg + tid;
+                    if (is_routed) {
+                        const int pos = p0 + i;
+                        tin[tid] = GATEUP ? p.sorted[pos] / p.k : pos;
+                        tout[tid] = pos;
                     } else {
-                        const float v = p.hin[row * p.hin_ld + elem];
-                        const float amax = warp_max(fabsf(v));
-                        if (amax != 0.f) {
-                            d[0] = (int8_t)q8_code(v, __fdiv_rn(127.f, amax));
-                            sig = __fdiv_rn(amax, 127.f);
-                        }
+                        tin[tid] = GATEUP ? i : (int)p.sh_in_row0 + i;
+                        tout[tid] = (int)p.sh_out_row0 + i;
+                    }
+                }
+                __syncthreads();
+                const int n16 = RL.bytes / 16;     // copy the group's records
+                for (int i = tid; i < nt * n16; i += NT) {
+                    const int t = i / n16, q = i % n16;
+                    reinterpret_cast<uint4 *>(dig + (size_t)t * RL.bytes)[q] =
+                        reinterpret_cast<const uint4 *>(p.xrec + (size_t)tin[t] * RL.bytes)[q];
+                }
+                __syncthreads();
+            }
+            cur_s = cu.s;
+            cur_j = cu.j;
+        }
+        const int stage = n % p.stages;
+        if (!mbar_wait(smem_u32(&mbar[stage]), (uint32_t)((n / p.stages) & 1))) {
+            *abort_flag = 1;
+            raise_status(DERR_TIMEOUT);
+            break;
+        }
+        const unsigned char *sbase = ring + (size_t)stage * M.stage_bytes;
+        const unsigned char *blk = sbase + (size_t)team * R * p.row_bytes + (size_t)c * 16;
+        float *rst = red + (size_t)stage * M.red_stage;
+        for (int t0 = 0; t0 < nt; t0 += TP) {
+            float part[V];
+#pragma unroll
+            for (int tt = 0; tt < TP; ++tt) {
+                if (t0 + tt < nt) {
+                    if constexpr (TP == 1) {
+                        uint4 wv[R];
+#pragma unroll
+                        for (int r = 0; r < R; ++r)
+                            wv[r] = *reinterpret_cast<const uint4 *>(blk + (size_t)r * p.row_bytes);
+#pragma unroll
+                        for (int r = 0; r < R; ++r) part[r] = dreg.dot(wv[r]);
+                    } else {
+                        LD d;
+                        d.load(dig + (size_t)(t0 + tt) * RL.bytes, RL, c, K);
+#pragma unroll
+                        for (int r = 0; r < R; ++r)
+                            part[r * TP + tt] =
+                                d.dot(*reinterpret_cast<const uint4 *>(blk + (size_t)r * p.row_bytes));
                     }
                 } else {
-                    float v;
-                    if constexpr (GATEUP) {
-                        if (p.afmt == QRX_A_BF16)
-                            v = __bfloat162float(
-                                reinterpret_cast<const __nv_bfloat16 *>(p.x)[row * K + elem]);
-                        else
-                            v = reinterpret_cast<const float *>(p.x)[row * K + elem];
-                    } else {
-                        v = p.hin[row * p.hin_ld + elem];
-                        if (p.afmt == QRX_A_BF16) v = __bfloat162float(__float2bfloat16_rn(v));
-                    }
-                    const float amax = warp_max(fabsf(v));
-                    if (amax != 0.f) {
-                        const int sh = fixed_shift(amax);
-                        split3(__float2int_rn(ldexpf(v, sh)), d[0], d[1], d[2]);
-                        sig = ldexpf(1.f, -sh);
-                    }
-                }
-                const int cc = elem / F::EPC, l = elem % F::EPC;
-                int wd, by;
-                digit_slot<WB>(l, wd, by);
 #pragma unroll
-                for (int pl = 0; pl < NDIG; ++pl)
-                    digb[((((size_t)i * NDIG + pl) * cpr + cc) * F::DW + wd) * 4 + by] =
-                        (unsigned char)d[pl];
-                if (lane == 0) bsc[i * nb + bb] = sig;
+                    for (int r = 0; r < R; ++r) part[r * TP + tt] = 0.f;
+                }
             }
-            __syncthreads();
-
-            // ---- this group's blocks in my range
-            for (int64_t bb = bfirst; bb < bend; ++bb) {
-                const int rblk = (int)bb;
-                const int rowbase = rblk * p.rb + team * R;
-                uint4 wv[R];
+            // warp partials of this pass -> rst[token][team][wit][row]
+            if (cpr >= 32) {
+                const float tot = warp_tr_reduce<V>(part, lane);
+                const int vi = lane >> (5 - LV);
+                const int r = vi / TP, tt = vi % TP;
+                if ((lane & ((1 << (5 - LV)) - 1)) == 0 && t0 + tt < nt)
+                    rst[(((t0 + tt) * p.tpc + team) * p.wpt + wit) * R + r] = tot;
+            } else {
 #pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const int row = rowbase + r;
-                    wv[r] = row < p.rows
-                                ? ld_stream16(W + (int64_t)row * p.row_bytes + (int64_t)c * 16)
-                                : make_uint4(0u, 0u, 0u, 0u);
-                }
-                for (int t0 = 0; t0 < nt; t0 += TP) {
-                    float part[V];
-#pragma unroll
-                    for (int tt = 0; tt < TP; ++tt) {
-                        if (t0 + tt < nt) {
-                            const int ti = t0 + tt;
-                            uint32_t dw[NDIG][F::DW];
-#pragma unroll
-                            for (int pl = 0; pl < NDIG; ++pl) {
-                                const uint4 *src = reinterpret_cast<const uint4 *>(
-                                    dig + (((size_t)ti * NDIG + pl) * cpr + c) * F::DW);
-#pragma unroll
-                                for (int q4 = 0; q4 < F::DW / 4; ++q4) {
-                                    const uint4 v4 = src[q4];
-                                    dw[pl][4 * q4 + 0] = v4.x;
-                                    dw[pl][4 * q4 + 1] = v4.y;
-                                    dw[pl][4 * q4 + 2] = v4.z;
-                                    dw[pl][4 * q4 + 3] = v4.w;
-                                }
-                            }
-                            float sig[NBC];
-                            int corr[NBC][NDIG];
-#pragma unroll
-                            for (int bc = 0; bc < NBC; ++bc) {
-                                const int sb = WB == 8 ? (c >> 1) : (WB == 4 ? c : 2 * c + bc);
-                                sig[bc] = bsc[ti * nb + sb];
-#pragma unroll
-                                for (int pl = 0; pl < NDIG; ++pl) {
-                                    int sum = 0;
-                                    if constexpr (F::OFF != 0) {
-                                        constexpr int WPB = F::DW / NBC;
-#pragma unroll
-                                        for (int q = 0; q < WPB; ++q)
-                                            sum = dp4a(dw[pl][bc * WPB + q], 0x01010101u, sum);
-                                    }
-                                    corr[bc][pl] = -F::OFF * sum;
-                                }
-                            }
-#pragma unroll
-                            for (int r = 0; r < R; ++r) {
-                                int acc[NBC][NDIG];
-#pragma unroll
-                                for (int bc = 0; bc < NBC; ++bc)
-#pragma unroll
-                                    for (int pl = 0; pl < NDIG; ++pl) acc[bc][pl] = corr[bc][pl];
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    uint32_t u[F::UPW];
-                                    unpack_word<WB>(word_of(wv[r], i), u);
-                                    const int bc = WB == 2 ? (i >> 1) : 0;
-#pragma unroll
-                                    for (int j = 0; j < F::UPW; ++j)
-#pragma unroll
-                                        for (int pl = 0; pl < NDIG; ++pl)
-                                            acc[bc][pl] = dp4a(u[j], dw[pl][i * F::UPW + j], acc[bc][pl]);
-                                }
-                                float v = 0.f;
-#pragma unroll
-                                for (int bc = 0; bc < NBC; ++bc) {
-                                    float cv;
-                                    if constexpr (NDIG == 3)
-                                        cv = fmaf(__int2float_rn(acc[bc][2]), 65536.f,
-                                                  __int2float_rn(acc[bc][0] + 256 * acc[bc][1]));
-                                    else
-                                        cv = __int2float_rn(acc[bc][0]);
-                                    v = fmaf(sig[bc], cv, v);
-                                }
-                                part[r * TP + tt] = v;
-                            }
-                        } else {
-#pragma unroll
-                            for (int r = 0; r < R; ++r) part[r * TP + tt] = 0.f;
-                        }
-                    }
-                    // ---- reduce over the team
-                    float *rbuf = red + (pass & 1) * p.redn;
-                    if (cpr >= 32) {
-                        const float tot = warp_tr_reduce<V>(part, lane);
-                        if ((lane & ((1 << (5 - LV)) - 1)) == 0)
-                            rbuf[(team * p.wpt + wit) * V + (lane >> (5 - LV))] = tot;
-                    } else {
-#pragma unroll
-                        for (int vi = 0; vi < V; ++vi) {
-                            float xv = part[vi];
-                            for (int o = cpr >> 1; o; o >>= 1) xv += __shfl_xor_sync(0xffffffffu, xv, o);
-                            if (c == 0) rbuf[team * V + vi] = xv;
-                        }
-                    }
-                    __syncthreads();
-                    // ---- finalize: scales, SwiGLU, store
-                    if constexpr (GATEUP) {
-                        const int per_team = (R / 2) * TP;
-                        for (int f = tid; f < p.tpc * per_team; f += GV_NT) {
-                            const int tf = f / per_team, rem = f % per_team;
-                            const int q = rem / TP, tt = rem % TP;
-                            const int row_g = rblk * p.rb + tf * R + 2 * q;
-                            if (t0 + tt >= nt || row_g >= p.rows) continue;
-                            float G = 0.f, U = 0.f;
-                            for (int w2 = 0; w2 < p.wpt; ++w2) {
-                                G += rbuf[(tf * p.wpt + w2) * V + (2 * q) * TP + tt];
-                                U += rbuf[(tf * p.wpt + w2) * V + (2 * q + 1) * TP + tt];
-                            }
-                            const float g = S[row_g] * G, u = S[row_g + 1] * U;
-                            p.out[(int64_t)tout[t0 + tt] * p.out_ld + (row_g >> 1)] = silu_mul(g, u);
-                        }
-                    } else {
-                        const int per_team = R * TP;
-                        for (int f = tid; f < p.tpc * per_team; f += GV_NT) {
-                            const int tf = f / per_team, rem = f % per_team;
-                            const int r = rem / TP, tt = rem % TP;
-                            const int row = rblk * p.rb + tf * R + r;
-                            if (t0 + tt >= nt || row >= p.rows) continue;
-                            float Y = 0.f;
-                            for (int w2 = 0; w2 < p.wpt; ++w2) Y += rbuf[(tf * p.wpt + w2) * V + r * TP + tt];
-                            p.out[(int64_t)tout[t0 + tt] * p.out_ld + row] = S[row] * Y;
-                        }
-                    }
-                    ++pass;
+                for (int vi = 0; vi < V; ++vi) {
+                    float xv = part[vi];
+                    for (int o = cpr >> 1; o; o >>= 1) xv += __shfl_xor_sync(0xffffffffu, xv, o);
+                    const int r = vi / TP, tt = vi % TP;
+                    if (c == 0 && t0 + tt < nt) rst[((t0 + tt) * p.tpc + team) * R + r] = xv;
                 }
             }
         }
+        // ---- arrive; the last warp of this unit finalizes it and refills the stage
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+            __threadfence_block();
+            last = atomicAdd(&cnt[stage], 1) == NWARPS - 1;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+            __threadfence_block();
+            const float *scl = reinterpret_cast<const float *>(sbase + M.scales_off);
+            const int rblk = (int)cu.b;
+            if constexpr (GATEUP) {
+                const int per = p.tpc * (R / 2);
+                for (int f = lane; f < nt * per; f += 32) {
+                    const int t = f / per, rem = f % per;
+                    const int tf = rem / (R / 2), q = rem % (R / 2);
+                    const int lrow = tf * R + 2 * q;
+                    const int row_g = rblk * p.rb + lrow;
+                    if (row_g >= p.rows) continue;
+                    const float *src = rst + ((t * p.tpc + tf) * p.wpt) * R;
+                    float G = 0.f, U = 0.f;
+                    for (int w2 = 0; w2 < p.wpt; ++w2) {
+                        G += src[w2 * R + 2 * q];
+                        U += src[w2 * R + 2 * q + 1];
+                    }
+                    const int orow = TP == 1 ? tout1 : tout[t];
+                    p.out[(int64_t)orow * p.out_ld + (row_g >> 1)] =
+                        silu_mul(scl[lrow] * G, scl[lrow + 1] * U);
+                }
+            } else {
+                const int per = p.tpc * R;
+                for (int f = lane; f < nt * per; f += 32) {
+                    const int t = f / per, lrow = f % per;
+                    const int tf = lrow / R, r = lrow % R;
+                    const int row = rblk * p.rb + lrow;
+                    if (row >= p.rows) continue;
+                    const float *src = rst + ((t * p.tpc + tf) * p.wpt) * R;
+                    float Y = 0.f;
+                    for (int w2 = 0; w2 < p.wpt; ++w2) Y += src[w2 * R + r];
+                    const int orow = TP == 1 ? tout1 : tout[t];
+                    p.out[(int64_t)orow * p.out_ld + row] = scl[lrow] * Y;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                cnt[stage] = 0;
+                if (pu.valid) issue(pu, stage);
+            }
+        }
+        units_advance(pu, p);
+        ++n;
+        units_advance(cu, p);
+    }
+    if (*abort_flag && tid == 0) {
+        // a wait gave up: wait (bounded) for this CTA's copies still in flight
+        for (int m = n; m < n + p.stages; ++m)
+            mbar_wait(smem_u32(&mbar[m % p.stages]), (uint32_t)((m / p.stages) & 1));
     }
 }
 
@@ -382,39 +768,49 @@ struct GemvPlan {
     int tp;
 };
 
-static inline int gemv_smem_limit() { return 200 * 1024; }
-
-// Fill geometry for a matrix of `rows` x `K` codes at `wbits`, for slots of
-// at most `maxtok` tokens with NDIG digit planes.
+// Geometry for a matrix of `rows` x `K` codes at `wbits`, slots of at most
+// `maxtok` tokens, NDIG digit planes.  Picks the deepest weight ring and the
+// largest token group that fit in shared memory.
 static inline bool gemv_plan(GemvPlan &pl, int wbits, int ndig, int K, int rows, int maxtok,
                              int maxslots)
 {
     GemvP &p = pl.p;
+    const int NT = GvShape<4, 3>::NT;
+    const int R = GV_BLK / (NT * 16);
+    p.nthreads = NT;
     p.K = K;
     p.rows = rows;
     p.row_bytes = K * wbits / 8;
     p.cpr = p.row_bytes / 16;
-    if (p.cpr <= 0 || GV_NT % p.cpr != 0) return false;
+    if (p.cpr <= 0 || p.row_bytes % 16 != 0 || NT % p.cpr != 0) return false;
     if (p.cpr < 32 && (32 % p.cpr) != 0) return false;
     if (p.cpr > 32 && (p.cpr % 32) != 0) return false;
-    p.tpc = GV_NT / p.cpr;
-    p.rb = p.tpc * GV_R;
+    p.tpc = NT / p.cpr;
+    p.rb = p.tpc * R;
     p.nblk = (rows + p.rb - 1) / p.rb;
     p.wpt = p.cpr >= 32 ? p.cpr / 32 : 1;
+    if (p.rb * 4 % 16 != 0) return false;
     pl.tp = maxtok <= 1 ? 1 : (ndig == 1 ? 4 : 2);
-    const int V = GV_R * pl.tp;
-    p.redn = p.tpc * p.wpt * V;
-    const size_t fixed = (size_t)2 * p.redn * 4 + 64 + (size_t)8 * (maxslots + 2);
-    const size_t per_tok = (size_t)ndig * K + (size_t)(K / 32) * 4 + 8;
-    const size_t lim = (size_t)gemv_smem_limit();
-    if (fixed + per_tok > lim) return false;
-    int ts = (int)((lim - fixed) / per_tok);
-    if (ts > maxtok) ts = maxtok;
-    if (ts < 1) ts = 1;
-    p.ts = ts;
-    pl.smem = (size_t)ts * ndig * K + (size_t)ts * (K / 32) * 4 + (size_t)2 * p.redn * 4 +
-              (size_t)2 * (ts + 1) * 4 + (size_t)8 * (maxslots + 2);
-    return true;
+    p.rec = rec_layout(ndig, K);
+    p.maxslots = maxslots;
+    const int tries[3] = {4, 3, 2};
+    for (int i = (maxtok <= 1 ? 0 : 1); i < 3; ++i) {
+        const int stages = tries[i];
+        auto total = [&](int ts) {
+            return gv_smem(stages, ts, p.rec.bytes, p.rb, p.tpc, p.wpt, R, maxslots).total;
+        };
+        if (total(1) > GV_SMEM_MAX) continue;
+        int ts = maxtok;
+        const int per = total(2) - total(1);
+        if (total(1) + (int64_t)(ts - 1) * per > GV_SMEM_MAX) ts = 1 + (GV_SMEM_MAX - total(1)) / per;
+        while (ts > 1 && total(ts) > GV_SMEM_MAX) --ts;
+        p.stages = stages;
+        p.ts = ts;
+        p.sm = gv_smem(stages, ts, p.rec.bytes, p.rb, p.tpc, p.wpt, R, maxslots);
+        pl.smem = (size_t)p.sm.total;
+        return true;
+    }
+    return false;
 }
 
 template <int WB, int NDIG, int TP, bool GU>
@@ -426,13 +822,11 @@ static cudaError_t gemv_go(const GemvPlan &pl, int grid, cudaStream_t st)
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev >= 64 || !(configured >> dev & 1ull)) {
-        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   gemv_smem_limit() + 4096);
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_MAX);
         if (err != cudaSuccess) return err;
         if (dev < 64) configured |= 1ull << dev;
     }
-    kern<<<grid, GV_NT, pl.smem, st>>>(pl.p);
-    return cudaGetLastError();
+    return launch_k(kern, dim3(grid), dim3(GvShape<WB, NDIG>::NT), pl.smem, st, pl.p);
 }
 
 template <bool GU>
@@ -459,9 +853,26 @@ static inline void gemv_common(GemvP &p, const FfnArgs &a)
     p.k = a.k;
     p.T = a.T;
     p.afmt = a.afmt;
-    p.x = a.x;
-    p.xq = a.xq;
-    p.xd = a.xd;
+}
+
+// Bytes of the digit records of `rows` activation rows of length K.
+static inline size_t act_records_bytes(int afmt, int K, int rows)
+{
+    return (size_t)rows * rec_layout(afmt == QRX_A_Q8_0 ? 1 : 3, K).bytes;
+}
+
+cudaError_t launch_act_digits(const FfnArgs &a, cudaStream_t st)
+{
+    const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
+    const int64_t warps = (int64_t)a.T * (a.H / 32);
+    const unsigned grid = (unsigned)((warps + 7) / 8);
+#define QRX_AD(WB, ND) \
+    if (a.wbits == WB && ndig == ND) \
+        return launch_k(k_act_digits<WB, ND>, dim3(grid), dim3(256), 0, st, a.x, a.xq, a.xd, a.afmt, \
+                        a.T, a.H, a.xrec);
+    QRX_AD(4, 3) QRX_AD(4, 1) QRX_AD(8, 3) QRX_AD(8, 1) QRX_AD(2, 3) QRX_AD(2, 1)
+#undef QRX_AD
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
@@ -469,6 +880,10 @@ cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
     const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
     GemvPlan pl;
     if (!gemv_plan(pl, a.wbits, ndig, a.H, 2 * a.I, a.T, a.E + 1)) return cudaErrorInvalidValue;
+    if (a.prep_records) {
+        const cudaError_t err = launch_act_digits(a, st);
+        if (err != cudaSuccess) return err;
+    }
     GemvP &p = pl.p;
     gemv_common(p, a);
     p.w = a.w13;
@@ -477,8 +892,7 @@ cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
     p.s_stride = (int64_t)2 * a.I;
     p.w_sh = a.w13_sh;
     p.s_sh = a.s13_sh;
-    p.hin = nullptr;
-    p.hin_ld = 0;
+    p.xrec = a.xrec;
     p.sh_in_row0 = 0;
     p.out = a.h;
     p.out_ld = a.h_ld;
@@ -499,8 +913,21 @@ cudaError_t launch_ffn_down(const FfnArgs &a, int num_sms, cudaStream_t st)
     p.s_stride = a.H;
     p.w_sh = a.w2_sh;
     p.s_sh = a.s2_sh;
-    p.hin = a.h;
-    p.hin_ld = a.h_ld;
+    // h rows -> digit records (all rows the down projection reads)
+    const int hrows = max(a.routed ? a.T * a.k : 0, a.shared ? (int)a.sh_h_row0 + a.T : 0);
+    {
+        const int64_t warps = (int64_t)hrows * (a.I / 32);
+        const unsigned grid = (unsigned)((warps + 7) / 8);
+        cudaError_t err = cudaErrorInvalidValue;
+#define QRX_HD(WB, ND) \
+        if (a.wbits == WB && ndig == ND) \
+            err = launch_k(k_h_digits<WB, ND>, dim3(grid), dim3(256), 0, st, (const float *)a.h, a.h_ld, \
+                           hrows, a.I, a.afmt, a.hrec);
+        QRX_HD(4, 3) QRX_HD(4, 1) QRX_HD(8, 3) QRX_HD(8, 1) QRX_HD(2, 3) QRX_HD(2, 1)
+#undef QRX_HD
+        if (err != cudaSuccess) return err;
+    }
+    p.xrec = a.hrec;
     p.sh_in_row0 = a.sh_h_row0;
     p.out = a.y;
     p.out_ld = a.y_ld;

@@ -55,6 +55,8 @@ __global__ void __launch_bounds__(1024, 1) k_permute(const int32_t *__restrict__
     int *whist = psm;                          // [PERM_WARPS][E]
     int *tmp = psm + PERM_WARPS * E;           // [33]
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    pdl_wait();
+    pdl_trigger();
     for (int i = tid; i < PERM_WARPS * E; i += 1024) whist[i] = 0;
     __syncthreads();
 
@@ -128,8 +130,7 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const qrx_pe
                                                (int)smem);
         if (err != cudaSuccess) return err;
     }
-    k_permute<<<1, 1024, smem, st>>>(idx, T * k, E, p);
-    return cudaGetLastError();
+    return launch_k(k_permute, dim3(1), dim3(1024), smem, st, idx, T * k, E, p);
 }
 
 }  // namespace qrx

@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(256) k_quantize_act_q8(const float *__restrict
                                                          float *__restrict__ xd)
 {
     const int lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_trigger();
     const int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (b >= nblocks) return;
     const float v = x[b * 32 + lane];

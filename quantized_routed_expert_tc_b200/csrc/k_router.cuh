@@ -7,10 +7,12 @@
 // the k largest biased scores among their experts are chosen; weights are the
 // unbiased scores renormalised over the choice and scaled by rsf.
 //
-// Two kernels: k_router_partial computes split-K partial dot products in
-// double (tiles of 32 tokens x 64 experts, K split so that the grid fills the
-// GPU even at one token); k_router_select sums the partials in split order,
-// rounds the logit to f32 and selects, one warp per token.
+// Logits are summed in double and rounded to f32 once.  Few tokens
+// (T <= 64): k_router_gemv, two experts per CTA, each expert's row split over
+// four warps that keep their quarter of the row in registers and run every
+// token over it.  More tokens: k_router_tile, 32-token x 64-expert tiles
+// staged in shared memory.  Then k_router_select, one warp per token: sigmoid,
+// bias, group scores, group choice, top-k and weights.
 #pragma once
 #include "qrx_dev.cuh"
 
@@ -18,16 +20,85 @@ namespace qrx {
 
 constexpr int RT_T = 32, RT_E = 64, RT_KC = 32;
 
+constexpr int RG_ROWS = 2;           // experts per CTA in k_router_gemv
+constexpr int RG_TMAX = 64;          // tokens handled by k_router_gemv
+
 template <bool XBF16>
-__global__ void __launch_bounds__(256) k_router_partial(RouterArgs a, int kchunks_per_split)
+__device__ __forceinline__ float4 load_x4(const void *x, int64_t off)
+{
+    if constexpr (XBF16) {
+        const uint2 raw = *reinterpret_cast<const uint2 *>(
+            reinterpret_cast<const __nv_bfloat16 *>(x) + off);
+        const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&raw.x);
+        const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&raw.y);
+        const float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
+        return make_float4(a.x, a.y, b.x, b.y);
+    } else {
+        return *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(x) + off);
+    }
+}
+
+// Few tokens: warp (row r, quarter q) holds Wr[r][q*H/4 .. (q+1)*H/4) in
+// registers (float4 per lane, at most RG_W4 of them) and dots every token's
+// matching quarter of x with it in double.
+constexpr int RG_W4 = 12;            // float4 per lane: H/16/32 <= 12 -> H <= 6144
+
+template <bool XBF16>
+__global__ void __launch_bounds__(256) k_router_gemv(RouterArgs a)
+{
+    __shared__ double part[RG_ROWS][4][RG_TMAX];
+    pdl_trigger();                       // reads only inputs; waits before it exits
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int rl = w >> 2, q = w & 3;
+    const int e = blockIdx.x * RG_ROWS + rl;
+    const int n4 = a.H / 16;                 // float4 per quarter
+    const int64_t k0 = (int64_t)q * (a.H / 4);
+    float4 wv[RG_W4];
+#pragma unroll
+    for (int j = 0; j < RG_W4; ++j) {
+        const int i4 = lane + 32 * j;
+        wv[j] = (e < a.E && i4 < n4)
+                    ? *reinterpret_cast<const float4 *>(a.Wr + (int64_t)e * a.H + k0 + 4 * i4)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int t = 0; t < a.T; ++t) {
+        double acc = 0.0;
+#pragma unroll
+        for (int j = 0; j < RG_W4; ++j) {
+            const int i4 = lane + 32 * j;
+            if (i4 < n4) {
+                const float4 xv = load_x4<XBF16>(a.x, (int64_t)t * a.H + k0 + 4 * i4);
+                acc = fma((double)xv.x, (double)wv[j].x, acc);
+                acc = fma((double)xv.y, (double)wv[j].y, acc);
+                acc = fma((double)xv.z, (double)wv[j].z, acc);
+                acc = fma((double)xv.w, (double)wv[j].w, acc);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) part[rl][q][t] = acc;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < RG_ROWS * a.T; i += blockDim.x) {
+        const int r = i / a.T, t = i % a.T;
+        const int ee = blockIdx.x * RG_ROWS + r;
+        if (ee < a.E)
+            a.logits[(int64_t)t * a.E + ee] =
+                (float)(((part[r][0][t] + part[r][1][t]) + part[r][2][t]) + part[r][3][t]);
+    }
+    pdl_wait();
+}
+
+// Many tokens: 32-token x 64-expert tiles, K in chunks of 32 through shared memory.
+template <bool XBF16>
+__global__ void __launch_bounds__(256) k_router_tile(RouterArgs a)
 {
     __shared__ double xs[RT_T][RT_KC + 1];
     __shared__ double wsm[RT_E][RT_KC + 1];
+    pdl_trigger();                       // reads only inputs; waits before it exits
     const int tid = threadIdx.x;
-    const int e0 = blockIdx.x * RT_E, t0 = blockIdx.y * RT_T, ks = blockIdx.z;
-    const int nchunks = a.H / RT_KC;
-    const int c0 = ks * kchunks_per_split;
-    const int c1 = min(nchunks, c0 + kchunks_per_split);
+    const int e0 = blockIdx.x * RT_E, t0 = blockIdx.y * RT_T;
+    const int c0 = 0, c1 = a.H / RT_KC;
     const int tx = tid & 15, ty = tid >> 4;
     double acc[2][4];
 #pragma unroll
@@ -80,8 +151,9 @@ __global__ void __launch_bounds__(256) k_router_partial(RouterArgs a, int kchunk
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int t = t0 + ty + 16 * i, e = e0 + tx + 16 * j;
-            if (t < a.T && e < a.E) a.partial[((int64_t)ks * a.T + t) * a.E + e] = acc[i][j];
+            if (t < a.T && e < a.E) a.logits[(int64_t)t * a.E + e] = (float)acc[i][j];
         }
+    pdl_wait();
 }
 
 // One warp per token.  Dynamic shared memory per warp: s[E], sc[E] (f32),
@@ -97,12 +169,12 @@ __global__ void __launch_bounds__(256) k_router_select(RouterArgs a)
     float *sc_s = s_s + E;
     float *gsc = sc_s + E;
     int *kept = reinterpret_cast<int *>(gsc + G);
+    pdl_wait();
+    pdl_trigger();
     if (t >= a.T) return;
 
     for (int e = lane; e < E; e += 32) {
-        double acc = 0.0;
-        for (int ks = 0; ks < a.KS; ++ks) acc += a.partial[((int64_t)ks * a.T + t) * E + e];
-        const float lg = (float)acc;
+        const float lg = a.logits[(int64_t)t * E + e];
         const float s = (float)(1.0 / (1.0 + exp(-(double)lg)));
         s_s[e] = s;
         sc_s[e] = __fadd_rn(s, a.bias[e]);
@@ -164,25 +236,17 @@ __global__ void __launch_bounds__(256) k_router_select(RouterArgs a)
     }
 }
 
-int router_ksplit(int T, int H, int E, int num_sms)
-{
-    const int nchunks = H / RT_KC;
-    const int base = ((E + RT_E - 1) / RT_E) * ((T + RT_T - 1) / RT_T);
-    int want = (2 * num_sms + base - 1) / base;
-    if (want < 1) want = 1;
-    int cps = nchunks / want;
-    if (cps < 1) cps = 1;
-    return (nchunks + cps - 1) / cps;
-}
-
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t st)
 {
-    const int nchunks = a.H / RT_KC;
-    const int cps = (nchunks + a.KS - 1) / a.KS;
-    dim3 grid((a.E + RT_E - 1) / RT_E, (a.T + RT_T - 1) / RT_T, a.KS);
-    if (a.x_bf16) k_router_partial<true><<<grid, 256, 0, st>>>(a, cps);
-    else k_router_partial<false><<<grid, 256, 0, st>>>(a, cps);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err;
+    if (a.T <= RG_TMAX && a.H <= 16 * 32 * RG_W4) {
+        const unsigned grid = (unsigned)((a.E + RG_ROWS - 1) / RG_ROWS);
+        err = launch_k(a.x_bf16 ? k_router_gemv<true> : k_router_gemv<false>, dim3(grid), dim3(256), 0,
+                       st, a);
+    } else {
+        dim3 grid((a.E + RT_E - 1) / RT_E, (a.T + RT_T - 1) / RT_T);
+        err = launch_k(a.x_bf16 ? k_router_tile<true> : k_router_tile<false>, grid, dim3(256), 0, st, a);
+    }
     if (err != cudaSuccess) return err;
     const size_t smem = (size_t)8 * (2 * a.E + 2 * a.G) * 4;
     if (smem > 48 * 1024) {
@@ -190,8 +254,7 @@ cudaError_t launch_router(const RouterArgs &a, cudaStream_t st)
                                    (int)smem);
         if (err != cudaSuccess) return err;
     }
-    k_router_select<<<(a.T + 7) / 8, 256, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_k(k_router_select, dim3((a.T + 7) / 8), dim3(256), smem, st, a);
 }
 
 }  // namespace qrx

@@ -21,10 +21,17 @@
 
 using namespace qrx;
 
+thread_local bool qrx::g_pdl = false;
+
 namespace {
 
+// Sets the programmatic-dependent-launch switch for the launches in its scope.
+struct PdlScope {
+    explicit PdlScope(bool on) { g_pdl = on; }
+    ~PdlScope() { g_pdl = false; }
+};
+
 constexpr int kMaxDevices = 64;
-constexpr int kMaxSmsForSizing = 256;   // workspace sizing bound on SMs per device
 
 int num_sms_current()
 {
@@ -54,7 +61,8 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 // Workspace regions for T tokens.
 struct Ws {
-    size_t partial, counts, offsets, sorted, inv, uids, nu, xq, xd, h, y, xdev, outdev, idx, w, total;
+    size_t logits, counts, offsets, sorted, inv, uids, nu, xq, xd, xrec, hrec, h, y, xdev, outdev,
+        idx, w, total;
 };
 
 Ws ws_layout(const qrx_cfg *c, int T)
@@ -68,8 +76,7 @@ Ws ws_layout(const qrx_cfg *c, int T)
         off = align256(off + bytes);
         return at;
     };
-    const int KS = router_ksplit(T, (int)H, (int)E, kMaxSmsForSizing);
-    L.partial = take((size_t)KS * T * E * sizeof(double));
+    L.logits = take((size_t)T * E * sizeof(float));
     L.counts = take(E * 4);
     L.offsets = take((E + 1) * 4);
     L.sorted = take(A * 4);
@@ -78,6 +85,8 @@ Ws ws_layout(const qrx_cfg *c, int T)
     L.nu = take(4);
     L.xq = take((size_t)T * H);
     L.xd = take((size_t)T * (H / 32) * 4);
+    L.xrec = take(act_records_bytes(c->afmt, (int)H, T));
+    L.hrec = take(act_records_bytes(c->afmt, (int)I, (int)(A + T)));
     L.h = take((size_t)(A + T) * I * 4);
     L.y = take((size_t)(A + T) * H * 4);
     L.xdev = take((size_t)T * H * 4);
@@ -117,7 +126,8 @@ int check_ws(const qrx_cfg *c, int T, void *ws, size_t ws_bytes)
 int check_experts(const qrx_experts *x)
 {
     if (!x || !x->w13 || !x->s13 || !x->w2 || !x->s2) return QRX_EINVAL;
-    if (!aligned(x->w13, 16) || !aligned(x->w2, 16)) return QRX_EINVAL;
+    if (!aligned(x->w13, 16) || !aligned(x->w2, 16) || !aligned(x->s13, 16) || !aligned(x->s2, 16))
+        return QRX_EINVAL;
     return QRX_OK;
 }
 
@@ -281,8 +291,7 @@ int qrx_route(const qrx_cfg *c, const void *x, int32_t T, const float *Wr, const
     a.Gk = c->topk_group;
     a.k = c->top_k;
     a.rsf = c->routed_scaling_factor;
-    a.partial = at<double>(ws, L.partial);
-    a.KS = router_ksplit(T, a.H, a.E, num_sms_current());
+    a.logits = at<float>(ws, L.logits);
     a.idx = topk_idx;
     a.w = topk_w;
     return cuda_code(launch_router(a, (cudaStream_t)stream));
@@ -311,6 +320,9 @@ int qrx_expert_ffn(const qrx_cfg *c, const qrx_experts *routed, const qrx_perm *
     set_act(a, act);
     set_routed(a, routed, perm);
     a.h = h_sorted ? h_sorted : at<float>(ws, L.h);
+    a.xrec = at<unsigned char>(ws, L.xrec);
+    a.hrec = at<unsigned char>(ws, L.hrec);
+    a.prep_records = 1;
     a.h_ld = c->inter;
     a.y = y_sorted;
     a.y_ld = c->hidden;
@@ -332,6 +344,7 @@ int qrx_expert_down(const qrx_cfg *c, const qrx_experts *routed, const qrx_perm 
     if ((v = check_ws(c, T, ws, ws_bytes))) return v;
     FfnArgs a = ffn_args(c, T);
     set_routed(a, routed, perm);
+    a.hrec = at<unsigned char>(ws, ws_layout(c, T).hrec);
     a.h = const_cast<float *>(h_sorted);
     a.h_ld = c->inter;
     a.y = y_sorted;
@@ -352,6 +365,9 @@ int qrx_shared_ffn(const qrx_cfg *c, const qrx_experts *shared, const qrx_act *a
     set_act(a, act);
     set_shared(a, shared);
     a.h = h_sh ? h_sh : at<float>(ws, L.h);
+    a.xrec = at<unsigned char>(ws, L.xrec);
+    a.hrec = at<unsigned char>(ws, L.hrec);
+    a.prep_records = 1;
     a.h_ld = c->inter;
     a.y = y_sh;
     a.y_ld = c->hidden;
@@ -399,28 +415,26 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     const int sms = num_sms_current();
     const int64_t A = (int64_t)T * c->top_k;
 
+    // 1. activation records (reads only x; ordinary stream order with what came before)
+    FfnArgs a = ffn_args(c, T);
+    a.x = x;                      // Q8_0: the records kernel quantises x itself
+    a.xrec = at<unsigned char>(ws, L.xrec);
+    a.hrec = at<unsigned char>(ws, L.hrec);
     if (!mark(0)) return QRX_ECUDA;
+    cudaError_t e = launch_act_digits(a, st);
+    if (e != cudaSuccess || !mark(1)) return QRX_ECUDA;
+    // 2.. the rest chained with programmatic dependent launch
+    PdlScope pdl(true);
     if ((v = qrx_route(c, x, T, Wr, bias, topk_idx, topk_w, ws, ws_bytes, stream))) return v;
-    if (!mark(1)) return QRX_ECUDA;
+    if (!mark(2)) return QRX_ECUDA;
     qrx_perm perm{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.sorted),
                   at<int32_t>(ws, L.inv), at<int32_t>(ws, L.uids), at<int32_t>(ws, L.nu)};
-    cudaError_t e = launch_permute(topk_idx, T, c->top_k, c->n_experts, perm, st);
-    if (e != cudaSuccess || !mark(2)) return QRX_ECUDA;
-
-    qrx_act act{x, nullptr, nullptr};
-    if (c->afmt == QRX_A_Q8_0) {
-        act.xq = at<int8_t>(ws, L.xq);
-        act.xd = at<float>(ws, L.xd);
-        e = launch_quantize_act_q8(static_cast<const float *>(x), (int64_t)T * c->hidden / 32,
-                                   const_cast<int8_t *>(act.xq), const_cast<float *>(act.xd), st);
-        if (e != cudaSuccess) return QRX_ECUDA;
-    }
-    if (!mark(3)) return QRX_ECUDA;
+    e = launch_permute(topk_idx, T, c->top_k, c->n_experts, perm, st);
+    if (e != cudaSuccess || !mark(3)) return QRX_ECUDA;
     float *h = at<float>(ws, L.h), *y = at<float>(ws, L.y);
-    FfnArgs a = ffn_args(c, T);
-    set_act(a, &act);
     set_routed(a, routed, &perm);
     if (shared) set_shared(a, shared);
+    a.prep_records = 0;
     a.h = h;
     a.h_ld = c->inter;
     a.y = y;
@@ -496,7 +510,7 @@ int qrx_moe_forward_hostio(const qrx_cfg *c, const void *x_host, int32_t T, cons
 // looked up once per device with that device current.
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;   // 4 MiB per device
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;   // 8 MiB per device
 
 }  // namespace
 
@@ -532,7 +546,9 @@ extern "C" int qrx_expert_ffn_noalloc(const qrx_cfg *c, const qrx_experts *route
     if (v) return v;
     if ((v = check_experts(routed)) || (v = check_perm(perm)) || (v = check_act(c, act))) return v;
     if (!y_sorted) return QRX_EINVAL;
-    const size_t need = (size_t)T * c->top_k * c->inter * sizeof(float);
+    const size_t hbytes = align256((size_t)T * c->top_k * c->inter * sizeof(float));
+    const size_t xbytes = align256(act_records_bytes(c->afmt, c->hidden, T));
+    const size_t need = hbytes + xbytes + act_records_bytes(c->afmt, c->inter, T * c->top_k);
     if (need > kNoAllocScratchBytes) return QRX_ENOSPACE;
     void *scratch = nullptr;
     if ((v = noalloc_scratch(&scratch))) return v;
@@ -540,6 +556,9 @@ extern "C" int qrx_expert_ffn_noalloc(const qrx_cfg *c, const qrx_experts *route
     set_act(a, act);
     set_routed(a, routed, perm);
     a.h = static_cast<float *>(scratch);
+    a.xrec = static_cast<unsigned char *>(scratch) + hbytes;
+    a.hrec = static_cast<unsigned char *>(scratch) + hbytes + xbytes;
+    a.prep_records = 1;
     a.h_ld = c->inter;
     a.y = y_sorted;
     a.y_ld = c->hidden;

@@ -151,6 +151,15 @@ __device__ __forceinline__ float silu_mul(float g, float u)
     return g / (1.0f + expf(-g)) * u;
 }
 
+// Programmatic dependent launch.  pdl_wait() blocks until the previous kernel
+// in the stream has completed and its memory is visible (a no-op when the
+// kernel was launched without the programmatic-serialization attribute);
+// pdl_trigger() lets the next kernel begin launching.  Every kernel triggers
+// only after its own wait, so a kernel that starts early can rely on all
+// kernels before its predecessor having completed.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Device-side sticky status flag (set by kernels, read by qrx_last_error).
 // The library is built as one translation unit, so there is one flag per device.
 enum { DERR_NONE = 0, DERR_BOUNDS = 1, DERR_TIMEOUT = 2, DERR_BADIDX = 3 };

@@ -8,6 +8,27 @@
 
 namespace qrx {
 
+// Launches made while g_pdl is set carry the programmatic-stream-serialization
+// attribute (the layer forward sets it for every kernel after its first).
+extern thread_local bool g_pdl;
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = g_pdl ? attr : nullptr;
+    cfg.numAttrs = g_pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // device status flag (one per device, in k_quant.cu)
 cudaError_t read_and_clear_device_flag(int *flag);
 
@@ -27,12 +48,10 @@ struct RouterArgs {
     const float *bias;      // [E]
     int T, H, E, G, Gk, k;
     float rsf;
-    double *partial;        // [KS][T][E]
-    int KS;
+    float *logits;          // [T][E] scratch
     int32_t *idx;           // [T][k]
     float *w;               // [T][k]
 };
-int router_ksplit(int T, int H, int E, int num_sms);
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t st);
 
 cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const qrx_perm &p,
@@ -53,6 +72,9 @@ struct FfnArgs {
     const void *x;          // f32 / bf16 [T][H]
     const int8_t *xq;       // Q8 [T][H]
     const float *xd;        // Q8 [T][H/32]
+    unsigned char *xrec;    // scratch: gate/up input digit records [T][record bytes]
+    int prep_records;       // launch_ffn_gateup first builds xrec from x / xq, xd
+    unsigned char *hrec;    // scratch: down input digit records, one per h row
     // positions: routed p in [0, T*k), shared p = T*k + t
     float *h;               // [P][I] intermediate (gate/up output, down input)
     float *y;               // [P][H]
@@ -60,6 +82,7 @@ struct FfnArgs {
     // where the shared expert's rows live: h + sh_h_off*h_ld, y + sh_y_off*y_ld
     int64_t sh_h_row0, sh_y_row0;
 };
+cudaError_t launch_act_digits(const FfnArgs &a, cudaStream_t st);
 cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st);
 cudaError_t launch_ffn_down(const FfnArgs &a, int num_sms, cudaStream_t st);
 

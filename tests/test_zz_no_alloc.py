@@ -72,7 +72,7 @@ def test_noalloc_matches_workspace_version(dev, wl):
 
 
 def test_noalloc_refuses_sizes_above_its_array(dev):
-    wl = W.GLM_DECODE_T1.with_(n_experts=16, T=65)      # 65*8*2048*4 B > 4 MiB
+    wl = W.GLM_DECODE_T1.with_(n_experts=16, T=97)      # 97 * (65536 + 21504) B > 8 MiB
     c = qrx.cfg_of(wl)
     ex = qrx.Experts.empty(16, wl.hidden, wl.inter, 4)
     perm = qrx.Perm.empty(wl.T, wl.top_k, wl.n_experts)
