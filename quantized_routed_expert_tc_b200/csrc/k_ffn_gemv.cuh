@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
     int *tout = reinterpret_cast<int *>(smem + M.tout);
     int64_t *pre = reinterpret_cast<int64_t *>(smem + M.pre);
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int K = p.K, cpr = p.cpr;
     const int c = tid % cpr, team = tid / cpr, wit = c >> 5;
     const RecLayout RL = p.rec;
@@ -877,6 +877,7 @@ cudaError_t launch_act_digits(const FfnArgs &a, cudaStream_t st)
 
 cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
 {
+    if (ffn_use_tc(a)) return launch_ffn_tc_gateup(a, num_sms, st);
     const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
     GemvPlan pl;
     if (!gemv_plan(pl, a.wbits, ndig, a.H, 2 * a.I, a.T, a.E + 1)) return cudaErrorInvalidValue;
@@ -902,6 +903,7 @@ cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
 
 cudaError_t launch_ffn_down(const FfnArgs &a, int num_sms, cudaStream_t st)
 {
+    if (ffn_use_tc(a)) return launch_ffn_tc_down(a, num_sms, st);
     const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
     GemvPlan pl;
     if (!gemv_plan(pl, a.wbits, ndig, a.I, a.H, a.T, a.E + 1)) return cudaErrorInvalidValue;

@@ -157,18 +157,20 @@ __global__ void __launch_bounds__(256) k_router_tile(RouterArgs a)
 }
 
 // One warp per token.  Dynamic shared memory per warp: s[E], sc[E] (f32),
-// gscore[G] (f32), kept[G] (int).
+// gscore[G] (f32), kept[G] (int), sel[32] (int, the chosen experts in order).
+__host__ __device__ inline size_t select_smem_per_warp(int E, int G) { return (size_t)(2 * E + 2 * G + 32) * 4; }
+
 __global__ void __launch_bounds__(256) k_router_select(RouterArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int t = blockIdx.x * 8 + wid;
     const int E = a.E, G = a.G, gs = a.E / a.G;
-    const size_t per_warp = (size_t)(2 * E + 2 * G) * 4;
-    float *s_s = reinterpret_cast<float *>(smem_raw + per_warp * wid);
+    float *s_s = reinterpret_cast<float *>(smem_raw + select_smem_per_warp(E, G) * wid);
     float *sc_s = s_s + E;
     float *gsc = sc_s + E;
     int *kept = reinterpret_cast<int *>(gsc + G);
+    int *sel = kept + G;
     pdl_wait();
     pdl_trigger();
     if (t >= a.T) return;
@@ -200,6 +202,7 @@ __global__ void __launch_bounds__(256) k_router_select(RouterArgs a)
         kept[g] = rank < a.Gk;
     }
     __syncwarp();
+    // candidates of this lane: experts lane + 32 i in kept groups
     uint32_t taken = 0;   // bit i: expert lane + 32 i taken
     for (int j = 0; j < a.k; ++j) {
         float best = -INFINITY;
@@ -223,16 +226,18 @@ __global__ void __launch_bounds__(256) k_router_select(RouterArgs a)
             return;
         }
         if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        if (lane == 0) a.idx[(int64_t)t * a.k + j] = be;
+        if (lane == 0) sel[j] = be;
     }
     __syncwarp();
-    if (lane == 0) {
-        double ssum = 0.0;
-        for (int j = 0; j < a.k; ++j) ssum += (double)s_s[a.idx[(int64_t)t * a.k + j]];
-        for (int j = 0; j < a.k; ++j) {
-            const float s = s_s[a.idx[(int64_t)t * a.k + j]];
-            a.w[(int64_t)t * a.k + j] = (float)((double)s / ssum * (double)a.rsf);
-        }
+    // weights: s_j / sum(s) * rsf, the sum in double in selection order
+    double ssum = 0.0;
+    if (lane == 0)
+        for (int j = 0; j < a.k; ++j) ssum += (double)s_s[sel[j]];
+    ssum = __shfl_sync(0xffffffffu, ssum, 0);
+    if (lane < a.k) {
+        const int e = sel[lane];
+        a.idx[(int64_t)t * a.k + lane] = e;
+        a.w[(int64_t)t * a.k + lane] = (float)((double)s_s[e] / ssum * (double)a.rsf);
     }
 }
 
@@ -248,7 +253,7 @@ cudaError_t launch_router(const RouterArgs &a, cudaStream_t st)
         err = launch_k(a.x_bf16 ? k_router_tile<true> : k_router_tile<false>, grid, dim3(256), 0, st, a);
     }
     if (err != cudaSuccess) return err;
-    const size_t smem = (size_t)8 * (2 * a.E + 2 * a.G) * 4;
+    const size_t smem = (size_t)8 * select_smem_per_warp(a.E, a.G);
     if (smem > 48 * 1024) {
         err = cudaFuncSetAttribute(k_router_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)smem);

@@ -17,6 +17,7 @@
 #include "k_router.cuh"
 #include "k_permute.cuh"
 #include "k_ffn_gemv.cuh"
+#include "k_ffn_tc.cuh"
 #include "k_combine.cuh"
 
 using namespace qrx;
@@ -61,8 +62,8 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 // Workspace regions for T tokens.
 struct Ws {
-    size_t logits, counts, offsets, sorted, inv, uids, nu, xq, xd, xrec, hrec, h, y, xdev, outdev,
-        idx, w, total;
+    size_t logits, counts, offsets, sorted, inv, uids, nu, xq, xd, xrec, hrec, xperm, hperm, h, y,
+        xdev, outdev, idx, w, total;
 };
 
 Ws ws_layout(const qrx_cfg *c, int T)
@@ -87,6 +88,8 @@ Ws ws_layout(const qrx_cfg *c, int T)
     L.xd = take((size_t)T * (H / 32) * 4);
     L.xrec = take(act_records_bytes(c->afmt, (int)H, T));
     L.hrec = take(act_records_bytes(c->afmt, (int)I, (int)(A + T)));
+    L.xperm = take((size_t)T * H * 2);
+    L.hperm = take((size_t)(A + T) * I * 2);
     L.h = take((size_t)(A + T) * I * 4);
     L.y = take((size_t)(A + T) * H * 4);
     L.xdev = take((size_t)T * H * 4);
@@ -322,6 +325,9 @@ int qrx_expert_ffn(const qrx_cfg *c, const qrx_experts *routed, const qrx_perm *
     a.h = h_sorted ? h_sorted : at<float>(ws, L.h);
     a.xrec = at<unsigned char>(ws, L.xrec);
     a.hrec = at<unsigned char>(ws, L.hrec);
+    a.xperm = at<unsigned char>(ws, L.xperm);
+    a.hperm = at<unsigned char>(ws, L.hperm);
+    a.hperm_ready = 1;
     a.prep_records = 1;
     a.h_ld = c->inter;
     a.y = y_sorted;
@@ -345,6 +351,9 @@ int qrx_expert_down(const qrx_cfg *c, const qrx_experts *routed, const qrx_perm 
     FfnArgs a = ffn_args(c, T);
     set_routed(a, routed, perm);
     a.hrec = at<unsigned char>(ws, ws_layout(c, T).hrec);
+    a.xperm = at<unsigned char>(ws, ws_layout(c, T).xperm);
+    a.hperm = at<unsigned char>(ws, ws_layout(c, T).hperm);
+    a.hperm_ready = 0;
     a.h = const_cast<float *>(h_sorted);
     a.h_ld = c->inter;
     a.y = y_sorted;
@@ -367,6 +376,9 @@ int qrx_shared_ffn(const qrx_cfg *c, const qrx_experts *shared, const qrx_act *a
     a.h = h_sh ? h_sh : at<float>(ws, L.h);
     a.xrec = at<unsigned char>(ws, L.xrec);
     a.hrec = at<unsigned char>(ws, L.hrec);
+    a.xperm = at<unsigned char>(ws, L.xperm);
+    a.hperm = at<unsigned char>(ws, L.hperm);
+    a.hperm_ready = 1;
     a.prep_records = 1;
     a.h_ld = c->inter;
     a.y = y_sh;
@@ -420,12 +432,18 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     a.x = x;                      // Q8_0: the records kernel quantises x itself
     a.xrec = at<unsigned char>(ws, L.xrec);
     a.hrec = at<unsigned char>(ws, L.hrec);
+    a.xperm = at<unsigned char>(ws, L.xperm);
+    a.hperm = at<unsigned char>(ws, L.hperm);
+    a.hperm_ready = 1;
     if (!mark(0)) return QRX_ECUDA;
-    cudaError_t e = launch_act_digits(a, st);
+    const bool tc = ffn_use_tc(a);     // the tensor-core path needs no digit records
+    cudaError_t e = tc ? cudaSuccess : launch_act_digits(a, st);
     if (e != cudaSuccess || !mark(1)) return QRX_ECUDA;
-    // 2.. the rest chained with programmatic dependent launch
-    PdlScope pdl(true);
+    // 2.. the rest chained with programmatic dependent launch (the first kernel
+    // of the call never is: it must follow whatever the stream held before)
+    PdlScope pdl(!tc);
     if ((v = qrx_route(c, x, T, Wr, bias, topk_idx, topk_w, ws, ws_bytes, stream))) return v;
+    g_pdl = true;
     if (!mark(2)) return QRX_ECUDA;
     qrx_perm perm{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.sorted),
                   at<int32_t>(ws, L.inv), at<int32_t>(ws, L.uids), at<int32_t>(ws, L.nu)};

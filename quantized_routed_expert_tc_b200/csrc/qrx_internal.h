@@ -75,6 +75,9 @@ struct FfnArgs {
     unsigned char *xrec;    // scratch: gate/up input digit records [T][record bytes]
     int prep_records;       // launch_ffn_gateup first builds xrec from x / xq, xd
     unsigned char *hrec;    // scratch: down input digit records, one per h row
+    void *xperm;            // scratch (tensor-core path): bf16 x, chunk-permuted [T][H]
+    void *hperm;            // scratch (tensor-core path): bf16 h, chunk-permuted, one per h row
+    int hperm_ready;        // the gate/up call of this layer already wrote hperm
     // positions: routed p in [0, T*k), shared p = T*k + t
     float *h;               // [P][I] intermediate (gate/up output, down input)
     float *y;               // [P][H]
@@ -83,6 +86,9 @@ struct FfnArgs {
     int64_t sh_h_row0, sh_y_row0;
 };
 cudaError_t launch_act_digits(const FfnArgs &a, cudaStream_t st);
+bool ffn_use_tc(const FfnArgs &a);
+cudaError_t launch_ffn_tc_gateup(const FfnArgs &a, int num_sms, cudaStream_t st);
+cudaError_t launch_ffn_tc_down(const FfnArgs &a, int num_sms, cudaStream_t st);
 cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st);
 cudaError_t launch_ffn_down(const FfnArgs &a, int num_sms, cudaStream_t st);
 

@@ -306,6 +306,38 @@ def test_tiny_large_batch_many_token_groups(tiny):
         check_layer(glay, olay, wl, x, [0, 77, 299])
 
 
+def test_tiny_bf16_many_tokens_tensor_cores(tiny):
+    """T >= 256 with bf16 activations runs the expert FFN as tcgen05 grouped GEMMs."""
+    glay, olay = tiny
+    for T in (256, 300):
+        wl = W.TINY.with_(T=T, afmt=W.A_BF16)
+        x = activations(wl, T, batch=4)
+        check_layer(glay, olay, wl, x, [0, 131, T - 1])
+    # stage isolation: the down projection from the oracle's h, and h itself
+    wl = W.TINY.with_(T=300, afmt=W.A_BF16)
+    x = activations(wl, 300, batch=4)
+    _, bias = router_weights(wl)
+    r = oracle.router(wl, x, olay.Wr, bias)
+    p = oracle.permute(r["idx"], wl.n_experts)
+    ex = olay.experts(r["idx"].ravel(), wl.wbits)
+    h_o, y_o = oracle.expert_ffn(wl, ex, p, x)
+    c = qrx.cfg_of(wl)
+    ws = qrx.workspace(c, 300)
+    perm = qrx.Perm.empty(300, wl.top_k, wl.n_experts)
+    qrx.qrx_permute(c, cu(r["idx"]), perm)
+    A = 300 * wl.top_k
+    hs = torch.empty((A, wl.inter), dtype=torch.float32, device="cuda")
+    ys = torch.empty((A, wl.hidden), dtype=torch.float32, device="cuda")
+    qrx.qrx_expert_ffn(c, glay.routed[4], perm, 300, ys, ws, x=to_device_act(wl, x), h_sorted=hs)
+    yd = torch.empty((A, wl.hidden), dtype=torch.float32, device="cuda")
+    qrx.qrx_expert_down(c, glay.routed[4], perm, cu(h_o), 300, yd, ws)
+    torch.cuda.synchronize()
+    assert qrx.qrx_last_error() == qrx.QRX_OK
+    assert rel_err(np_(hs), h_o) <= TOL
+    assert rel_err(np_(ys), y_o) <= TOL
+    assert rel_err(np_(yd), y_o) <= TOL
+
+
 # ------------------------------------------------------------------ GLM-shaped layer, full size
 def test_glm_decode_t1(glm):
     glay, olay = glm
