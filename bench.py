@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling case: fewer routed experts (same per-launch work at T=1)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="profiling case: another token count per step")
     ap.add_argument("--no-settle", action="store_true",
                     help="skip the 1 s clock-settle loop (for ncu launch counting)")
     return ap.parse_args()
@@ -63,10 +65,31 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
-    """Hash of the GEMV kernel source: traffic figures apply only to this version."""
+FALLBACK_BF16_TFLOPS = 1590.0
+TC_MIN_T = 256          # tokens from which bf16 x int4 batches run on the tensor cores
+
+
+def uses_tensor_cores(wl) -> bool:
+    """Whether the library takes the tcgen05 path for this workload's expert FFN."""
+    return wl.afmt == 2 and wl.wbits == 4 and wl.T >= TC_MIN_T
+
+
+def tensor_peak():
+    """Dense bf16 tensor peak (burst: the kernel is timed between its own events)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured (burst)"
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def kernel_source_hash(kernel: str = "k_ffn_gemv_gateup") -> str:
+    """Hash of a kernel's source: traffic figures apply only to this version."""
     h = hashlib.sha256()
-    for f in ("k_ffn_gemv.cuh", "qrx_dev.cuh"):
+    files = ("k_ffn_tc.cuh", "qrx_dev.cuh") if kernel.startswith("k_ffn_tc") else \
+        ("k_ffn_gemv.cuh", "qrx_dev.cuh")
+    for f in files:
         with open(os.path.join(ROOT, "quantized_routed_expert_tc_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -80,7 +103,7 @@ def recorded_traffic(kernel: str, workload: str):
     with open(path) as f:
         d = json.load(f)
     rec = d.get(kernel, {}).get(workload)
-    if not rec or rec.get("source_sha") != kernel_source_hash():
+    if not rec or rec.get("source_sha") != kernel_source_hash(kernel):
         return None
     return rec.get("bytes_per_launch")
 
@@ -309,9 +332,16 @@ def run_qrx(args, wl, rank, world, local_rank):
     gu_ms = per[:, 3]          # the gate/up kernel alone (stage 3)
     achieved = float((gateup_bytes / (gu_ms / 1e3)).mean() / 1e9)
     peak, peak_kind = peaks()
+    tc = uses_tensor_cores(wl)
+    if tc:
+        # tensor-core path: 2 flops per weight x token product, every assignment
+        # plus the shared expert's T tokens, gate and up rows (2I x H)
+        gateup_flops = 2.0 * (T * k + T) * (2 * I) * H
+        tc_achieved = gateup_flops / float(gu_ms.mean() / 1e3) / 1e12
+        tc_peak, tc_peak_kind = tensor_peak()
     nu_all = np.array([unions[i % npool] for i in range(args.steps)], dtype=np.float64)
     weight_gbs = float(((nu_all + 1) * exp_bytes).mean() / (ms_step / 1e3) / 1e9)
-    traffic = recorded_traffic("k_ffn_gemv_gateup", wl.name)
+    traffic = recorded_traffic("k_ffn_tc_gateup" if tc else "k_ffn_gemv_gateup", wl.name)
 
     e2e = None
     if not args.no_e2e:
@@ -349,7 +379,8 @@ def run_qrx(args, wl, rank, world, local_rank):
         line = {
             "metric": METRIC, "value": T * world / (ms_step / 1e3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if tc else "int32",
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights quantised by the "
                     "library; no trained weights)",
             "config": workload_config(wl),
@@ -360,11 +391,18 @@ def run_qrx(args, wl, rank, world, local_rank):
             "stage_us": {s: float(per[:, j].mean() * 1e3) for j, s in enumerate(stages)},
             "stage_note": "from qrx_moe_forward_profiled: events between kernels disable the "
                           "launch overlap, so the stages sum to more than ms_per_step",
-            "roofline": {"kernel": "k_ffn_gemv (gate/up + SwiGLU)", "bound": "hbm",
-                         "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_kind": peak_kind,
-                         "traffic": traffic,
-                         "algorithmic_bytes_per_launch": float(gateup_bytes.mean())},
+            "roofline": ({"kernel": "k_ffn_tc (gate/up + SwiGLU, tcgen05)", "bound": "tensor",
+                          "achieved": tc_achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                          "frac": tc_achieved / tc_peak, "peak_kind": tc_peak_kind,
+                          "traffic": traffic, "algorithmic_flops_per_launch": gateup_flops,
+                          "weight_bytes_per_launch": float(gateup_bytes.mean()),
+                          "weight_gbs": achieved}
+                         if tc else
+                         {"kernel": "k_ffn_gemv (gate/up + SwiGLU)", "bound": "hbm",
+                          "achieved": achieved, "peak": peak, "unit": "GB/s",
+                          "frac": achieved / peak, "peak_kind": peak_kind,
+                          "traffic": traffic,
+                          "algorithmic_bytes_per_launch": float(gateup_bytes.mean())}),
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
@@ -379,6 +417,8 @@ def main():
     wl = W.ALL[args.workload]
     if args.experts:
         wl = wl.with_(name=f"{wl.name}_e{args.experts}", n_experts=args.experts)
+    if args.tokens:
+        wl = wl.with_(name=f"{wl.name}_t{args.tokens}", T=args.tokens)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -101,7 +101,8 @@ typedef struct {
  *   QRX_A_F32:  x = f32 [T][H];        xq, xd unused.
  *   QRX_A_BF16: x = bf16 [T][H];       xq, xd unused.
  *   QRX_A_Q8_0: xq = int8 [T][H] and xd = f32 [T][H/32] from
- *               qrx_quantize_act_q8;   x unused. */
+ *               qrx_quantize_act_q8;   x unused.
+ * Device pointers, 16-byte aligned (QRX_EINVAL otherwise). */
 typedef struct {
     const void *x;
     const int8_t *xq;
@@ -118,6 +119,19 @@ int qrx_validate(const qrx_cfg *cfg);
 
 /* Bytes of scratch the calls below need for T tokens (a multiple of 256). */
 size_t qrx_workspace_bytes(const qrx_cfg *cfg, int32_t T);
+
+/* Which engine runs the expert FFN (gate/up + SwiGLU and down) of a call with
+ * this configuration and T tokens (the routed, shared and whole-layer entry
+ * points that take a workspace):
+ *   QRX_ENGINE_GEMV  the HBM-streaming integer-digit GEMV (any format);
+ *   QRX_ENGINE_TC    grouped GEMMs on the tcgen05 tensor cores: bf16
+ *                    activations, int4 weights, T >= 256, H and I multiples
+ *                    of 256.
+ * Returns QRX_EINVAL for an invalid configuration or T <= 0.  The
+ * allocation-free entry point always uses the GEMV. */
+#define QRX_ENGINE_GEMV 0
+#define QRX_ENGINE_TC 1
+int qrx_ffn_engine(const qrx_cfg *cfg, int32_t T);
 
 /* Sticky device status: synchronises the current device, returns QRX_OK,
  * QRX_EDEVICE or QRX_ETIMEOUT (and clears the flag), or QRX_ECUDA if the
@@ -240,7 +254,13 @@ int qrx_expert_ffn_noalloc(const qrx_cfg *cfg, const qrx_experts *routed,
  * The kernels after the first are chained with programmatic dependent launch:
  * each may start while its predecessor drains and waits for it only where it
  * reads its output (the down kernel starts streaming its weights first).
- * shared may be NULL.  topk_idx, topk_w: outputs [T][k].  out [T][H] f32. */
+ * shared may be NULL.  x: the activations in cfg->afmt (f32 or bf16 [T][H];
+ * Q8_0 is quantised from f32 x inside the call), 16-byte aligned.
+ * topk_idx, topk_w: outputs [T][k].  out [T][H] f32, 16-byte aligned.
+ * Expert FFN engine: bf16 activations, int4 experts, T >= 256 and H, I
+ * multiples of 256 run gate/up and down as grouped GEMMs on the tcgen05 tensor
+ * cores (bf16 x bf16 -> f32; int4 codes are exact in bf16); every other case
+ * runs the HBM-streaming integer GEMV. */
 int qrx_moe_forward(const qrx_cfg *cfg, const void *x, int32_t T, const float *W_router,
                     const float *bias, const qrx_experts *routed, const qrx_experts *shared,
                     int32_t *topk_idx, float *topk_w, float *out, void *ws,

@@ -5,64 +5,101 @@
 // README "JustVugg/colibri", section "已实现的功能": batch-union MoE (each
 // unique expert of a batch is read once and applied to all positions routed
 // to it); packed int4 weights with per-row scales, dequantised on use.  With
-// ~64 tokens per expert the work is a dense contraction, so it runs on the
+// ~100 tokens per expert the work is a dense contraction, so it runs on the
 // tensor cores: int4 codes are exact in bf16, products accumulate in f32, and
 // the per-row scale multiplies the accumulator in the epilogue.
 //
-// Tiles.  A work item is (slot, 128 weight rows, up to 256 tokens): the
-// weights are the MMA's M side and the tokens its N side, K advances in
-// stages of 64 (one 128-byte swizzle atom of bf16).  Roles per CTA (one CTA
-// per SM, persistent over items):
-//   warps 0-3  loaders: cp.async of the int4 weight rows (each thread owns one
-//              row) and of the token rows; each thread dequantises its own
-//              row into the 128B-swizzled K-major A tile, then arrives on the
-//              stage's "full" mbarrier;
-//   warp 4     allocates 512 TMEM columns (two 128x256 f32 accumulators) and
-//              issues tcgen05.mma (M=128, N<=256, K=16, four per stage); each
-//              stage is released with tcgen05.commit to its "empty" mbarrier,
-//              each finished item with a commit to its accumulator's "full";
-//   warps 5-8  epilogue: tcgen05.ld of the accumulator, row scales, SwiGLU
-//              (gate/up) or the output rows (down), stores.
+// Tiles.  A work item is (slot, 256 weight rows, up to 128 tokens): the
+// weights are the MMA's M side (two M=128 halves sharing one B tile) and the
+// tokens its N side; K advances in stages of 64 (one 128-byte swizzle atom of
+// bf16).  B is always a run of consecutive rows of one bf16 matrix: for
+// gate/up the tokens gathered into expert order by k_gather_x, for down the
+// rows of h that gate/up wrote in the same order.  Roles per CTA (one CTA per
+// SM, persistent over items):
+//   warp 0      TMA producer: the packed int4 rows of the item, 128 bytes
+//               (4 k-stages) per row at a time, into a 128B-swizzled "raw"
+//               stage, after an L2 prefetch of the same box issued TC_PF raw
+//               stages earlier; the token rows of each k-stage into its B tile;
+//   warp 1      allocates 512 TMEM columns (two 256x128 f32 accumulators) and
+//               issues tcgen05.mma (M=128, N<=128, K=16; two halves x four
+//               per stage); each stage is released with tcgen05.commit to its
+//               "empty" mbarrier, each finished item with a commit to its
+//               accumulator's "full";
+//   warps 4-7   epilogue: tcgen05.ld of the accumulator, row scales, SwiGLU
+//               (gate/up) or the output rows (down), stores;
+//   8 warps     dequantisers (2, 3, 8, 10, 11, 12, 14, 15): thread r turns
+//               row r's 64 codes of the stage into bf16 in the 128B-swizzled
+//               K-major A tile.
+// One thread issues the MMAs: the tensor core's queue is only a few
+// instructions deep, so everything that thread does between two stages (its
+// barrier checks, the commit) is time the tensor core may sit idle; the other
+// roles that wait long (producer, epilogue) sleep between polls.
 // Dequantisation writes the 8 codes of a packed word in the order
 // (0,4,1,5,2,6,3,7); the token rows (and h for the down projection) are kept
 // in the same order within every 8-element chunk, so the contraction is
 // unchanged.  All mbarrier waits are bounded; a timeout raises the device
-// status flag and every role leaves its loops before TMEM is freed.
+// status flag, every role leaves its loops, the producer waits (bounded) for
+// the copies it started, and only then is TMEM freed.
 #pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <mutex>
 #include "qrx_dev.cuh"
 
 namespace qrx {
 
-constexpr int TC_M = 128, TC_BK = 64, TC_NMAX = 256, TC_STAGES = 4, TC_LOOKAHEAD = 3;
-constexpr int TC_LOADERS = 128, TC_THREADS = 288;                // 9 warps
-constexpr int TC_A_BYTES = TC_M * 128;                           // bf16 A tile, 16 KB
-constexpr int TC_RAW_BYTES = TC_M * 32;                          // int4 A tile, 4 KB
-constexpr int TC_B_BYTES = TC_NMAX * 128;                        // bf16 B tile, 32 KB
-constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES + TC_RAW_BYTES;
-// dynamic shared memory: 1024-byte alignment slack, the stages, 128 bytes of
-// barriers and flags, the item prefix over up to maxslots slots
+constexpr int TC_HALF = 128;                 // rows per MMA (M)
+constexpr int TC_M = 2 * TC_HALF;            // weight rows per item
+constexpr int TC_BK = 64;                    // K per stage
+constexpr int TC_RK = 4;                     // stages per raw (int4) stage: 128 bytes of a row
+constexpr int TC_NMAX = 128;                 // tokens per item
+constexpr int TC_S = 3;                      // stages of (bf16 A tile, B tile)
+constexpr int TC_RS = 2;                     // raw stages (int4 rows from HBM)
+constexpr int TC_PF = 4;                     // raw stages prefetched into L2 ahead of their copy
+constexpr int TC_BOX_ROWS = 32;              // token rows per B copy
+constexpr int TC_A_BYTES = TC_M * 128;       // bf16 A tile (two halves), 32 KB
+constexpr int TC_B_BYTES = TC_NMAX * 128;    // bf16 B tile, 16 KB
+constexpr int TC_RAW_BYTES = TC_M * 128;     // int4 rows, 4 stages, 32 KB
+// Warp roles.  Warp w issues from SM sub-partition w % 4, and the MMA thread
+// runs a serial chain (barrier checks, descriptors, MMAs, commit) that loses
+// every issue arbitration against busy warps: its sub-partition (1) holds only
+// the MMA warp, one epilogue warp (asleep between items) and two idle warps,
+// while the eight dequantiser warps share sub-partitions 0, 2 and 3.
+constexpr int TC_PRODUCER = 0, TC_MMA = 1, TC_EPI0 = 4;  // epilogue: warps 4..7 (TMEM quarter = warp % 4)
+constexpr int TC_DQ_WARPS = 8;
+constexpr int TC_THREADS = 16 * 32;                      // warps 9 and 13 idle
+// dequantiser index of warp w (-1: not a dequantiser): warps 2, 3, 8, 10, 11, 12, 14, 15
+__host__ __device__ constexpr int tc_dq_index(int w)
+{
+    return w == 2 ? 0 : w == 3 ? 1 : w == 8 ? 2 : w == 10 ? 3 : w == 11 ? 4 : w == 12 ? 5 : w == 14 ? 6
+         : w == 15 ? 7 : -1;
+}
+#ifndef TC_BS
+#define TC_BS 16                              // mbarrier spacing in 8-byte words: one per 128-byte line
+#endif
+constexpr int TC_NBARS = 3 * TC_S + 2 * TC_RS + 5;   // + acc_full[2], acc_empty[2], drain
+constexpr int TC_CTL_BYTES = (TC_NBARS + 1) * TC_BS * 8;
+// dynamic shared memory: 1024-byte alignment slack, the stages, barriers and
+// flags, the item prefix over up to maxslots slots
 __host__ __device__ constexpr int tc_smem_bytes(int maxslots)
 {
-    return 1024 + TC_STAGE_BYTES * TC_STAGES + 128 + (maxslots + 2) * 8;
+    return 1024 + TC_S * (TC_A_BYTES + TC_B_BYTES) + TC_RS * TC_RAW_BYTES + TC_CTL_BYTES +
+           (maxslots + 2) * 8;
 }
 
-// Position p within an 8-element chunk holds element kPermTC[p].
+// Position p within an 8-element chunk holds element tc_perm(p).
 __host__ __device__ constexpr int tc_perm(int p) { return (p & 1) ? 4 + (p >> 1) : (p >> 1); }
 __host__ __device__ constexpr int tc_inv_perm(int e) { return e < 4 ? 2 * e : 2 * (e - 4) + 1; }
 
 struct TcP {
-    int rows, K, row_bytes, mtiles, kstages;
-    const uint8_t *w;       // routed weights, expert stride w_stride bytes
-    int64_t w_stride;
+    int rows, K, mtiles, kstages;
     const float *s;         // routed row scales, expert stride s_stride
     int64_t s_stride;
-    const uint8_t *w_sh;
     const float *s_sh;
     int routed, shared, E, k, T;
-    const int32_t *offsets, *sorted, *union_ids, *n_union;
-    const __nv_bfloat16 *bsrc;   // B rows (bf16, chunk-permuted): tokens (gate/up) or h rows (down)
-    int64_t sh_in_row0;          // down: B row of the shared expert's first token
-    float *out;                  // gate/up: h f32 [rows of positions][I]; down: y f32
+    const int32_t *offsets, *union_ids, *n_union;
+    int64_t b_sh_row0;           // B row of the shared expert's first token
+    float *out;                  // gate/up: h f32 [rows of positions][I] (may be null); down: y f32
     int64_t out_ld, sh_out_row0;
     __nv_bfloat16 *hperm;        // gate/up: h bf16 chunk-permuted [positions][I] (may be null)
     int gateup;
@@ -78,13 +115,8 @@ __device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr)
 __device__ __forceinline__ uint32_t tc_idesc(int N)
 {
     // D f32, A bf16, B bf16, both K-major, N >> 3, M >> 4.
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(TC_M >> 4) << 24);
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-                 : "memory");
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(TC_HALF >> 4) << 24);
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t mbar)
@@ -92,7 +124,46 @@ __device__ __forceinline__ void mbar_arrive(uint32_t mbar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
 }
 
-// Item geometry for slot s: token tiles of at most 256, balanced, multiple of 16.
+__device__ __forceinline__ void mbar_expect(uint32_t mbar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes)
+                 : "memory");
+}
+
+// Tiled TMA loads (no multicast) completing on `mbar`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t mbar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(mbar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z,
+                                            uint32_t mbar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::
+            "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(mbar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, int y, int z)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint32_t mbar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
+}
+
+// Item geometry for slot s: token tiles of at most 128, balanced, multiple of 16.
 struct TcSlot {
     int ntok, ntiles, nbase;
 };
@@ -112,21 +183,132 @@ __device__ __forceinline__ TcSlot tc_slot(const TcP &p, int s, int nu)
     return r;
 }
 
-__global__ void __launch_bounds__(TC_THREADS, 1) k_ffn_tc(const TcP p)
+// One work item, decoded from its index through the item prefix over slots.
+struct TcItem {
+    int slot, mt, n0, nv, nn, e;
+    bool routed;
+    int64_t b0;             // first B row
+};
+
+__device__ __forceinline__ TcItem tc_decode(const TcP &p, const int64_t *pre, int nslots, int nu,
+                                            int64_t it)
+{
+    int lo = 0, hi = nslots;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (pre[mid] <= it) lo = mid; else hi = mid;
+    }
+    TcItem d;
+    d.slot = lo;
+    const TcSlot sl = tc_slot(p, lo, nu);
+    const int64_t r = it - pre[lo];
+    const int ni = (int)(r / p.mtiles);
+    d.mt = (int)(r % p.mtiles);
+    d.n0 = ni * sl.nbase;
+    d.nv = min(sl.nbase, sl.ntok - d.n0);
+    d.nn = sl.nbase;
+    d.routed = lo < nu;
+    d.e = 0;
+    int64_t p0 = p.b_sh_row0;
+    if (d.routed) {
+        const int e = p.union_ids[lo];
+        d.e = (e >= 0 && e < p.E) ? e : 0;
+        p0 = p.offsets[d.e];
+    }
+    d.b0 = p0 + d.n0;
+    return d;
+}
+
+// Bounded wait that also gives up (false, no new status) once another role
+// has raised the abort flag; on its own timeout it raises both.  Roles off
+// the MMA's critical path poll with a sleep in between (sleep_ns > 0), which
+// leaves the issue slots of their SM sub-partition to the warps that work.
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                        unsigned sleep_ns = 0)
+{
+    const uint32_t a = smem_u32(bar);
+    for (long long it = 0; it < GV_WAIT_CAP; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (sleep_ns) {
+            __nanosleep(sleep_ns);
+            if (*abort_flag) return false;
+        } else if ((it & 255) == 255 && *abort_flag) {
+            return false;
+        }
+    }
+    *abort_flag = 1;
+    raise_status(DERR_TIMEOUT);
+    return false;
+}
+
+// tc_wait with a one-instruction fast path for a phase that has already
+// completed (the common case on the MMA thread).
+__device__ __forceinline__ bool tc_wait_fast(uint64_t *bar, uint32_t parity, volatile int *abort_flag)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done ? true : tc_wait(bar, parity, abort_flag);
+}
+
+// One tcgen05.mma (kind::f16, cta_group::1): D[tmem] (+)= A[smem] * B[smem].
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred pd;\n\t"
+        "setp.ne.b32 pd, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, pd;\n\t}" ::"r"(d),
+        "l"(da), "l"(db), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// tc_wait for a whole warp: lane 0 polls (one shared-memory request per poll
+// instead of 32) and broadcasts the outcome.
+__device__ __forceinline__ bool tc_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             unsigned sleep_ns = 0)
+{
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = tc_wait(bar, parity, abort_flag, sleep_ns) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    k_ffn_tc(const __grid_constant__ CUtensorMap mw, const __grid_constant__ CUtensorMap mwsh,
+             const __grid_constant__ CUtensorMap mb, const TcP p)
 {
     extern __shared__ __align__(1024) unsigned char tsm_raw[];
     // 1024-byte alignment for the swizzled tiles
     unsigned char *tsm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~(uintptr_t)1023);
-    unsigned char *ctl = tsm + TC_STAGE_BYTES * TC_STAGES;
-    uint64_t *full = reinterpret_cast<uint64_t *>(ctl);            // [STAGES]
-    uint64_t *empty = full + TC_STAGES;                            // [STAGES]
-    uint64_t *acc_full = empty + TC_STAGES;                        // [2]
-    uint64_t *acc_empty = acc_full + 2;                            // [2]
-    uint64_t *drain = acc_empty + 2;                               // [1]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    unsigned char *sA = tsm;                                   // [S][256 rows][128 B]
+    unsigned char *sB = sA + TC_S * TC_A_BYTES;                // [S][128 rows][128 B]
+    unsigned char *sR = sB + TC_S * TC_B_BYTES;                // [RS][256 rows][128 B]
+    unsigned char *ctl = sR + TC_RS * TC_RAW_BYTES;
+    // barriers TC_BS words apart (each on its own 128-byte line at the default)
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(ctl);      // [S]  dequantisers
+    uint64_t *full_b = full_a + TC_S * TC_BS;                  // [S]  B copies
+    uint64_t *empty = full_b + TC_S * TC_BS;                   // [S]  MMA done with the stage
+    uint64_t *raw_full = empty + TC_S * TC_BS;                 // [RS] int4 copies
+    uint64_t *raw_empty = raw_full + TC_RS * TC_BS;            // [RS] dequantisers done
+    uint64_t *acc_full = raw_empty + TC_RS * TC_BS;            // [2]
+    uint64_t *acc_empty = acc_full + 2 * TC_BS;                // [2]
+    uint64_t *drain = acc_empty + 2 * TC_BS;                   // [1]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + TC_BS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int64_t *pre = reinterpret_cast<int64_t *>(ctl + 128);        // [nslots + 1] item prefix
+    int64_t *pre = reinterpret_cast<int64_t *>(ctl + TC_CTL_BYTES);   // [nslots + 1] item prefix
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_wait();
@@ -135,26 +317,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_ffn_tc(const TcP p)
     const int nslots = nu + (p.shared ? 1 : 0);
 
     if (tid == 0) {
-        for (int i = 0; i < TC_STAGES; ++i) {
-            mbar_init(smem_u32(&full[i]), TC_LOADERS);
-            mbar_init(smem_u32(&empty[i]), 1);
+        for (int i = 0; i < TC_S; ++i) {
+            mbar_init(smem_u32(&full_a[(i) * TC_BS]), TC_DQ_WARPS);
+            mbar_init(smem_u32(&full_b[(i) * TC_BS]), 1);
+            mbar_init(smem_u32(&empty[(i) * TC_BS]), 1);
+        }
+        for (int i = 0; i < TC_RS; ++i) {
+            mbar_init(smem_u32(&raw_full[(i) * TC_BS]), 1);
+            mbar_init(smem_u32(&raw_empty[(i) * TC_BS]), TC_DQ_WARPS);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&acc_full[i]), 1);
-            mbar_init(smem_u32(&acc_empty[i]), 4);
+            mbar_init(smem_u32(&acc_full[(i) * TC_BS]), 1);
+            mbar_init(smem_u32(&acc_empty[(i) * TC_BS]), 4);
         }
         mbar_init(smem_u32(drain), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 4) {
+    if (warp == TC_MMA) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
                          smem_u32(tmem_slot))
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // item prefix over slots (warp 5): items of slot s = ntiles * mtiles
-    if (warp == 5) {
+    // item prefix over slots: items of slot s = ntiles * mtiles
+    if (warp == TC_EPI0) {
         int64_t run = 0;
         for (int s0 = 0; s0 < nslots; s0 += 32) {
             const int s = s0 + lane;
@@ -177,89 +364,219 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_ffn_tc(const TcP p)
     const uint32_t tmem = *tmem_slot;
     const int64_t nitems = pre[nslots];
 
-    // decode item -> (slot, m tile, token tile)
-    auto decode = [&](int64_t it, int &s, int &mt, int &n0, int &nv, int &nn) {
-        int lo = 0, hi = nslots;
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (pre[mid] <= it) lo = mid; else hi = mid;
-        }
-        s = lo;
-        const TcSlot sl = tc_slot(p, s, nu);
-        const int64_t r = it - pre[s];
-        const int ni = (int)(r / p.mtiles);
-        mt = (int)(r % p.mtiles);
-        n0 = ni * sl.nbase;
-        nv = min(sl.nbase, sl.ntok - n0);
-        nn = sl.nbase;
-    };
-
-    if (warp < 4) {
-        // ================= loaders =================
-        const int row = tid;                       // weight row within the tile
-        int64_t g = 0;                             // global stage counter
-        int64_t issued = 0;
-        // per-item state for the stages being issued
-        for (int64_t it = blockIdx.x; it < nitems && !*abort_flag; it += gridDim.x) {
-            int s, mt, n0, nv, nn;
-            decode(it, s, mt, n0, nv, nn);
-            const bool routed = s < nu;
-            int e = 0, p0 = 0;
-            if (routed) {
-                e = p.union_ids[s];
-                e = (e >= 0 && e < p.E) ? e : 0;
-                p0 = p.offsets[e];
+    if (warp == TC_PRODUCER) {
+        // ================= TMA producer (one thread) =================
+        if (lane == 0) {
+            uint32_t g = 0, rg = 0;
+            bool ok = true;
+            // L2 prefetch cursor, TC_PF raw stages ahead of the copies
+            const int kraw = p.kstages / TC_RK;
+            int64_t pf_it = blockIdx.x;
+            int pf_kr = 0;
+            TcItem pf_d{};
+            if (pf_it < nitems) pf_d = tc_decode(p, pre, nslots, nu, pf_it);
+            auto pf_step = [&]() {
+                if (pf_it >= nitems) return;
+                const CUtensorMap *m = pf_d.routed ? &mw : &mwsh;
+                const int zz = pf_d.routed ? pf_d.e : 0;
+                tma_prefetch_3d(m, pf_kr * 128, pf_d.mt * TC_M, zz);
+                tma_prefetch_3d(m, pf_kr * 128, pf_d.mt * TC_M + TC_HALF, zz);
+                if (++pf_kr == kraw) {
+                    pf_kr = 0;
+                    pf_it += gridDim.x;
+                    if (pf_it < nitems) pf_d = tc_decode(p, pre, nslots, nu, pf_it);
+                }
+            };
+            for (int i = 0; i < TC_PF; ++i) pf_step();
+            for (int64_t it = blockIdx.x; ok && it < nitems && !*abort_flag; it += gridDim.x) {
+                const TcItem d = tc_decode(p, pre, nslots, nu, it);
+                const CUtensorMap *wm = d.routed ? &mw : &mwsh;
+                const int z = d.routed ? d.e : 0;
+                const int nbox = (d.nn + TC_BOX_ROWS - 1) / TC_BOX_ROWS;
+                for (int kb = 0; kb < p.kstages; ++kb) {
+                    if (kb % TC_RK == 0) {
+                        const uint32_t rs = rg % TC_RS;
+                        if (rg >= TC_RS && !tc_wait(&raw_empty[(rs) * TC_BS], ((rg / TC_RS) - 1) & 1, abort_flag, 64)) {
+                            ok = false;
+                            break;
+                        }
+                        pf_step();
+                        const uint32_t dst = smem_u32(sR + rs * TC_RAW_BYTES);
+                        const uint32_t bar = smem_u32(&raw_full[(rs) * TC_BS]);
+                        mbar_expect(bar, TC_RAW_BYTES);
+                        tma_load_3d(dst, wm, (kb / TC_RK) * 128, d.mt * TC_M, z, bar);
+                        tma_load_3d(dst + TC_RAW_BYTES / 2, wm, (kb / TC_RK) * 128, d.mt * TC_M + TC_HALF, z,
+                                    bar);
+                        ++rg;
+                    }
+                    const uint32_t sb = g % TC_S;
+                    if (g >= TC_S && !tc_wait(&empty[(sb) * TC_BS], ((g / TC_S) - 1) & 1, abort_flag, 64)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar = smem_u32(&full_b[(sb) * TC_BS]);
+                    mbar_expect(bar, (uint32_t)(nbox * TC_BOX_ROWS * 128));
+                    for (int j = 0; j < nbox; ++j)
+                        tma_load_2d(smem_u32(sB + sb * TC_B_BYTES + j * TC_BOX_ROWS * 128), &mb, kb * TC_BK,
+                                    (int)(d.b0 + j * TC_BOX_ROWS), bar);
+                    ++g;
+                }
             }
-            const uint8_t *W = (routed ? p.w + (int64_t)e * p.w_stride : p.w_sh) +
-                               ((int64_t)mt * TC_M + row) * p.row_bytes;
-            // B source row of token n of this item
-            auto brow = [&](int n) -> int64_t {
-                const int i = n0 + n;
-                if (p.gateup) return routed ? p.sorted[p0 + i] / p.k : i;
-                return routed ? p0 + i : p.sh_in_row0 + i;
-            };
-            auto issue_stage = [&](int kb, int64_t gs) {
-                const int st = (int)(gs % TC_STAGES);
-                unsigned char *sb = tsm + (size_t)st * TC_STAGE_BYTES;
-                // wait until the MMA has released this stage
-                if (*abort_flag) return;
-                if (gs >= TC_STAGES &&
-                    !mbar_wait(smem_u32(&empty[st]), (uint32_t)(((gs / TC_STAGES) - 1) & 1))) {
-                    *abort_flag = 1;
-                    raise_status(DERR_TIMEOUT);
-                    return;
+            // the copies started above land before the CTA may leave: wait for
+            // the last phase armed on every barrier (already complete unless a
+            // consumer gave up)
+            for (uint32_t i = 0; i < (uint32_t)TC_S && i < g; ++i) {
+                const uint32_t n = (g - 1 - i) / TC_S + 1;
+                if (!mbar_wait(smem_u32(&full_b[(i) * TC_BS]), (n - 1) & 1)) raise_status(DERR_TIMEOUT);
+            }
+            for (uint32_t i = 0; i < (uint32_t)TC_RS && i < rg; ++i) {
+                const uint32_t n = (rg - 1 - i) / TC_RS + 1;
+                if (!mbar_wait(smem_u32(&raw_full[(i) * TC_BS]), (n - 1) & 1)) raise_status(DERR_TIMEOUT);
+            }
+        }
+        __syncwarp();
+    } else if (warp == TC_MMA) {
+        // ================= MMA issue (one thread) =================
+        // The tensor core takes the next MMA only when its short queue has
+        // room, and each issue already costs tens of cycles, so the issuing
+        // thread runs a minimal chain: descriptors of stage 0 computed once and
+        // moved by constants, stage/phase counters kept incrementally, one
+        // try_wait per barrier when the phase has completed, one commit.
+        if (lane == 0) {
+            const uint64_t dA0 = tc_desc_sw128(smem_u32(sA)), dB0 = tc_desc_sw128(smem_u32(sB));
+            uint32_t st = 0, ph = 0;              // ring position, carried across items
+            uint64_t da = dA0, db = dB0;          // descriptors of stage st
+            int local = 0;
+            bool ok = true;
+            for (int64_t it = blockIdx.x; ok && it < nitems && !*abort_flag; it += gridDim.x, ++local) {
+                const TcItem d = tc_decode(p, pre, nslots, nu, it);
+                const int a = local & 1;
+                if (local >= 2 && !tc_wait(&acc_empty[(a) * TC_BS], ((local >> 1) - 1) & 1, abort_flag)) break;
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t d0 = tmem + (uint32_t)(a * 2 * TC_NMAX), d1 = d0 + TC_NMAX;
+                const uint32_t idesc = tc_idesc(d.nn);
+                for (int kb = 0; kb < p.kstages; ++kb) {
+                    if (!tc_wait_fast(&full_b[(st) * TC_BS], ph, abort_flag) || !tc_wait_fast(&full_a[(st) * TC_BS], ph, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    const uint32_t first = kb > 0 ? 1u : 0u;
+                    // descriptor units are 16 bytes: K step of 16 bf16 = 2, half of A = 1024
+                    tc_mma(d0, da, db, idesc, first);
+                    tc_mma(d0, da + 2, db + 2, idesc, 1u);
+                    tc_mma(d0, da + 4, db + 4, idesc, 1u);
+                    tc_mma(d0, da + 6, db + 6, idesc, 1u);
+                    tc_mma(d1, da + 1024, db, idesc, first);
+                    tc_mma(d1, da + 1026, db + 2, idesc, 1u);
+                    tc_mma(d1, da + 1028, db + 4, idesc, 1u);
+                    tc_mma(d1, da + 1030, db + 6, idesc, 1u);
+                    tc_commit(smem_u32(&empty[(st) * TC_BS]));
+                    if (++st == TC_S) {
+                        st = 0;
+                        ph ^= 1u;
+                        da = dA0;
+                        db = dB0;
+                    } else {
+                        da += TC_A_BYTES >> 4;
+                        db += TC_B_BYTES >> 4;
+                    }
                 }
-                const uint32_t raw = smem_u32(sb + TC_A_BYTES + TC_B_BYTES) + row * 32;
-                cp_async16(raw, W + kb * 32, 16);
-                cp_async16(raw + 16, W + kb * 32 + 16, 16);
-                const uint32_t bt = smem_u32(sb + TC_A_BYTES);
-                for (int q = tid; q < nn * 8; q += TC_LOADERS) {
-                    const int n = q >> 3, c = q & 7;
-                    const bool ok = n < nv;
-                    const __nv_bfloat16 *src = p.bsrc + (ok ? brow(n) : 0) * (int64_t)p.K + kb * 64 + c * 8;
-                    cp_async16(bt + n * 128 + ((c ^ (n & 7)) << 4), src, ok ? 16 : 0);
+                if (ok) tc_commit(smem_u32(&acc_full[(a) * TC_BS]));
+            }
+            // every MMA issued above has completed before TMEM is freed
+            tc_commit(smem_u32(drain));
+            if (!mbar_wait(smem_u32(drain), 0u)) raise_status(DERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else if (warp >= TC_EPI0 && warp < TC_EPI0 + 4) {
+        // ================= epilogue (warps 4..7) =================
+        const int q4 = warp & 3;                   // TMEM lane quarter of this warp
+        int local = 0;
+        for (int64_t it = blockIdx.x; it < nitems && !*abort_flag; it += gridDim.x, ++local) {
+            const TcItem d = tc_decode(p, pre, nslots, nu, it);
+            const float *sc_base = d.routed ? p.s + (int64_t)d.e * p.s_stride : p.s_sh;
+            const int row0 = d.mt * TC_M + q4 * 32 + lane;           // row of half 0
+            const float sc0 = sc_base[row0], sc1 = sc_base[row0 + TC_HALF];
+            const int64_t orow0 = d.routed ? d.b0 : p.sh_out_row0 + d.n0;
+            const int a = local & 1;
+            if (!tc_wait_warp(&acc_full[(a) * TC_BS], (local >> 1) & 1, abort_flag, 256)) break;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                const int rowg = row0 + hf * TC_HALF;
+                const float sc = hf ? sc1 : sc0;
+#pragma unroll 1
+                for (int c0 = 0; c0 < d.nn; c0 += 32) {
+                    uint32_t v[32];
+                    const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) +
+                                           (uint32_t)(a * 2 * TC_NMAX + hf * TC_NMAX + c0);
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+                        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+                          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+                          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+                          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+                          "=r"(v[31])
+                        : "r"(taddr));
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = c0 + j;
+                        const float acc = sc * __uint_as_float(v[j]);
+                        const int64_t orow = orow0 + n;
+                        if (p.gateup) {
+                            // gate on even rows, up on the odd row after it
+                            const float other = __shfl_xor_sync(0xffffffffu, acc, 1);
+                            if ((lane & 1) || n >= d.nv) continue;
+                            const int pair = rowg >> 1;
+                            const float h = silu_mul(acc, other);
+                            if (p.out) p.out[orow * p.out_ld + pair] = h;
+                            if (p.hperm)
+                                p.hperm[orow * (p.rows / 2) + (pair & ~7) + tc_inv_perm(pair & 7)] =
+                                    __float2bfloat16_rn(h);
+                        } else {
+                            if (n >= d.nv) continue;
+                            p.out[orow * p.out_ld + rowg] = acc;
+                        }
+                    }
                 }
-                asm volatile("cp.async.commit_group;" ::: "memory");
-            };
-            // prologue: the first stages of this item
-            int kissue = 0;
-            for (; kissue < TC_LOOKAHEAD && kissue < p.kstages; ++kissue) issue_stage(kissue, issued++);
-            for (int kb = 0; kb < p.kstages && !*abort_flag; ++kb, ++g) {
-                if (kissue < p.kstages) {
-                    issue_stage(kissue++, issued++);
-                } else {
-                    asm volatile("cp.async.commit_group;" ::: "memory");
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[(a) * TC_BS]));
+        }
+    } else if (tc_dq_index(warp) >= 0) {
+        // ================= dequantisers: thread r owns row r =================
+        const int r = tc_dq_index(warp) * 32 + lane;
+        const int hf = r >> 7, rr = r & 127, sw = rr & 7;
+        const __nv_bfloat162 off = __floats2bfloat162_rn(136.f, 136.f);
+        uint32_t g = 0, rg = 0;
+        bool ok = true;
+        for (int64_t it = blockIdx.x; ok && it < nitems && !*abort_flag; it += gridDim.x) {
+            for (int kb = 0; kb < p.kstages; ++kb) {
+                const uint32_t rs = rg % TC_RS;
+                if (kb % TC_RK == 0 && !tc_wait_warp(&raw_full[(rs) * TC_BS], (rg / TC_RS) & 1, abort_flag, 32)) {
+                    ok = false;
+                    break;
                 }
-                asm volatile("cp.async.wait_group %0;" ::"n"(TC_LOOKAHEAD) : "memory");
-                const int st = (int)(g % TC_STAGES);
-                unsigned char *sb = tsm + (size_t)st * TC_STAGE_BYTES;
-                // dequantise this thread's row: 64 codes -> 8 swizzled 16-byte chunks
-                const uint4 *rawp = reinterpret_cast<const uint4 *>(sb + TC_A_BYTES + TC_B_BYTES + row * 32);
-                const uint4 r0 = rawp[0], r1 = rawp[1];
+                const uint32_t st = g % TC_S;
+                if (g >= TC_S && !tc_wait_warp(&empty[(st) * TC_BS], ((g / TC_S) - 1) & 1, abort_flag, 32)) {
+                    ok = false;
+                    break;
+                }
+                // this row's 32 bytes of the stage: 16-byte chunks 2*sub and 2*sub+1
+                const unsigned char *rrow = sR + rs * TC_RAW_BYTES + hf * (TC_RAW_BYTES / 2) + rr * 128;
+                const int sub = kb % TC_RK;
+                const uint4 r0 = *reinterpret_cast<const uint4 *>(rrow + (((2 * sub) ^ sw) << 4));
+                const uint4 r1 = *reinterpret_cast<const uint4 *>(rrow + (((2 * sub + 1) ^ sw) << 4));
                 const uint32_t words[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-                const __nv_bfloat162 off = __floats2bfloat162_rn(136.f, 136.f);
+                unsigned char *arow = sA + st * TC_A_BYTES + hf * (TC_A_BYTES / 2) + rr * 128;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
+                    // two's-complement nibble -> offset binary -> bf16 (128 + code + 8) - 136
                     const uint32_t o = words[j] ^ 0x88888888u;
                     uint32_t q[4];
 #pragma unroll
@@ -269,157 +586,47 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_ffn_tc(const TcP p)
                         b = __hsub2(b, off);
                         q[h] = *reinterpret_cast<uint32_t *>(&b);
                     }
-                    *reinterpret_cast<uint4 *>(sb + row * 128 + ((j ^ (row & 7)) << 4)) =
-                        make_uint4(q[0], q[1], q[2], q[3]);
+                    *reinterpret_cast<uint4 *>(arow + ((j ^ sw) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                mbar_arrive(smem_u32(&full[st]));
-            }
-        }
-        asm volatile("cp.async.wait_all;" ::: "memory");
-    } else if (warp == 4) {
-        // ================= MMA issue =================
-        int64_t g = 0;
-        int local = 0;
-        for (int64_t it = blockIdx.x; it < nitems && !*abort_flag; it += gridDim.x, ++local) {
-            int s, mt, n0, nv, nn;
-            decode(it, s, mt, n0, nv, nn);
-            const int a = local & 1;
-            if (local >= 2 &&
-                !mbar_wait(smem_u32(&acc_empty[a]), (uint32_t)(((local >> 1) - 1) & 1))) {
-                *abort_flag = 1;
-                raise_status(DERR_TIMEOUT);
-                break;
-            }
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t d = tmem + (uint32_t)(a * TC_NMAX);
-            const uint32_t idesc = tc_idesc(nn);
-            for (int kb = 0; kb < p.kstages; ++kb, ++g) {
-                const int st = (int)(g % TC_STAGES);
-                if (!mbar_wait(smem_u32(&full[st]), (uint32_t)((g / TC_STAGES) & 1))) {
-                    *abort_flag = 1;
-                    raise_status(DERR_TIMEOUT);
-                    break;
-                }
-                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                if (lane == 0) {
-                    unsigned char *sb = tsm + (size_t)st * TC_STAGE_BYTES;
-                    const uint64_t da = tc_desc_sw128(smem_u32(sb));
-                    const uint64_t db = tc_desc_sw128(smem_u32(sb + TC_A_BYTES));
-#pragma unroll
-                    for (int k = 0; k < TC_BK / 16; ++k) {
-                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-                        asm volatile(
-                            "{\n\t.reg .pred pd;\n\t"
-                            "setp.ne.b32 pd, %4, 0;\n\t"
-                            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, pd;\n\t}"
-                            ::"r"(d), "l"(da + 2 * k), "l"(db + 2 * k), "r"(idesc), "r"(acc),
-                            "r"(0), "r"(0), "r"(0), "r"(0)
-                            : "memory");
-                    }
-                    asm volatile(
-                        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                            smem_u32(&empty[st]))
-                        : "memory");
-                }
                 __syncwarp();
-            }
-            if (*abort_flag) break;
-            if (lane == 0)
-                asm volatile(
-                    "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                        smem_u32(&acc_full[a]))
-                    : "memory");
-            __syncwarp();
-        }
-        // every MMA issued above has completed before TMEM is freed
-        if (lane == 0) {
-            asm volatile(
-                "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                    smem_u32(drain))
-                : "memory");
-            if (!mbar_wait(smem_u32(drain), 0u)) raise_status(DERR_TIMEOUT);
-        }
-        __syncwarp();
-    } else {
-        // ================= epilogue (warps 5..8) =================
-        const int q4 = warp & 3;                   // TMEM lane quarter of this warp
-        const int lrow = q4 * 32 + lane;           // accumulator row = weight row in tile
-        int local = 0;
-        for (int64_t it = blockIdx.x; it < nitems && !*abort_flag; it += gridDim.x, ++local) {
-            int s, mt, n0, nv, nn;
-            decode(it, s, mt, n0, nv, nn);
-            const bool routed = s < nu;
-            int e = 0, p0 = 0;
-            if (routed) {
-                e = p.union_ids[s];
-                e = (e >= 0 && e < p.E) ? e : 0;
-                p0 = p.offsets[e];
-            }
-            const int rowg = mt * TC_M + lrow;
-            const float sc = (routed ? p.s + (int64_t)e * p.s_stride : p.s_sh)[rowg];
-            const int a = local & 1;
-            if (!mbar_wait(smem_u32(&acc_full[a]), (uint32_t)((local >> 1) & 1))) {
-                *abort_flag = 1;
-                raise_status(DERR_TIMEOUT);
-                break;
-            }
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            for (int c0 = 0; c0 < nn; c0 += 16) {
-                uint32_t v[16];
-                const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(a * TC_NMAX + c0);
-                asm volatile(
-                    "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                      "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-                      "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-                    : "r"(taddr));
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int n = c0 + j;
-                    const float acc = sc * __uint_as_float(v[j]);
-                    const int i = n0 + n;
-                    int orow;
-                    if (p.gateup) {
-                        const float other = __shfl_xor_sync(0xffffffffu, acc, 1);
-                        if ((lane & 1) || n >= nv) continue;
-                        orow = routed ? p0 + i : (int)p.sh_out_row0 + i;
-                        const int pair = rowg >> 1;
-                        const float h = silu_mul(acc, other);
-                        p.out[(int64_t)orow * p.out_ld + pair] = h;
-                        if (p.hperm)
-                            p.hperm[(int64_t)orow * (p.rows / 2) + (pair & ~7) + tc_inv_perm(pair & 7)] =
-                                __float2bfloat16_rn(h);
-                    } else {
-                        if (n >= nv) continue;
-                        orow = routed ? p0 + i : (int)p.sh_out_row0 + i;
-                        p.out[(int64_t)orow * p.out_ld + rowg] = acc;
-                    }
+                if (lane == 0) mbar_arrive(smem_u32(&full_a[(st) * TC_BS]));
+                ++g;
+                if (sub == TC_RK - 1) {
+                    if (lane == 0) mbar_arrive(smem_u32(&raw_empty[(rs) * TC_BS]));
+                    ++rg;
                 }
             }
-            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[a]));
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
-    if (warp == 4) {
+    if (warp == TC_MMA) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
     }
 }
 
-// x (bf16 [T][K]) -> chunk-permuted copy; h (f32 rows, stride ld) -> bf16 chunk-permuted.
-__global__ void __launch_bounds__(256) k_perm_bf16(const __nv_bfloat16 *__restrict__ x, int64_t rows,
-                                                   int K, __nv_bfloat16 *__restrict__ out)
+// B rows for gate/up: row r < A is the token of sorted assignment r, rows
+// A..A+T-1 are the tokens in order (shared expert); each row chunk-permuted.
+__global__ void __launch_bounds__(256) k_gather_x(const __nv_bfloat16 *__restrict__ x, int T, int H,
+                                                  const int32_t *__restrict__ sorted, int64_t A, int k,
+                                                  int64_t rows, __nv_bfloat16 *__restrict__ out)
 {
     pdl_wait();
     pdl_trigger();
     const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (id >= rows * (K / 8)) return;
-    const uint4 v = reinterpret_cast<const uint4 *>(x)[id];
+    const int chunks = H / 8;
+    if (id >= rows * chunks) return;
+    const int64_t r = id / chunks;
+    const int c = (int)(id % chunks);
+    int64_t t = r - A;
+    if (r < A) {
+        const int32_t a = sorted[r];
+        t = (a >= 0 && a < A) ? a / k : -1;
+    }
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (t >= 0 && t < T) v = reinterpret_cast<const uint4 *>(x + t * H)[c];
     const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&v);
     __nv_bfloat16 o[8];
 #pragma unroll
@@ -427,6 +634,7 @@ __global__ void __launch_bounds__(256) k_perm_bf16(const __nv_bfloat16 *__restri
     reinterpret_cast<uint4 *>(out)[id] = *reinterpret_cast<const uint4 *>(o);
 }
 
+// h (f32 rows, stride ld) -> bf16 chunk-permuted rows.
 __global__ void __launch_bounds__(256) k_perm_f32(const float *__restrict__ h, int64_t ld, int64_t rows,
                                                   int K, __nv_bfloat16 *__restrict__ out)
 {
@@ -444,20 +652,81 @@ __global__ void __launch_bounds__(256) k_perm_f32(const float *__restrict__ h, i
     reinterpret_cast<uint4 *>(out)[id] = *reinterpret_cast<const uint4 *>(o);
 }
 
+// ---------------------------------------------------------------- host side
 constexpr int TC_MIN_T = 256;   // tokens from which the tensor-core path is used
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 tc_encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        else
+            (void)cudaGetLastError();
+    });
+    return fn;
+}
+
+// Packed weight rows of nexp experts: u8 [nexp][rows][row_bytes]; box 128 B x 128 rows.
+static bool tc_map_weights(CUtensorMap *m, const void *w, int row_bytes, int rows, int nexp, int64_t stride)
+{
+    const auto fn = tc_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)nexp};
+    const cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)stride};
+    const cuuint32_t box[3] = {128, (cuuint32_t)TC_HALF, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(w), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 rows [nrows][K]; box 64 elements x 32 rows.
+static bool tc_map_rows(CUtensorMap *m, const void *b, int K, int64_t nrows)
+{
+    const auto fn = tc_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)nrows};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)TC_BK, (cuuint32_t)TC_BOX_ROWS};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(b), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tc_shape_ok(int afmt, int wbits, int64_t T, int64_t H, int64_t I)
+{
+    return afmt == QRX_A_BF16 && wbits == 4 && T >= TC_MIN_T && H % (TC_BK * TC_RK) == 0 &&
+           I % (TC_BK * TC_RK) == 0 && H % TC_M == 0 && (2 * I) % TC_M == 0 && tc_encode_fn() != nullptr;
+}
 
 bool ffn_use_tc(const FfnArgs &a)
 {
-    return a.afmt == QRX_A_BF16 && a.wbits == 4 && a.T >= TC_MIN_T && (2 * a.I) % TC_M == 0 &&
-           a.H % TC_M == 0 && a.H % TC_BK == 0 && a.I % TC_BK == 0 && a.xperm && a.hperm;
+    return tc_shape_ok(a.afmt, a.wbits, a.T, a.H, a.I) && a.xperm && a.hperm;
 }
 
-static cudaError_t tc_go(TcP &p, int num_sms, cudaStream_t st, int maxslots)
+static cudaError_t tc_go(TcP &p, const void *w, const void *w_sh, int64_t w_stride, const void *b,
+                         int64_t brows, int num_sms, cudaStream_t st, int maxslots)
 {
-    p.row_bytes = p.K / 2;
     p.mtiles = p.rows / TC_M;
     p.kstages = p.K / TC_BK;
+    const int row_bytes = p.K / 2;
+    CUtensorMap mw, mwsh, mb;
+    bool ok = true;
+    if (p.routed) ok = ok && tc_map_weights(&mw, w, row_bytes, p.rows, p.E, w_stride);
+    if (p.shared) ok = ok && tc_map_weights(&mwsh, w_sh, row_bytes, p.rows, 1, (int64_t)p.rows * row_bytes);
+    if (!p.routed) mw = mwsh;
+    if (!p.shared) mwsh = mw;
+    ok = ok && tc_map_rows(&mb, b, p.K, brows);
+    if (!ok) return cudaErrorInvalidValue;
     const int smem = tc_smem_bytes(maxslots);
+    if (smem > GV_SMEM_MAX) return cudaErrorInvalidValue;
     static unsigned long long configured = 0;
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -467,8 +736,7 @@ static cudaError_t tc_go(TcP &p, int num_sms, cudaStream_t st, int maxslots)
         if (err != cudaSuccess) return err;
         if (dev < 64) configured |= 1ull << dev;
     }
-    if (smem > GV_SMEM_MAX) return cudaErrorInvalidValue;
-    return launch_k(k_ffn_tc, dim3(num_sms), dim3(TC_THREADS), (size_t)smem, st, p);
+    return launch_k(k_ffn_tc, dim3(num_sms), dim3(TC_THREADS), (size_t)smem, st, mw, mwsh, mb, p);
 }
 
 static void tc_common(TcP &p, const FfnArgs &a)
@@ -479,43 +747,43 @@ static void tc_common(TcP &p, const FfnArgs &a)
     p.k = a.k;
     p.T = a.T;
     p.offsets = a.offsets;
-    p.sorted = a.sorted;
     p.union_ids = a.union_ids;
     p.n_union = a.n_union;
 }
 
 cudaError_t launch_ffn_tc_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
 {
-    __nv_bfloat16 *xperm = static_cast<__nv_bfloat16 *>(a.xperm);
-    const int64_t n = (int64_t)a.T * (a.H / 8);
-    cudaError_t err = launch_k(k_perm_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st,
-                               static_cast<const __nv_bfloat16 *>(a.x), (int64_t)a.T, a.H, xperm);
+    if (!a.routed && !a.shared) return cudaSuccess;
+    const int64_t A = a.routed ? (int64_t)a.T * a.k : 0;
+    const int64_t rows = A + (a.shared ? a.T : 0);
+    __nv_bfloat16 *xs = static_cast<__nv_bfloat16 *>(a.xperm);
+    const int64_t n = rows * (a.H / 8);
+    cudaError_t err = launch_k(k_gather_x, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st,
+                               static_cast<const __nv_bfloat16 *>(a.x), a.T, a.H, a.sorted, A, a.k, rows, xs);
     if (err != cudaSuccess) return err;
     TcP p{};
     tc_common(p, a);
     p.rows = 2 * a.I;
     p.K = a.H;
-    p.w = a.w13;
-    p.w_stride = (int64_t)2 * a.I * (a.H / 2);
     p.s = a.s13;
     p.s_stride = 2 * a.I;
-    p.w_sh = a.w13_sh;
     p.s_sh = a.s13_sh;
-    p.bsrc = xperm;
-    p.sh_in_row0 = 0;
+    p.b_sh_row0 = A;
     p.out = a.h;
     p.out_ld = a.h_ld;
     p.sh_out_row0 = a.sh_h_row0;
     p.hperm = static_cast<__nv_bfloat16 *>(a.hperm);
     p.gateup = 1;
-    return tc_go(p, num_sms, st, a.E + 1);
+    return tc_go(p, a.w13, a.w13_sh, (int64_t)2 * a.I * (a.H / 2), xs, rows, num_sms, st, a.E + 1);
 }
 
 cudaError_t launch_ffn_tc_down(const FfnArgs &a, int num_sms, cudaStream_t st)
 {
+    if (!a.routed && !a.shared) return cudaSuccess;
     __nv_bfloat16 *hperm = static_cast<__nv_bfloat16 *>(a.hperm);
+    const int64_t rows = std::max(a.routed ? (int64_t)a.T * a.k : (int64_t)0,
+                                  a.shared ? a.sh_h_row0 + a.T : (int64_t)0);
     if (!a.hperm_ready) {       // h given in f32: round to bf16 and permute it here
-        const int64_t rows = max(a.routed ? (int64_t)a.T * a.k : 0, a.shared ? a.sh_h_row0 + a.T : 0);
         const int64_t n = rows * (a.I / 8);
         cudaError_t err = launch_k(k_perm_f32, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st,
                                    (const float *)a.h, a.h_ld, rows, a.I, hperm);
@@ -525,20 +793,16 @@ cudaError_t launch_ffn_tc_down(const FfnArgs &a, int num_sms, cudaStream_t st)
     tc_common(p, a);
     p.rows = a.H;
     p.K = a.I;
-    p.w = a.w2;
-    p.w_stride = (int64_t)a.H * (a.I / 2);
     p.s = a.s2;
     p.s_stride = a.H;
-    p.w_sh = a.w2_sh;
     p.s_sh = a.s2_sh;
-    p.bsrc = hperm;
-    p.sh_in_row0 = a.sh_h_row0;
+    p.b_sh_row0 = a.sh_h_row0;
     p.out = a.y;
     p.out_ld = a.y_ld;
     p.sh_out_row0 = a.sh_y_row0;
     p.hperm = nullptr;
     p.gateup = 0;
-    return tc_go(p, num_sms, st, a.E + 1);
+    return tc_go(p, a.w2, a.w2_sh, (int64_t)a.H * (a.I / 2), hperm, rows, num_sms, st, a.E + 1);
 }
 
 }  // namespace qrx

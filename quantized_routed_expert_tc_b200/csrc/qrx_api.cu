@@ -88,7 +88,7 @@ Ws ws_layout(const qrx_cfg *c, int T)
     L.xd = take((size_t)T * (H / 32) * 4);
     L.xrec = take(act_records_bytes(c->afmt, (int)H, T));
     L.hrec = take(act_records_bytes(c->afmt, (int)I, (int)(A + T)));
-    L.xperm = take((size_t)T * H * 2);
+    L.xperm = take((size_t)(A + T) * H * 2);     // tokens gathered in expert order, then in order
     L.hperm = take((size_t)(A + T) * I * 2);
     L.h = take((size_t)(A + T) * I * 4);
     L.y = take((size_t)(A + T) * H * 4);
@@ -137,8 +137,9 @@ int check_experts(const qrx_experts *x)
 int check_act(const qrx_cfg *c, const qrx_act *a)
 {
     if (!a) return QRX_EINVAL;
-    if (c->afmt == QRX_A_Q8_0) return (a->xq && a->xd) ? QRX_OK : QRX_EINVAL;
-    return a->x ? QRX_OK : QRX_EINVAL;
+    if (c->afmt == QRX_A_Q8_0)
+        return (a->xq && a->xd && aligned(a->xq, 16) && aligned(a->xd, 16)) ? QRX_OK : QRX_EINVAL;
+    return (a->x && aligned(a->x, 16)) ? QRX_OK : QRX_EINVAL;
 }
 
 int check_perm(const qrx_perm *p)
@@ -216,6 +217,12 @@ size_t qrx_workspace_bytes(const qrx_cfg *c, int32_t T)
 {
     if (qrx_validate(c) != QRX_OK || T <= 0) return 0;
     return ws_layout(c, T).total;
+}
+
+int qrx_ffn_engine(const qrx_cfg *c, int32_t T)
+{
+    if (qrx_validate(c) != QRX_OK || T <= 0) return QRX_EINVAL;
+    return tc_shape_ok(c->afmt, c->wfmt, T, c->hidden, c->inter) ? QRX_ENGINE_TC : QRX_ENGINE_GEMV;
 }
 
 int qrx_last_error(void)
@@ -332,6 +339,7 @@ int qrx_expert_ffn(const qrx_cfg *c, const qrx_experts *routed, const qrx_perm *
     a.h_ld = c->inter;
     a.y = y_sorted;
     a.y_ld = c->hidden;
+    if (!h_sorted && ffn_use_tc(a)) a.h = nullptr;   // down reads the bf16 copy of h
     const int sms = num_sms_current();
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = launch_ffn_gateup(a, sms, st);
@@ -418,6 +426,7 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     int v = check_common(c, T);
     if (v) return v;
     if (!x || !Wr || !bias || !topk_idx || !topk_w || !out) return QRX_EINVAL;
+    if (!aligned(x, 16)) return QRX_EINVAL;
     if ((v = check_experts(routed))) return v;
     if (shared && (v = check_experts(shared))) return v;
     if ((v = check_ws(c, T, ws, ws_bytes))) return v;
@@ -453,7 +462,7 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     set_routed(a, routed, &perm);
     if (shared) set_shared(a, shared);
     a.prep_records = 0;
-    a.h = h;
+    a.h = tc ? nullptr : h;       // the tensor-core down projection reads the bf16 copy of h
     a.h_ld = c->inter;
     a.y = y;
     a.y_ld = c->hidden;

@@ -87,6 +87,7 @@ struct FfnArgs {
 };
 cudaError_t launch_act_digits(const FfnArgs &a, cudaStream_t st);
 bool ffn_use_tc(const FfnArgs &a);
+bool tc_shape_ok(int afmt, int wbits, int64_t T, int64_t H, int64_t I);
 cudaError_t launch_ffn_tc_gateup(const FfnArgs &a, int num_sms, cudaStream_t st);
 cudaError_t launch_ffn_tc_down(const FfnArgs &a, int num_sms, cudaStream_t st);
 cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st);

@@ -18,6 +18,7 @@ from . import build as _build
 
 QRX_OK, QRX_EINVAL, QRX_EUNSUPPORTED, QRX_ECUDA, QRX_ETIMEOUT, QRX_EDEVICE, QRX_ENOSPACE = \
     0, -1, -2, -3, -4, -5, -6
+QRX_ENGINE_GEMV, QRX_ENGINE_TC = 0, 1
 W_INT8, W_INT4, W_INT2 = 8, 4, 2
 A_F32, A_Q8_0, A_BF16 = 0, 1, 2
 
@@ -59,6 +60,7 @@ P = ctypes.POINTER
 _SIGS = {
     "qrx_validate": ([P(Cfg)], ctypes.c_int),
     "qrx_workspace_bytes": ([P(Cfg), i32], sz),
+    "qrx_ffn_engine": ([P(Cfg), i32], ctypes.c_int),
     "qrx_last_error": ([], ctypes.c_int),
     "qrx_strerror": ([ctypes.c_int], ctypes.c_char_p),
     "qrx_quantize_weights": ([vp, i64, i64, i32, vp, i64, vp, i64, vp], ctypes.c_int),
@@ -193,6 +195,14 @@ def qrx_validate(cfg: Cfg) -> int:
 
 def qrx_workspace_bytes(cfg: Cfg, T: int) -> int:
     return lib().qrx_workspace_bytes(ctypes.byref(cfg), T)
+
+
+def qrx_ffn_engine(cfg: Cfg, T: int) -> int:
+    """QRX_ENGINE_TC or QRX_ENGINE_GEMV: the expert-FFN engine for this cfg and T."""
+    v = lib().qrx_ffn_engine(ctypes.byref(cfg), T)
+    if v < 0:
+        raise QrxError("qrx_ffn_engine", v)
+    return v
 
 
 def qrx_last_error() -> int:

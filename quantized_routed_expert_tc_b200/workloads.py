@@ -95,5 +95,10 @@ def sweep() -> list[Workload]:
     return out
 
 
+# Smallest layer the tensor-core expert engine takes (bf16 x int4, T >= 256,
+# hidden and inter multiples of 256): 2 row tiles per projection, 8 K stages
+# for gate/up, experts with more tokens than one 128-token tile.
+SMALL_TC = TINY.with_(name="small_t300_int4_bf16", hidden=512, inter=256, afmt=A_BF16, T=300)
+
 ALL = {w.name: w for w in [TINY, GLM_DECODE_T1, GLM_DECODE_T32_Q8, GLM_VERIFY_T4_BF16,
-                           GLM_PREFILL_T2048_BF16, *sweep()]}
+                           GLM_PREFILL_T2048_BF16, SMALL_TC, *sweep()]}

@@ -36,6 +36,11 @@ def tiny(dev):
 
 
 @pytest.fixture(scope="session")
+def small_tc(dev):
+    return GpuLayer(W.SMALL_TC, formats=(4,)), OracleLayer(W.SMALL_TC)
+
+
+@pytest.fixture(scope="session")
 def glm(dev):
     return GpuLayer(W.GLM_DECODE_T1, formats=(4, 8, 2)), OracleLayer(W.GLM_DECODE_T1)
 
@@ -306,35 +311,64 @@ def test_tiny_large_batch_many_token_groups(tiny):
         check_layer(glay, olay, wl, x, [0, 77, 299])
 
 
-def test_tiny_bf16_many_tokens_tensor_cores(tiny):
-    """T >= 256 with bf16 activations runs the expert FFN as tcgen05 grouped GEMMs."""
+def test_tiny_bf16_many_tokens_gemv(tiny):
+    """bf16 with many tokens but inter = 128 (not a multiple of 256): the GEMV engine."""
     glay, olay = tiny
-    for T in (256, 300):
-        wl = W.TINY.with_(T=T, afmt=W.A_BF16)
-        x = activations(wl, T, batch=4)
-        check_layer(glay, olay, wl, x, [0, 131, T - 1])
-    # stage isolation: the down projection from the oracle's h, and h itself
     wl = W.TINY.with_(T=300, afmt=W.A_BF16)
-    x = activations(wl, 300, batch=4)
+    assert qrx.qrx_ffn_engine(qrx.cfg_of(wl), 300) == qrx.QRX_ENGINE_GEMV
+    check_layer(glay, olay, wl, activations(wl, 300, batch=4), [0, 131, 299])
+
+
+def test_small_bf16_tensor_cores_all_tokens(small_tc):
+    """tcgen05 grouped GEMMs: every token of ragged batches, expert tiles split in N."""
+    glay, olay = small_tc
+    for T in (256, 300, 517):
+        wl = W.SMALL_TC.with_(T=T)
+        assert qrx.qrx_ffn_engine(qrx.cfg_of(wl), T) == qrx.QRX_ENGINE_TC
+        assert qrx.qrx_ffn_engine(qrx.cfg_of(wl), 255) == qrx.QRX_ENGINE_GEMV
+        check_layer(glay, olay, wl, activations(wl, T, batch=4 + T), range(T))
+
+
+def test_small_bf16_tensor_cores_skewed_routing(small_tc):
+    """A bias that sends every token to experts 0..3: 300 tokens per expert, three
+    N tiles each, 12 of 16 experts idle."""
+    glay, olay = small_tc
+    wl = W.SMALL_TC
+    bias = np.zeros(wl.n_experts, np.float32)
+    bias[:4] = 10.0
+    res = check_layer(glay, olay, wl, activations(wl, 300, batch=9), [0, 100, 299], bias_np=bias)
+    assert sorted(np.unique(res["idx"]).tolist()) == [0, 1, 2, 3]
+
+
+def test_small_bf16_tensor_cores_stages(small_tc):
+    """Stage isolation on the tensor-core engine: h and y of the routed FFN, and the
+    down projection alone from the oracle's h."""
+    glay, olay = small_tc
+    wl = W.SMALL_TC
+    T = wl.T
+    x = activations(wl, T, batch=4)
     _, bias = router_weights(wl)
     r = oracle.router(wl, x, olay.Wr, bias)
     p = oracle.permute(r["idx"], wl.n_experts)
     ex = olay.experts(r["idx"].ravel(), wl.wbits)
     h_o, y_o = oracle.expert_ffn(wl, ex, p, x)
     c = qrx.cfg_of(wl)
-    ws = qrx.workspace(c, 300)
-    perm = qrx.Perm.empty(300, wl.top_k, wl.n_experts)
+    ws = qrx.workspace(c, T)
+    perm = qrx.Perm.empty(T, wl.top_k, wl.n_experts)
     qrx.qrx_permute(c, cu(r["idx"]), perm)
-    A = 300 * wl.top_k
+    A = T * wl.top_k
     hs = torch.empty((A, wl.inter), dtype=torch.float32, device="cuda")
     ys = torch.empty((A, wl.hidden), dtype=torch.float32, device="cuda")
-    qrx.qrx_expert_ffn(c, glay.routed[4], perm, 300, ys, ws, x=to_device_act(wl, x), h_sorted=hs)
+    qrx.qrx_expert_ffn(c, glay.routed[4], perm, T, ys, ws, x=to_device_act(wl, x), h_sorted=hs)
+    ys2 = torch.full((A, wl.hidden), float("nan"), dtype=torch.float32, device="cuda")
+    qrx.qrx_expert_ffn(c, glay.routed[4], perm, T, ys2, ws, x=to_device_act(wl, x))
     yd = torch.empty((A, wl.hidden), dtype=torch.float32, device="cuda")
-    qrx.qrx_expert_down(c, glay.routed[4], perm, cu(h_o), 300, yd, ws)
+    qrx.qrx_expert_down(c, glay.routed[4], perm, cu(h_o), T, yd, ws)
     torch.cuda.synchronize()
     assert qrx.qrx_last_error() == qrx.QRX_OK
     assert rel_err(np_(hs), h_o) <= TOL
     assert rel_err(np_(ys), y_o) <= TOL
+    assert np.array_equal(np_(ys2), np_(ys))          # without h_sorted: same y
     assert rel_err(np_(yd), y_o) <= TOL
 
 
