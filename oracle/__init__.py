@@ -79,6 +79,10 @@ def _load():
                 "qo_combine": ([P(Cfg), ctypes.c_int, vp, vp, vp, vp, vp], None),
                 "qo_moe_forward": ([P(Cfg), vp, ctypes.c_int, vp, vp, vp, P(CExpert), vp, vp, vp],
                                    None),
+                "qo_moe_forward_opts": ([P(Cfg), vp, ctypes.c_int, vp, vp, vp, P(CExpert),
+                                         ctypes.c_double, vp, vp, vp], None),
+                "qo_topp_prune": ([ctypes.c_int, ctypes.c_int, ctypes.c_double, f32, vp, vp],
+                                  i64),
             }
             for name, (args, res) in sig.items():
                 fn = getattr(lib, name)
@@ -296,8 +300,26 @@ def combine(w, y_sorted: np.ndarray, y_sh, wt: np.ndarray, inv: np.ndarray):
     return out
 
 
+def topp_prune(idx: np.ndarray, wt: np.ndarray, p: float, rsf: float):
+    """Adaptive expert top-p on the router's output (copies): (idx, w, kept)."""
+    idx = _c(idx, np.int32).copy()
+    wt = _c(wt, np.float32).copy()
+    T, k = idx.shape
+    # p and rsf are f32 values at the library's boundary: the threshold is
+    # (double)p * (double)rsf of those
+    kept = _load().qo_topp_prune(T, k, float(np.float32(p)), float(np.float32(rsf)), _p(idx), _p(wt))
+    return idx, wt, int(kept)
+
+
+def usage(idx: np.ndarray, E: int) -> np.ndarray:
+    """Expert-usage histogram of one layer call: assignments per expert (dropped
+    slots, idx = -1, not counted)."""
+    idx = np.asarray(idx).ravel()
+    return np.bincount(idx[idx >= 0], minlength=E).astype(np.uint64)
+
+
 def moe_forward(w, act: np.ndarray, Wr: np.ndarray, bias: np.ndarray, experts: dict,
-                shared: Expert | None):
+                shared: Expert | None, topp: float = 0.0):
     act = _act(w, act)
     T = act.shape[0]
     idx = np.zeros((T, w.top_k), np.int32)
@@ -306,6 +328,7 @@ def moe_forward(w, act: np.ndarray, Wr: np.ndarray, bias: np.ndarray, experts: d
     tab = _expert_table(experts, w.n_experts)
     c = cfg_struct(w)
     sh = None if shared is None else ctypes.byref(shared.cstruct())
-    _load().qo_moe_forward(ctypes.byref(c), _p(act), T, _p(_c(Wr, np.float32)),
-                           _p(_c(bias, np.float32)), tab, sh, _p(idx), _p(wt), _p(out))
+    _load().qo_moe_forward_opts(ctypes.byref(c), _p(act), T, _p(_c(Wr, np.float32)),
+                                _p(_c(bias, np.float32)), tab, sh, float(np.float32(topp)), _p(idx), _p(wt),
+                                _p(out))
     return idx, wt, out

@@ -350,6 +350,54 @@ void qo_router(const qo_cfg *c, const void *act, int T, const float *Wr,
 }
 
 /* ------------------------------------------------------------------------ */
+/* adaptive expert top-p                                                    */
+/* ------------------------------------------------------------------------ */
+/* README "JustVugg/colibri", section "快速开始" (the --topp knob, adaptive
+ * expert top-p, default 0.7) and "社区基准（实测）" (its measured effect):
+ * drop the low-weight experts of each token so fewer experts are read.
+ * [reading] applied to the router's output, per token: the k selections are
+ * ordered by weight, largest first (equal weights: the lower slot j first);
+ * the shortest leading run whose weights summed in that order (in double)
+ * reach p * rsf (p of the total weight, which is rsf) is kept; every other
+ * slot becomes idx = -1, w = 0.  [reading] the kept weights are not
+ * renormalised.  p outside (0, 1) keeps every slot (so does k > 64, beyond
+ * this reference's scratch).  Returns the number of slots kept. */
+int64_t qo_topp_prune(int T, int k, double p, float rsf, int32_t *idx, float *w)
+{
+    if (!(p > 0.0 && p < 1.0) || k > 64) return (int64_t)T * k;
+    const double thr = p * (double)rsf;
+    int64_t kept = 0;
+    int order[64];
+    for (int t = 0; t < T; ++t) {
+        int32_t *it = idx + (int64_t)t * k;
+        float *wt = w + (int64_t)t * k;
+        for (int j = 0; j < k; ++j) order[j] = j;
+        /* insertion sort: weight descending, slot ascending */
+        for (int i = 1; i < k; ++i) {
+            int j = i, v = order[i];
+            while (j > 0 && (wt[order[j - 1]] < wt[v] || (wt[order[j - 1]] == wt[v] && order[j - 1] > v))) {
+                order[j] = order[j - 1];
+                --j;
+            }
+            order[j] = v;
+        }
+        double c = 0.0;
+        int n = 0;
+        while (n < k) {
+            c += (double)wt[order[n]];
+            ++n;
+            if (c >= thr) break;
+        }
+        for (int i = n; i < k; ++i) {
+            it[order[i]] = -1;
+            wt[order[i]] = 0.0f;
+        }
+        kept += n;
+    }
+    return kept;
+}
+
+/* ------------------------------------------------------------------------ */
 /* permutation (batch-union)                                                */
 /* ------------------------------------------------------------------------ */
 /* README "已实现的功能" (batch-union MoE) and the blog's "同一批次里相同的专家
@@ -357,19 +405,26 @@ void qo_router(const qo_cfg *c, const void *act, int T, const float *Wr,
  * present in the batch is visited once for all its positions.
  * [reading] the order is fixed so the result is unique: a stable counting
  * sort by (expert, a).  counts[E], offsets[E+1] (exclusive prefix sum),
- * sorted[p] = a, inv[a] = p, union_ids = experts with count > 0 ascending. */
+ * sorted[p] = a, inv[a] = p, union_ids = experts with count > 0 ascending.
+ * A slot with idx = -1 (dropped by adaptive top-p, below) takes no position:
+ * it is not counted and inv[a] = -1. */
 void qo_permute(const int32_t *idx, int T, int k, int E, int32_t *counts,
                 int32_t *offsets, int32_t *sorted, int32_t *inv,
                 int32_t *union_ids, int32_t *n_union)
 {
     const int64_t A = (int64_t)T * k;
     for (int e = 0; e < E; ++e) counts[e] = 0;
-    for (int64_t a = 0; a < A; ++a) counts[idx[a]]++;
+    for (int64_t a = 0; a < A; ++a)
+        if (idx[a] >= 0) counts[idx[a]]++;
     offsets[0] = 0;
     for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
     int32_t *cursor = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
     for (int e = 0; e < E; ++e) cursor[e] = offsets[e];
     for (int64_t a = 0; a < A; ++a) {
+        if (idx[a] < 0) {          /* slot dropped by adaptive top-p: no position */
+            inv[a] = -1;
+            continue;
+        }
         int32_t p = cursor[idx[a]]++;
         sorted[p] = (int32_t)a;
         inv[a] = p;
@@ -550,7 +605,7 @@ void qo_shared_ffn(const qo_cfg *c, const qo_expert *shared, const void *act, in
 
 /* Weighted combine: out[t] = y_sh[t] + sum_j w[t,j] * y_sorted[inv[t*k+j]],
  * summed in double in j order, rounded to f32.  y_sh may be NULL (no shared
- * expert term). */
+ * expert term).  Slots with inv = -1 (dropped) contribute nothing. */
 void qo_combine(const qo_cfg *c, int T, const float *y_sorted, const float *y_sh,
                 const float *w, const int32_t *inv, float *out)
 {
@@ -561,17 +616,19 @@ void qo_combine(const qo_cfg *c, int T, const float *y_sorted, const float *y_sh
             double acc = y_sh ? (double)y_sh[(int64_t)t * H + h] : 0.0;
             for (int j = 0; j < k; ++j) {
                 int64_t a = (int64_t)t * k + j;
+                if (inv[a] < 0) continue;          /* dropped slot */
                 acc += (double)w[a] * (double)y_sorted[(int64_t)inv[a] * H + h];
             }
             out[(int64_t)t * H + h] = (float)acc;
         }
 }
 
-/* The whole layer: route, permute, routed FFN over the union, shared expert,
- * combine.  Scratch is allocated here (this is the slow reference). */
-void qo_moe_forward(const qo_cfg *c, const void *act, int T, const float *Wr,
-                    const float *bias, const qo_expert *experts, const qo_expert *shared,
-                    int32_t *idx, float *w, float *out)
+/* The whole layer: route, (adaptive top-p when 0 < topp < 1), permute,
+ * routed FFN over the union, shared expert, combine.  Scratch is allocated
+ * here (this is the slow reference). */
+void qo_moe_forward_opts(const qo_cfg *c, const void *act, int T, const float *Wr,
+                         const float *bias, const qo_expert *experts, const qo_expert *shared,
+                         double topp, int32_t *idx, float *w, float *out)
 {
     const int E = c->n_experts, k = c->top_k, H = c->hidden;
     const int64_t A = (int64_t)T * k;
@@ -584,9 +641,17 @@ void qo_moe_forward(const qo_cfg *c, const void *act, int T, const float *Wr,
     float *ysh = shared ? (float *)malloc(sizeof(float) * (size_t)T * H) : NULL;
     int32_t nu = 0;
     qo_router(c, act, T, Wr, bias, idx, w, NULL, NULL, NULL);
+    qo_topp_prune(T, k, topp, c->routed_scaling_factor, idx, w);
     qo_permute(idx, T, k, E, counts, offsets, sorted, inv, uid, &nu);
     qo_expert_ffn(c, experts, offsets, sorted, uid, nu, act, NULL, ys);
     if (shared) qo_shared_ffn(c, shared, act, T, NULL, ysh);
     qo_combine(c, T, ys, ysh, w, inv, out);
     free(counts); free(offsets); free(sorted); free(inv); free(uid); free(ys); free(ysh);
+}
+
+void qo_moe_forward(const qo_cfg *c, const void *act, int T, const float *Wr,
+                    const float *bias, const qo_expert *experts, const qo_expert *shared,
+                    int32_t *idx, float *w, float *out)
+{
+    qo_moe_forward_opts(c, act, T, Wr, bias, experts, shared, 0.0, idx, w, out);
 }

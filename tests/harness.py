@@ -34,18 +34,21 @@ class OracleLayer:
     def shared(self, bits=None) -> oracle.Expert:
         return self.expert(self.wl.n_experts, bits)
 
-    def forward_tokens(self, wl, x: np.ndarray, tokens, bias=None):
+    def forward_tokens(self, wl, x: np.ndarray, tokens, bias=None, topp: float = 0.0):
         """Oracle layer output rows for the listed tokens of batch x (routing uses the
-        tokens' own rows; every token is independent)."""
+        tokens' own rows; every token is independent).  topp in (0, 1): adaptive
+        expert top-p on the router's output (r then holds the pruned idx, w)."""
         bias = self.bias if bias is None else bias
         r = oracle.router(wl, x, self.Wr, bias)
+        if 0.0 < topp < 1.0:
+            r["idx"], r["w"], _ = oracle.topp_prune(r["idx"], r["w"], topp, wl.rsf)
         outs = []
         for t in tokens:
             w1 = wl.with_(T=1)
             xt = x[t:t + 1]
             idx = r["idx"][t:t + 1]
             p = oracle.permute(idx, wl.n_experts)
-            ex = self.experts(idx.ravel(), wl.wbits)
+            ex = self.experts(idx.ravel()[idx.ravel() >= 0], wl.wbits)
             _, ys = oracle.expert_ffn(w1, ex, p, xt)
             _, ysh = oracle.shared_ffn(w1, self.shared(wl.wbits), xt)
             outs.append(oracle.combine(w1, ys, ysh, r["w"][t:t + 1], p["inv"])[0])

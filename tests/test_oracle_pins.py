@@ -452,3 +452,76 @@ def test_combine_and_layer():
     # x = 0: every expert output is 0, so the layer output is 0
     _, _, out0 = oracle.moe_forward(wl, np.zeros_like(x), Wr, bias, ex, shared)
     assert not out0.any()
+
+
+# --------------------------------------------------------------------------- adaptive top-p
+def test_topp_fixture():
+    """Hand-derived cases: README "JustVugg/colibri", "快速开始" (--topp)."""
+    for case, rsf, p, T, k, idx_in, w_in, idx_out, w_out in read_golden("topp_prune.txt"):
+        T, k = int(T), int(k)
+        idx = np.array(ints(idx_in), np.int32).reshape(T, k)
+        wt = np.array(floats(w_in), np.float32).reshape(T, k)
+        i2, w2, kept = oracle.topp_prune(idx, wt, float(p), float(rsf))
+        assert i2.ravel().tolist() == ints(idx_out), case
+        assert w2.ravel().tolist() == floats(w_out), case
+        assert kept == sum(v >= 0 for v in ints(idx_out)), case
+
+
+@pytest.mark.parametrize("p", [0.3, 0.7, 0.9])
+def test_topp_minimal_prefix_brute_force(p):
+    """On real router outputs: the kept set reaches p * rsf, and no smaller set of
+    slots does (every subset of one fewer slots is checked), and among sets of its
+    size it holds the largest weights."""
+    wl, ex, shared, x, Wr, bias = _tiny_layer(T=40)
+    r = oracle.router(wl, x, Wr, bias)
+    i2, w2, kept = oracle.topp_prune(r["idx"], r["w"], p, wl.rsf)
+    thr = float(np.float32(p)) * float(np.float32(wl.rsf))
+    total = 0
+    for t in range(wl.T):
+        keep = [j for j in range(wl.top_k) if i2[t, j] >= 0]
+        drop = [j for j in range(wl.top_k) if i2[t, j] < 0]
+        total += len(keep)
+        assert keep, "at least one slot kept"
+        assert all(i2[t, j] == r["idx"][t, j] and w2[t, j] == r["w"][t, j] for j in keep)
+        assert all(w2[t, j] == 0.0 for j in drop)
+        wts = [float(r["w"][t, j]) for j in range(wl.top_k)]
+        if drop:
+            assert sum(wts[j] for j in keep) >= thr * (1 - 1e-12)
+        for sub in itertools.combinations(range(wl.top_k), len(keep) - 1):
+            assert sum(wts[j] for j in sub) < thr * (1 + 1e-12)
+        assert min(wts[j] for j in keep) >= max([wts[j] for j in drop], default=0.0)
+    assert total == kept
+
+
+def test_topp_bounds_and_layer():
+    """p outside (0,1) changes nothing; top-p feeds a permutation without the dropped
+    slots, and the layer's routed part sums only the kept experts."""
+    wl, ex, shared, x, Wr, bias = _tiny_layer(T=9)
+    r = oracle.router(wl, x, Wr, bias)
+    for p in (0.0, 1.0, 1.5, -0.1):
+        i2, w2, kept = oracle.topp_prune(r["idx"], r["w"], p, wl.rsf)
+        assert np.array_equal(i2, r["idx"]) and np.array_equal(w2, r["w"]) and kept == wl.T * wl.top_k
+    i2, w2, kept = oracle.topp_prune(r["idx"], r["w"], 0.5, wl.rsf)
+    assert kept < wl.T * wl.top_k
+    perm = oracle.permute(i2, wl.n_experts)
+    assert int(perm["counts"].sum()) == kept == int(perm["offsets"][-1])
+    flat = i2.ravel()
+    assert all(perm["inv"][a] == -1 for a in range(flat.size) if flat[a] < 0)
+    # the kept slots keep their stable (expert, slot) order
+    order = sorted((int(flat[a]), a) for a in range(flat.size) if flat[a] >= 0)
+    assert perm["sorted"][:kept].tolist() == [a for _, a in order]
+    assert np.array_equal(oracle.usage(i2, wl.n_experts),
+                          perm["counts"].astype(np.uint64))
+    # the layer with top-p = the kept experts' weighted outputs plus the shared expert
+    idx_l, wt_l, out = oracle.moe_forward(wl, x, Wr, bias, ex, shared, topp=0.5)
+    assert np.array_equal(idx_l, i2) and np.array_equal(wt_l, w2)
+    for t in range(wl.T):
+        acc = _dense_ffn(wl, shared, x[t])[1].astype(np.float64)
+        for j in range(wl.top_k):
+            if idx_l[t, j] >= 0:
+                acc += float(wt_l[t, j]) * _dense_ffn(wl, ex[idx_l[t, j]], x[t])[1].astype(np.float64)
+        assert np.allclose(out[t], acc, rtol=1e-6, atol=1e-7 * np.abs(acc).max())
+    # top-p off through the options entry: bit-identical to the plain layer
+    _, _, out_off = oracle.moe_forward(wl, x, Wr, bias, ex, shared, topp=0.0)
+    _, _, out_plain = oracle.moe_forward(wl, x, Wr, bias, ex, shared)
+    assert np.array_equal(out_off, out_plain)
