@@ -83,6 +83,8 @@ def _load():
                                          ctypes.c_double, vp, vp, vp], None),
                 "qo_topp_prune": ([ctypes.c_int, ctypes.c_int, ctypes.c_double, f32, vp, vp],
                                   i64),
+                "qo_fp8_e4m3_to_f32": ([ctypes.c_uint8], f32),
+                "qo_requant_fp8": ([vp, i64, i64, i64, vp, ctypes.c_int, vp, vp], None),
             }
             for name, (args, res) in sig.items():
                 fn = getattr(lib, name)
@@ -309,6 +311,25 @@ def topp_prune(idx: np.ndarray, wt: np.ndarray, p: float, rsf: float):
     # (double)p * (double)rsf of those
     kept = _load().qo_topp_prune(T, k, float(np.float32(p)), float(np.float32(rsf)), _p(idx), _p(wt))
     return idx, wt, int(kept)
+
+
+def fp8_e4m3_to_f32(codes) -> np.ndarray:
+    """FP8 e4m3 byte codes -> f32 (NaN for S.1111.111)."""
+    codes = np.asarray(codes, np.uint8).ravel()
+    f = _load().qo_fp8_e4m3_to_f32
+    return np.array([f(int(b)) for b in codes], np.float32)
+
+
+def requant_fp8(w8: np.ndarray, bscale: np.ndarray, bits: int):
+    """FP8 [rows][K] with 128x128 block scales -> packed per-row codes and scales."""
+    w8 = _c(w8, np.uint8)
+    rows, K = w8.shape
+    bscale = _c(bscale, np.float32)
+    assert bscale.shape == ((rows + 127) // 128, (K + 127) // 128)
+    q = np.zeros((rows, K * bits // 8), np.uint8)
+    s = np.zeros(rows, np.float32)
+    _load().qo_requant_fp8(_p(w8), rows, K, K, _p(bscale), bits, _p(q), _p(s))
+    return q, s
 
 
 def usage(idx: np.ndarray, E: int) -> np.ndarray:

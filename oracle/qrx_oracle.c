@@ -160,6 +160,48 @@ void qo_quantize_rows(const float *w, int64_t rows, int64_t K, int bits,
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* FP8 (128x128 block scales) -> per-row packed requantisation              */
+/* ------------------------------------------------------------------------ */
+/* FP8 e4m3 (the "fn" variant: 1 sign bit, 4 exponent bits with bias 7, 3
+ * mantissa bits; exponent 0 is subnormal; no infinities; S.1111.111 is NaN),
+ * decoded from that definition: (-1)^s * 2^(e-7) * (1 + m/8), or
+ * (-1)^s * 2^-6 * (m/8) when e = 0. */
+float qo_fp8_e4m3_to_f32(uint8_t b)
+{
+    const int sgn = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double v = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (float)(sgn ? -v : v);
+}
+
+/* README "JustVugg/colibri", section "已实现的功能": the offline FP8->int4
+ * converter dequantises FP8 weights with 128x128 block scales and requantises
+ * them into the engine's container.  Per element: w[r][c] = f32(fp8[r][c]) *
+ * bscale[r/128][c/128] (one f32 multiply; [reading] a NaN code counts as 0);
+ * then each row as qo_quantize_rows (s = absmax / qmax, codes
+ * clamp(round-half-away(w / s))).  w8 [rows][K] with row stride ld8 bytes;
+ * bscale [ceil(rows/128)][ceil(K/128)] row-major. */
+void qo_requant_fp8(const uint8_t *w8, int64_t rows, int64_t K, int64_t ld8, const float *bscale,
+                    int bits, uint8_t *q, float *s)
+{
+    const int64_t nbk = (K + 127) / 128, rb = qo_row_bytes(bits, K);
+    #pragma omp parallel
+    {
+        float *row = (float *)malloc(sizeof(float) * (size_t)K);
+        #pragma omp for schedule(static)
+        for (int64_t r = 0; r < rows; ++r) {
+            for (int64_t c = 0; c < K; ++c) {
+                float f = qo_fp8_e4m3_to_f32(w8[r * ld8 + c]);
+                if (isnan(f)) f = 0.0f;
+                row[c] = f * bscale[(r / 128) * nbk + c / 128];
+            }
+            qo_quantize_rows(row, 1, K, bits, q + r * rb, s + r);
+        }
+        free(row);
+    }
+}
+
 /* Decode packed rows to their integer codes (test helper). */
 void qo_unpack_rows(const uint8_t *q, int64_t rows, int64_t K, int bits, int8_t *codes)
 {

@@ -525,3 +525,67 @@ def test_topp_bounds_and_layer():
     _, _, out_off = oracle.moe_forward(wl, x, Wr, bias, ex, shared, topp=0.0)
     _, _, out_plain = oracle.moe_forward(wl, x, Wr, bias, ex, shared)
     assert np.array_equal(out_off, out_plain)
+
+
+# --------------------------------------------------------------------------- FP8 requantisation
+def test_fp8_decode_matches_torch():
+    """Every e4m3 code decodes to torch's float8_e4m3fn value (NaN codes to NaN)."""
+    import torch
+    f = oracle.fp8_e4m3_to_f32(np.arange(256))
+    t = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    nan = np.isnan(t)
+    assert np.array_equal(np.isnan(f), nan) and nan.sum() == 2
+    assert np.array_equal(f[~nan].view(np.uint32), t[~nan].view(np.uint32))
+
+
+def _fixture_fp8():
+    w8 = np.zeros((2, 256), np.uint8)
+    w8[0, :128], w8[0, 128:] = 0x38, 0x40
+    w8[1, 0], w8[1, 5], w8[1, 200] = 0xC8, 0x7F, 0x30
+    return w8, np.array([[0.5, 0.25]], np.float32)
+
+
+def test_requant_fixture():
+    w8, bs = _fixture_fp8()
+    for bits, row, amax, c0, c5, c200, rest in read_golden("requant_fp8.txt"):
+        bits, row = int(bits), int(row)
+        q, s = oracle.requant_fp8(w8, bs, bits)
+        codes = np_codes(q, 256, bits)[row]
+        qmax = {8: 127, 4: 7, 2: 1}[bits]
+        assert s[row] == np.float32(float(amax)) / np.float32(qmax)
+        assert (codes[0], codes[5], codes[200]) == (int(c0), int(c5), int(c200))
+        others = np.delete(codes, [0, 5, 200])
+        assert (others == int(rest)).all()
+
+
+@pytest.mark.parametrize("bits", [8, 4, 2])
+def test_requant_against_torch_dequant(bits):
+    """Random codes (every byte value, NaN and subnormals included) and block scales on
+    a ragged 300 x 224 matrix: the result equals quantising the dequantised matrix,
+    the dequantisation done here with torch's float8 decode and one f32 multiply."""
+    import torch
+    rng = np.random.default_rng(5)
+    rows, K = 300, 224
+    w8 = rng.integers(0, 256, size=(rows, K), dtype=np.uint8)
+    bs = (rng.random((3, 2)) * 0.01 + 1e-4).astype(np.float32)
+    q, s = oracle.requant_fp8(w8, bs, bits)
+    f = torch.from_numpy(w8).view(torch.float8_e4m3fn).float().numpy()
+    f = np.where(np.isnan(f), np.float32(0), f)
+    scale = np.repeat(np.repeat(bs, 128, axis=0), 128, axis=1)[:rows, :K]
+    deq = (f * scale).astype(np.float32)
+    q2, s2 = oracle.quantize_rows(deq, bits)
+    assert np.array_equal(q, q2) and np.array_equal(s.view(np.uint32), s2.view(np.uint32))
+
+
+def test_requant_power_of_two_scales():
+    """Scaling every block scale by 2^m scales each row scale by 2^m exactly and leaves
+    the codes unchanged (multiplication by a power of two is exact)."""
+    rng = np.random.default_rng(6)
+    w8 = rng.integers(0, 126, size=(130, 256), dtype=np.uint8)   # finite codes only
+    bs = (rng.random((2, 2)) + 0.5).astype(np.float32)
+    for bits in (8, 4, 2):
+        q, s = oracle.requant_fp8(w8, bs, bits)
+        for m in (-3, 5):
+            q2, s2 = oracle.requant_fp8(w8, bs * np.float32(2.0 ** m), bits)
+            assert np.array_equal(q, q2)
+            assert np.array_equal(s2, s * np.float32(2.0 ** m))
