@@ -49,6 +49,12 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling case: fewer routed experts (same per-launch work at T=1)")
+    ap.add_argument("--topp", type=float, default=0.0,
+                    help="adaptive expert top-p (0: off) applied inside the layer")
+    ap.add_argument("--kernel", choices=["requant_fp8"], default=None,
+                    help="measure one auxiliary kernel instead of the layer")
+    ap.add_argument("--union-stats", action="store_true",
+                    help="union sizes of correlated verify batches (router + permutation)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="profiling case: another token count per step")
     ap.add_argument("--no-settle", action="store_true",
@@ -169,11 +175,11 @@ def run_reference(args, wl):
     experts = {e: oracle.quantize_expert(*expert_f32(wl, e), wl.wbits) for e in sorted(needed)}
     shared = oracle.quantize_expert(*expert_f32(wl, wl.n_experts), wl.wbits)
     for i in range(args.warmup if args.warmup < 2 else 1):
-        oracle.moe_forward(wl, xs[i % npool], Wr, bias, experts, shared)
+        oracle.moe_forward(wl, xs[i % npool], Wr, bias, experts, shared, topp=args.topp)
     times = []
     for i in range(args.steps):
         t0 = time.perf_counter()
-        oracle.moe_forward(wl, xs[i % npool], Wr, bias, experts, shared)
+        oracle.moe_forward(wl, xs[i % npool], Wr, bias, experts, shared, topp=args.topp)
         times.append(time.perf_counter() - t0)
     ms = 1e3 * sum(times) / len(times)
     value = wl.T / (ms / 1e3)
@@ -184,7 +190,7 @@ def run_reference(args, wl):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
-        "config": workload_config(wl),
+        "config": workload_config(wl, args.topp),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -192,9 +198,98 @@ def run_reference(args, wl):
     }))
 
 
-def workload_config(wl):
+def run_requant(args):
+    """FP8 (128x128 block scales) -> packed int4 rows over the gate/up and down
+    matrices of 16 GLM-shaped experts (HBM-bound): bytes = FP8 read + codes and
+    scales written, per launch; CUDA events, L2 flushed between launches."""
+    import numpy as np
+    import torch
+    from quantized_routed_expert_tc_b200 import build as qbuild, qrx
+    qbuild.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    nexp, H, I, bits = 16, 6144, 2048, 4
+    mats = [(nexp * 2 * I, H), (nexp * H, I)]          # stacked w13 rows, stacked w2 rows
+    gen = torch.Generator(device=dev).manual_seed(1234)
+    bufs = []
+    for rows, K in mats:
+        w8 = torch.randint(0, 126, (rows, K), dtype=torch.uint8, device=dev, generator=gen)
+        bs = torch.rand(((rows + 127) // 128, (K + 127) // 128), device=dev, generator=gen) * 1e-2 + 1e-4
+        q = torch.empty((rows, K * bits // 8), dtype=torch.uint8, device=dev)
+        sc = torch.empty(rows, dtype=torch.float32, device=dev)
+        bufs.append((w8, bs, q, sc))
+    nbytes = sum(w8.numel() + q.numel() + 4 * sc.numel() + 4 * bs.numel() for w8, bs, q, sc in bufs)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    def once():
+        for w8, bs, q, sc in bufs:
+            qrx.qrx_requant_fp8(w8, bs, bits, q, sc, stream)
+    for _ in range(args.warmup):
+        once()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        once()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    rc = qrx.qrx_last_error()
+    if rc != qrx.QRX_OK:
+        raise RuntimeError(qrx.qrx_strerror(rc))
+    ms = float(np.median(times))
+    peak, kind = peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    print(json.dumps({"metric": "FP8 128x128-block -> per-row int4 requantisation GB/s",
+                      "value": gbs, "unit": "GB/s", "ms_per_call": ms, "steps": args.steps,
+                      "config": {"experts": nexp, "matrices": [list(m) for m in mats], "bits": bits},
+                      "roofline": {"kernel": "k_requant_fp8", "bound": "hbm", "achieved": gbs,
+                                   "peak": peak, "peak_kind": kind, "unit": "GB/s",
+                                   "frac": gbs / peak, "bytes_per_call": nbytes},
+                      "gpu_launches": 2 * args.steps}))
+
+
+def run_union_stats(args):
+    """Expert-union size of verify batches whose tokens share router input structure
+    (token i = sqrt(rho) z + sqrt(1 - rho) z_i), through qrx_route + qrx_permute at
+    the GLM shape: loads per forward = union + 1 (shared expert)."""
+    import numpy as np
+    import torch
+    from quantized_routed_expert_tc_b200 import build as qbuild, qrx, workloads as W
+    from quantized_routed_expert_tc_b200.layer import activations_correlated, router_weights
+    qbuild.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    base = W.GLM_DECODE_T1
+    Wr_np, bias_np = router_weights(base)
+    Wr, bias = torch.from_numpy(Wr_np).to(dev), torch.from_numpy(bias_np).to(dev)
+    rows = []
+    for rho in (0.0, 0.5, 0.8, 0.9, 0.95, 1.0):
+        for T in (1, 2, 3, 4, 8, 16):
+            wl = base.with_(T=T)
+            c = qrx.cfg_of(wl)
+            ws = qrx.workspace(c, T, dev)
+            idx = torch.empty((T, wl.top_k), dtype=torch.int32, device=dev)
+            w = torch.empty((T, wl.top_k), dtype=torch.float32, device=dev)
+            perm = qrx.Perm.empty(T, wl.top_k, wl.n_experts)
+            nus = []
+            for b in range(32):
+                x = torch.from_numpy(activations_correlated(wl, T, rho, batch=b)).to(dev)
+                qrx.qrx_route(c, x, Wr, bias, idx, w, ws)
+                qrx.qrx_permute(c, idx, perm)
+                nus.append(int(perm.n_union.item()))
+            nu = float(np.mean(nus))
+            rows.append({"rho": rho, "T": T, "n_union_mean": nu, "loads_per_forward": nu + 1,
+                         "loads_per_token_if_all_accepted": (nu + 1) / T})
+    print(json.dumps({"metric": "verify-batch expert union (GLM shape, 32 batches each)",
+                      "rows": rows}))
+
+
+def workload_config(wl, topp: float = 0.0):
     from quantized_routed_expert_tc_b200 import workloads as W
-    return {"workload": wl.name, "tokens_per_step": wl.T, "hidden": wl.hidden,
+    extra = {"expert_top_p": topp} if topp else {}
+    return {**extra, "workload": wl.name, "tokens_per_step": wl.T, "hidden": wl.hidden,
             "routed_experts": wl.n_experts, "shared_experts": 1, "inter": wl.inter,
             "top_k": wl.top_k, "n_group": wl.n_group, "topk_group": wl.topk_group,
             "weights": f"int{wl.wbits} per-row f32 scale",
@@ -204,7 +299,7 @@ def workload_config(wl):
 
 
 # ----------------------------------------------------------------------------- CPU baseline
-def cpu_baseline(wl, seconds: float):
+def cpu_baseline(wl, seconds: float, topp: float = 0.0):
     import numpy as np
     import oracle
     from quantized_routed_expert_tc_b200.layer import activations, expert_f32, router_weights
@@ -219,7 +314,7 @@ def cpu_baseline(wl, seconds: float):
     n, t_total = 0, 0.0
     while t_total < seconds or n < 2:
         t0 = time.perf_counter()
-        oracle.moe_forward(wl, xs[n % 2], Wr, bias, experts, shared)
+        oracle.moe_forward(wl, xs[n % 2], Wr, bias, experts, shared, topp=topp)
         t_total += time.perf_counter() - t0
         n += 1
         if n >= 200:
@@ -259,8 +354,8 @@ def run_qrx(args, wl, rank, world, local_rank):
     unions = []
     for x in xs:
         qrx.qrx_moe_forward(cfg, x, glay.Wr, glay.bias, glay.routed[wl.wbits],
-                            glay.shared[wl.wbits], idx, w, out, ws)
-        unions.append(int(torch.unique(idx).numel()))
+                            glay.shared[wl.wbits], idx, w, out, ws, topp=args.topp)
+        unions.append(int(torch.unique(idx[idx >= 0]).numel()))
     torch.cuda.synchronize(dev)
     rc = qrx.qrx_last_error()
     if rc != qrx.QRX_OK:
@@ -270,14 +365,14 @@ def run_qrx(args, wl, rank, world, local_rank):
         flush.zero_()
         ev0.record(stream)
         qrx.qrx_moe_forward(cfg, xs[i % npool], glay.Wr, glay.bias, glay.routed[wl.wbits],
-                            glay.shared[wl.wbits], idx, w, out, ws, stream)
+                            glay.shared[wl.wbits], idx, w, out, ws, stream, topp=args.topp)
         ev1.record(stream)
 
     def step_profiled(i, evs):
         flush.zero_()
         qrx.qrx_moe_forward_profiled(cfg, xs[i % npool], glay.Wr, glay.bias,
                                      glay.routed[wl.wbits], glay.shared[wl.wbits], idx, w, out,
-                                     ws, evs, stream)
+                                     ws, evs, stream, topp=args.topp)
 
     sampler = ClockSampler(local_rank)
     sampler.start()
@@ -371,11 +466,15 @@ def run_qrx(args, wl, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, args.cpu_seconds)
+        cpu = cpu_baseline(wl, args.cpu_seconds, args.topp)
 
     if rank == 0:
         stages = ["act_records", "router", "permute", "gateup", "down", "combine"]
-        launches_per_step = 7 if wl.T <= 64 else 7
+        # library kernels per layer call: GEMV engine: activation records, router
+        # (dot + selection), permutation, gate/up, h records, down, combine = 8;
+        # tensor-core engine: router (2), permutation, token gather, gate/up, down,
+        # combine = 7 (top-p and usage add none)
+        launches_per_step = 7 if tc else 8
         line = {
             "metric": METRIC, "value": T * world / (ms_step / 1e3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -383,7 +482,7 @@ def run_qrx(args, wl, rank, world, local_rank):
             "dtype": "bf16" if tc else "int32",
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights quantised by the "
                     "library; no trained weights)",
-            "config": workload_config(wl),
+            "config": workload_config(wl, args.topp),
             "weight_gbs": weight_gbs,
             "weight_gbs_frac_of_measured_hbm": weight_gbs / peak,
             "weight_gbs_frac_of_8tbs": weight_gbs / SPEC_HBM_GBS,
@@ -419,9 +518,19 @@ def main():
         wl = wl.with_(name=f"{wl.name}_e{args.experts}", n_experts=args.experts)
     if args.tokens:
         wl = wl.with_(name=f"{wl.name}_t{args.tokens}", T=args.tokens)
+    if args.topp:
+        wl = wl.with_(name=f"{wl.name}_topp{args.topp:g}")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.kernel == "requant_fp8":
+        if rank == 0:
+            run_requant(args)
+        return
+    if args.union_stats:
+        if rank == 0:
+            run_union_stats(args)
+        return
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, wl)

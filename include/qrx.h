@@ -154,6 +154,19 @@ const char *qrx_strerror(int code);
 int qrx_quantize_weights(const float *w, int64_t rows, int64_t K, int32_t wbits,
                          uint8_t *q, int64_t ldq, float *scale, int64_t lds, void *stream);
 
+/* FP8 checkpoint rows -> the same packed per-row container (README
+ * "JustVugg/colibri", section "已实现的功能": the FP8->int4 converter
+ * dequantises with 128x128 block scales and requantises for the engine).
+ * Each value is f32(e4m3 code) * bscale[r/128][c/128] (one f32 multiply; a NaN
+ * code counts as 0), then quantised as qrx_quantize_weights does.
+ *   w8      [rows][K] FP8 e4m3 codes (device), row r at w8 + r*ld8 bytes
+ *   bscale  [ceil(rows/128)][ceil(K/128)] f32 block scales (device, row-major)
+ *   q, ldq, scale, lds: outputs as in qrx_quantize_weights
+ * K must be a multiple of 32, ld8 a multiple of 4, w8 4-byte aligned.
+ * Bit-exact with the CPU reference. */
+int qrx_requant_fp8(const uint8_t *w8, int64_t rows, int64_t K, int64_t ld8, const float *bscale,
+                    int32_t wbits, uint8_t *q, int64_t ldq, float *scale, int64_t lds, void *stream);
+
 /* Q8_0-style activations (README "已实现的功能": integer dot with Q8_0-style
  * int8 activations; blocks of 32 with an f32 absmax scale):
  * d = amax/127, q = clamp(round-half-away(x * (127/amax)), -127, 127), a zero
@@ -185,10 +198,29 @@ int qrx_route(const qrx_cfg *cfg, const void *x, int32_t T, const float *W_route
 
 /* Batch-union permutation (README "已实现的功能": batch-union MoE; blog:
  * same expert read once per batch): a stable counting sort of the T*k
- * assignments by expert.  Deterministic.  Sets the device error flag if an
- * index is outside [0, E). */
+ * assignments by expert.  Deterministic.  An index of -1 marks a slot dropped
+ * by adaptive top-p: it is not counted and its inv entry is -1.  Sets the
+ * device error flag if an index is outside [0, E) and not -1. */
 int qrx_permute(const qrx_cfg *cfg, const int32_t *topk_idx, int32_t T,
                 const qrx_perm *perm, void *stream);
+
+/* Adaptive expert top-p (README "JustVugg/colibri", section "快速开始": the
+ * --topp knob, default 0.7; "社区基准（实测）": its measured effect), applied
+ * in place to a router output topk_idx / topk_w [T][k] (device):
+ * per token, slots are taken by weight, largest first (equal weights: the
+ * lower slot first), their weights summed in double in that order, until the
+ * sum reaches (double)p * (double)rsf; the other slots become idx = -1,
+ * w = 0.  Kept weights are not renormalised.  p outside (0, 1) leaves the
+ * arrays unchanged.  QRX_EINVAL for NULL arrays or a NaN p. */
+int qrx_topp_prune(const qrx_cfg *cfg, int32_t *topk_idx, float *topk_w, int32_t T, float p,
+                   void *stream);
+
+/* Expert-usage histogram (README "JustVugg/colibri", "快速开始": the engine
+ * records which experts a run routes to; "如何测试，按顺序": the STATS file):
+ * usage[e] += perm->counts[e] for every expert, on device.  usage: caller-owned
+ * device array of E uint64 counters, 8-byte aligned, set to zero by the caller
+ * before the first call; calls on one stream accumulate in order. */
+int qrx_usage_accumulate(const qrx_cfg *cfg, const qrx_perm *perm, uint64_t *usage, void *stream);
 
 /* Routed experts' SwiGLU FFN over the batch union: for each expert of the
  * union, its gate/up rows are read once for all of its positions:
@@ -266,20 +298,37 @@ int qrx_moe_forward(const qrx_cfg *cfg, const void *x, int32_t T, const float *W
                     int32_t *topk_idx, float *topk_w, float *out, void *ws,
                     size_t ws_bytes, void *stream);
 
+/* Options of qrx_moe_forward_opts. */
+typedef struct {
+    float expert_top_p;   /* adaptive expert top-p (see qrx_topp_prune), applied
+                             inside the router's selection kernel; 0: off */
+    uint64_t *usage;      /* [E] device usage counters (see qrx_usage_accumulate),
+                             updated inside the permutation kernel; NULL: off */
+} qrx_moe_opts;
+
+/* qrx_moe_forward with options (opts may be NULL: same as qrx_moe_forward).
+ * With top-p on, dropped slots come back as topk_idx = -1, topk_w = 0 and
+ * take no part in the union, the expert FFN or the combine.  Neither option
+ * adds a kernel launch.  QRX_EINVAL for a NaN top-p or a misaligned usage. */
+int qrx_moe_forward_opts(const qrx_cfg *cfg, const void *x, int32_t T, const float *W_router,
+                         const float *bias, const qrx_experts *routed, const qrx_experts *shared,
+                         int32_t *topk_idx, float *topk_w, float *out, void *ws, size_t ws_bytes,
+                         const qrx_moe_opts *opts, void *stream);
+
 /* qrx_moe_forward with stage timing: events[0..6] are cudaEvent_t handles
  * (passed as void*) recorded on `stream` before the activation-record
  * kernel, after it, after the router, after the permutation, after the
  * gate/up kernel, after the down kernel and after the combine.  n_events must
  * be 7.  The events separate the kernels, so the launch overlap that
  * qrx_moe_forward gets from programmatic dependent launch is lost here: the
- * stage times add up to more than a plain call takes.  Everything else is as
- * qrx_moe_forward. */
+ * stage times add up to more than a plain call takes.  opts as in
+ * qrx_moe_forward_opts (may be NULL).  Everything else is as qrx_moe_forward. */
 int qrx_moe_forward_profiled(const qrx_cfg *cfg, const void *x, int32_t T,
                              const float *W_router, const float *bias,
                              const qrx_experts *routed, const qrx_experts *shared,
                              int32_t *topk_idx, float *topk_w, float *out, void *ws,
                              size_t ws_bytes, void *const *events, int32_t n_events,
-                             void *stream);
+                             const qrx_moe_opts *opts, void *stream);
 
 /* The same layer with HOST input and output: copies x_host (pinned or
  * pageable, T*H elements of the activation type) to the device, runs

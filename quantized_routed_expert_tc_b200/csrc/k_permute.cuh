@@ -6,6 +6,10 @@
 // it; blog "GLM-5.2 on slow computers", "让它变得可以忍受的那些装置": the same
 // expert in a batch is read only once.
 //
+// A slot with expert -1 (dropped by adaptive top-p) takes no position: it is
+// not counted and its inv entry is -1.  When a usage array is given, the
+// per-expert counts of this call are added to it (expert-usage histogram).
+//
 // One CTA of 32 warps.  Warp w owns a contiguous segment of assignments.
 // Pass 1 counts experts per segment (ballot-free: __match_any_sync leaders add
 // their group's size), a column scan over warps turns the counts into each
@@ -49,7 +53,7 @@ __device__ __forceinline__ int block_exclusive_scan_1024(int v, int *tmp, int &t
 }
 
 __global__ void __launch_bounds__(1024, 1) k_permute(const int32_t *__restrict__ idx, int A, int E,
-                                                     qrx_perm p)
+                                                     qrx_perm p, uint64_t *__restrict__ usage)
 {
     extern __shared__ __align__(16) int psm[];
     int *whist = psm;                          // [PERM_WARPS][E]
@@ -67,7 +71,9 @@ __global__ void __launch_bounds__(1024, 1) k_permute(const int32_t *__restrict__
         int e = -1;
         if (a < a1) {
             e = idx[a];
-            if (e < 0 || e >= E) { raise_status(DERR_BADIDX); e = -1; }
+            // -1: a slot dropped by adaptive top-p; anything else outside [0, E) is an error
+            if (e != -1 && (e < 0 || e >= E)) raise_status(DERR_BADIDX);
+            if (e < 0 || e >= E) e = -1;
         }
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         if (e >= 0 && lane == __ffs(peers) - 1) whist[wid * E + e] += __popc(peers);
@@ -91,6 +97,7 @@ __global__ void __launch_bounds__(1024, 1) k_permute(const int32_t *__restrict__
     if (tid < E) {
         p.counts[tid] = cnt;
         p.offsets[tid] = off;
+        if (usage && cnt) atomicAdd(reinterpret_cast<unsigned long long *>(usage + tid), (unsigned long long)cnt);
         if (present) p.union_ids[upos] = tid;
         for (int w = 0; w < PERM_WARPS; ++w) whist[w * E + tid] += off;
     }
@@ -122,7 +129,7 @@ __global__ void __launch_bounds__(1024, 1) k_permute(const int32_t *__restrict__
 }
 
 cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const qrx_perm &p,
-                           cudaStream_t st)
+                           cudaStream_t st, uint64_t *usage)
 {
     const size_t smem = ((size_t)PERM_WARPS * E + 40) * sizeof(int);
     if (smem > 48 * 1024) {
@@ -130,7 +137,24 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const qrx_pe
                                                (int)smem);
         if (err != cudaSuccess) return err;
     }
-    return launch_k(k_permute, dim3(1), dim3(1024), smem, st, idx, T * k, E, p);
+    return launch_k(k_permute, dim3(1), dim3(1024), smem, st, idx, T * k, E, p, usage);
+}
+
+// Expert-usage histogram (README "JustVugg/colibri", "快速开始": the engine
+// records which experts a run routes to): usage[e] += counts[e].
+__global__ void __launch_bounds__(256) k_usage_add(const int32_t *__restrict__ counts, int E,
+                                                   uint64_t *__restrict__ usage)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e < E && counts[e] > 0)
+        atomicAdd(reinterpret_cast<unsigned long long *>(usage + e), (unsigned long long)counts[e]);
+}
+
+cudaError_t launch_usage_add(const int32_t *counts, int E, uint64_t *usage, cudaStream_t st)
+{
+    return launch_k(k_usage_add, dim3((unsigned)((E + 255) / 256)), dim3(256), 0, st, counts, E, usage);
 }
 
 }  // namespace qrx

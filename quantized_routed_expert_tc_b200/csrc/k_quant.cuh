@@ -57,6 +57,73 @@ __global__ void __launch_bounds__(256) k_quantize_weights(const float *__restric
     }
 }
 
+// FP8 (e4m3, 128x128 block scales) -> per-row packed codes (README
+// "JustVugg/colibri", section "已实现的功能": the FP8->int4 converter
+// dequantises with 128x128 block scales and requantises into the per-row
+// container).  One warp per row; each value is f32(fp8) * block scale (a NaN
+// code counts as 0), recomputed in pass 2 instead of kept: the row's FP8
+// bytes are re-read from L2.  Pass 1: absmax; pass 2: codes as
+// k_quantize_weights.  Lanes read 4 bytes at a time: K % 32 == 0, rows
+// 4-byte aligned.
+__device__ __forceinline__ float fp8_value(uint32_t byte, float scale)
+{
+    __nv_fp8_e4m3 f8;
+    f8.__x = (__nv_fp8_storage_t)byte;
+    float f = static_cast<float>(f8);
+    if (f != f) f = 0.f;
+    return __fmul_rn(f, scale);
+}
+
+template <int WB>
+__global__ void __launch_bounds__(256) k_requant_fp8(const uint8_t *__restrict__ w8, int64_t rows, int64_t K,
+                                                     int64_t ld8, const float *__restrict__ bscale,
+                                                     uint8_t *__restrict__ q, int64_t ldq,
+                                                     float *__restrict__ scale, int64_t lds)
+{
+    constexpr int QMAX = WB == 8 ? 127 : (WB == 4 ? 7 : 1);
+    constexpr int QMIN = WB == 8 ? -128 : (WB == 4 ? -8 : -2);
+    constexpr int EPW = 32 / WB;     // codes per 32-bit word
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    pdl_wait();
+    pdl_trigger();
+    if (r >= rows) return;
+    const uint8_t *wr = w8 + r * ld8;
+    const float *bs = bscale + (r / 128) * ((K + 127) / 128);
+    float amax = 0.f;
+    for (int64_t i = lane * 4; i < K; i += 128) {
+        const uint32_t v = *reinterpret_cast<const uint32_t *>(wr + i);
+        const float sc = bs[i / 128];       // 4 consecutive columns share a block
+#pragma unroll
+        for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fabsf(fp8_value((v >> (8 * j)) & 0xFFu, sc)));
+    }
+    amax = warp_max(amax);
+    const float s = __fdiv_rn(amax, (float)QMAX);
+    if (lane == 0) scale[r * lds] = s;
+    uint32_t *qr = reinterpret_cast<uint32_t *>(q + r * ldq);
+    const int64_t nwords = K / EPW;
+    for (int64_t wd = lane; wd < nwords; wd += 32) {
+        const int64_t c0 = wd * EPW;
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < EPW; i += 4) {
+            const uint32_t v = *reinterpret_cast<const uint32_t *>(wr + c0 + i);
+            const float sc = bs[(c0 + i) / 128];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float x = fp8_value((v >> (8 * j)) & 0xFFu, sc);
+                int c = 0;
+                if (s != 0.f) {
+                    c = (int)roundf(__fdiv_rn(x, s));
+                    c = c > QMAX ? QMAX : (c < QMIN ? QMIN : c);
+                }
+                word |= ((uint32_t)c & ((1u << WB) - 1u)) << (WB * (i + j));
+            }
+        }
+        qr[wd] = word;
+    }
+}
+
 // One warp per 32-element block.
 __global__ void __launch_bounds__(256) k_quantize_act_q8(const float *__restrict__ x, int64_t nblocks,
                                                          int8_t *__restrict__ xq,
@@ -126,6 +193,16 @@ cudaError_t launch_quantize_weights(const float *w, int64_t rows, int64_t K, int
     else if (wbits == 4) k_quantize_weights<4><<<grid, block, 0, st>>>(w, rows, K, q, ldq, scale, lds);
     else k_quantize_weights<2><<<grid, block, 0, st>>>(w, rows, K, q, ldq, scale, lds);
     return cudaGetLastError();
+}
+
+cudaError_t launch_requant_fp8(const uint8_t *w8, int64_t rows, int64_t K, int64_t ld8, const float *bscale,
+                              int wbits, uint8_t *q, int64_t ldq, float *scale, int64_t lds, cudaStream_t st)
+{
+    const int wpb = 8;
+    const dim3 grid((unsigned)((rows + wpb - 1) / wpb)), block(32 * wpb);
+    if (wbits == 8) return launch_k(k_requant_fp8<8>, grid, block, 0, st, w8, rows, K, ld8, bscale, q, ldq, scale, lds);
+    if (wbits == 4) return launch_k(k_requant_fp8<4>, grid, block, 0, st, w8, rows, K, ld8, bscale, q, ldq, scale, lds);
+    return launch_k(k_requant_fp8<2>, grid, block, 0, st, w8, rows, K, ld8, bscale, q, ldq, scale, lds);
 }
 
 cudaError_t launch_quantize_act_q8(const float *x, int64_t nblocks, int8_t *xq, float *xd,

@@ -234,11 +234,38 @@ __global__ void __launch_bounds__(256) k_router_select(RouterArgs a)
     if (lane == 0)
         for (int j = 0; j < a.k; ++j) ssum += (double)s_s[sel[j]];
     ssum = __shfl_sync(0xffffffffu, ssum, 0);
+    const int e = lane < a.k ? sel[lane] : 0;
+    const float wv = lane < a.k ? (float)((double)s_s[e] / ssum * (double)a.rsf) : 0.f;
+    // adaptive top-p (when on): dropped slots become idx = -1, w = 0
+    const bool keep = a.topp_thr > 0.0 ? warp_topp_keep(lane, a.k, wv, a.topp_thr) : true;
     if (lane < a.k) {
-        const int e = sel[lane];
-        a.idx[(int64_t)t * a.k + lane] = e;
-        a.w[(int64_t)t * a.k + lane] = (float)((double)s_s[e] / ssum * (double)a.rsf);
+        a.idx[(int64_t)t * a.k + lane] = keep ? e : -1;
+        a.w[(int64_t)t * a.k + lane] = keep ? wv : 0.f;
     }
+}
+
+// Adaptive expert top-p on a router output already in memory: warp per token.
+__global__ void __launch_bounds__(256) k_topp_prune(int32_t *__restrict__ idx, float *__restrict__ w, int T,
+                                                    int k, double thr)
+{
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    pdl_wait();
+    pdl_trigger();
+    if (t >= T) return;
+    const int64_t a = (int64_t)t * k + lane;
+    const float wv = lane < k ? w[a] : 0.f;
+    const int32_t e = lane < k ? idx[a] : -1;
+    const bool keep = warp_topp_keep(lane, k, wv, thr);
+    if (lane < k) {
+        idx[a] = keep ? e : -1;
+        w[a] = keep ? wv : 0.f;
+    }
+}
+
+cudaError_t launch_topp_prune(int32_t *idx, float *w, int T, int k, double thr, cudaStream_t st)
+{
+    return launch_k(k_topp_prune, dim3((unsigned)((T + 7) / 8)), dim3(256), 0, st, idx, w, T, k, thr);
 }
 
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t st)

@@ -266,6 +266,17 @@ int qrx_quantize_weights(const float *w, int64_t rows, int64_t K, int32_t wbits,
                                              (cudaStream_t)stream));
 }
 
+int qrx_requant_fp8(const uint8_t *w8, int64_t rows, int64_t K, int64_t ld8, const float *bscale,
+                    int32_t wbits, uint8_t *q, int64_t ldq, float *scale, int64_t lds, void *stream)
+{
+    if (!w8 || !bscale || !q || !scale || rows <= 0 || K <= 0 || K % 32 != 0) return QRX_EINVAL;
+    if (wbits != 8 && wbits != 4 && wbits != 2) return QRX_EINVAL;
+    if (ld8 < K || ld8 % 4 != 0 || ldq < K * wbits / 8 || ldq % 4 != 0 || lds < 1) return QRX_EINVAL;
+    if (!aligned(w8, 4) || !aligned(bscale, 4) || !aligned(q, 4) || !aligned(scale, 4)) return QRX_EINVAL;
+    return cuda_code(launch_requant_fp8(w8, rows, K, ld8, bscale, wbits, q, ldq, scale, lds,
+                                        (cudaStream_t)stream));
+}
+
 int qrx_quantize_act_q8(const float *x, int64_t T, int64_t H, int8_t *xq, float *xd, void *stream)
 {
     if (!x || !xq || !xd || T <= 0 || H <= 0 || H % 32 != 0) return QRX_EINVAL;
@@ -281,8 +292,10 @@ int qrx_block_dots_q8(int32_t wbits, const uint8_t *q, int64_t rows, int64_t K, 
     return cuda_code(launch_block_dots_q8(wbits, q, rows, K, xq, acc, (cudaStream_t)stream));
 }
 
-int qrx_route(const qrx_cfg *c, const void *x, int32_t T, const float *Wr, const float *bias,
-              int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream)
+// The router, with adaptive top-p applied in its select kernel when topp_thr > 0.
+static int route_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr, const float *bias,
+                      int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream,
+                      double topp_thr)
 {
     int v = check_common(c, T);
     if (v) return v;
@@ -304,7 +317,38 @@ int qrx_route(const qrx_cfg *c, const void *x, int32_t T, const float *Wr, const
     a.logits = at<float>(ws, L.logits);
     a.idx = topk_idx;
     a.w = topk_w;
+    a.topp_thr = topp_thr;
     return cuda_code(launch_router(a, (cudaStream_t)stream));
+}
+
+// p * rsf for adaptive top-p, or 0 (off) when p is outside (0, 1).
+static double topp_threshold(const qrx_cfg *c, float p)
+{
+    return (p > 0.f && p < 1.f) ? (double)p * (double)c->routed_scaling_factor : 0.0;
+}
+
+int qrx_route(const qrx_cfg *c, const void *x, int32_t T, const float *Wr, const float *bias,
+              int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream)
+{
+    return route_impl(c, x, T, Wr, bias, topk_idx, topk_w, ws, ws_bytes, stream, 0.0);
+}
+
+int qrx_topp_prune(const qrx_cfg *c, int32_t *topk_idx, float *topk_w, int32_t T, float p, void *stream)
+{
+    int v = check_common(c, T);
+    if (v) return v;
+    if (!topk_idx || !topk_w || !(p == p)) return QRX_EINVAL;
+    const double thr = topp_threshold(c, p);
+    if (thr == 0.0) return QRX_OK;
+    return cuda_code(launch_topp_prune(topk_idx, topk_w, T, c->top_k, thr, (cudaStream_t)stream));
+}
+
+int qrx_usage_accumulate(const qrx_cfg *c, const qrx_perm *perm, uint64_t *usage, void *stream)
+{
+    int v = qrx_validate(c);
+    if (v) return v;
+    if (!perm || !perm->counts || !usage || !aligned(usage, 8)) return QRX_EINVAL;
+    return cuda_code(launch_usage_add(perm->counts, c->n_experts, usage, (cudaStream_t)stream));
 }
 
 int qrx_permute(const qrx_cfg *c, const int32_t *topk_idx, int32_t T, const qrx_perm *perm,
@@ -418,7 +462,7 @@ namespace {
 int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr,
                      const float *bias, const qrx_experts *routed, const qrx_experts *shared,
                      int32_t *topk_idx, float *topk_w, float *out, void *ws, size_t ws_bytes,
-                     void *const *events, void *stream)
+                     void *const *events, void *stream, const qrx_moe_opts *opts = nullptr)
 {
     auto mark = [&](int i) -> bool {
         return !events || cudaEventRecord((cudaEvent_t)events[i], (cudaStream_t)stream) == cudaSuccess;
@@ -431,6 +475,10 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     if (shared && (v = check_experts(shared))) return v;
     if ((v = check_ws(c, T, ws, ws_bytes))) return v;
     if (!aligned(out, 16)) return QRX_EINVAL;
+    if (opts && (!(opts->expert_top_p == opts->expert_top_p) || (opts->usage && !aligned(opts->usage, 8))))
+        return QRX_EINVAL;
+    const double topp_thr = opts ? topp_threshold(c, opts->expert_top_p) : 0.0;
+    uint64_t *usage = opts ? opts->usage : nullptr;
     const Ws L = ws_layout(c, T);
     cudaStream_t st = (cudaStream_t)stream;
     const int sms = num_sms_current();
@@ -451,12 +499,12 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     // 2.. the rest chained with programmatic dependent launch (the first kernel
     // of the call never is: it must follow whatever the stream held before)
     PdlScope pdl(!tc);
-    if ((v = qrx_route(c, x, T, Wr, bias, topk_idx, topk_w, ws, ws_bytes, stream))) return v;
+    if ((v = route_impl(c, x, T, Wr, bias, topk_idx, topk_w, ws, ws_bytes, stream, topp_thr))) return v;
     g_pdl = true;
     if (!mark(2)) return QRX_ECUDA;
     qrx_perm perm{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.sorted),
                   at<int32_t>(ws, L.inv), at<int32_t>(ws, L.uids), at<int32_t>(ws, L.nu)};
-    e = launch_permute(topk_idx, T, c->top_k, c->n_experts, perm, st);
+    e = launch_permute(topk_idx, T, c->top_k, c->n_experts, perm, st, usage);
     if (e != cudaSuccess || !mark(3)) return QRX_ECUDA;
     float *h = at<float>(ws, L.h), *y = at<float>(ws, L.y);
     set_routed(a, routed, &perm);
@@ -490,17 +538,26 @@ int qrx_moe_forward(const qrx_cfg *c, const void *x, int32_t T, const float *Wr,
                             nullptr, stream);
 }
 
+int qrx_moe_forward_opts(const qrx_cfg *c, const void *x, int32_t T, const float *Wr,
+                         const float *bias, const qrx_experts *routed, const qrx_experts *shared,
+                         int32_t *topk_idx, float *topk_w, float *out, void *ws, size_t ws_bytes,
+                         const qrx_moe_opts *opts, void *stream)
+{
+    return moe_forward_impl(c, x, T, Wr, bias, routed, shared, topk_idx, topk_w, out, ws, ws_bytes,
+                            nullptr, stream, opts);
+}
+
 int qrx_moe_forward_profiled(const qrx_cfg *c, const void *x, int32_t T, const float *Wr,
                              const float *bias, const qrx_experts *routed,
                              const qrx_experts *shared, int32_t *topk_idx, float *topk_w,
                              float *out, void *ws, size_t ws_bytes, void *const *events,
-                             int32_t n_events, void *stream)
+                             int32_t n_events, const qrx_moe_opts *opts, void *stream)
 {
     if (!events || n_events != 7) return QRX_EINVAL;
     for (int i = 0; i < 7; ++i)
         if (!events[i]) return QRX_EINVAL;
     return moe_forward_impl(c, x, T, Wr, bias, routed, shared, topk_idx, topk_w, out, ws, ws_bytes,
-                            events, stream);
+                            events, stream, opts);
 }
 
 int qrx_moe_forward_hostio(const qrx_cfg *c, const void *x_host, int32_t T, const float *Wr,

@@ -25,6 +25,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 namespace qrx {
 
@@ -168,6 +169,33 @@ __device__ int g_status;
 __device__ __forceinline__ void raise_status(int code)
 {
     atomicCAS(&g_status, 0, code);
+}
+
+// Adaptive expert top-p for one token, run by a whole warp (README
+// "JustVugg/colibri", section "快速开始": the --topp knob).  Lane j < k holds
+// the weight wv of slot j.  Slots are taken by weight, largest first (equal
+// weights: the lower slot first), their weights summed in double in that
+// order, until the sum reaches thr = p * rsf; returns whether this lane's slot
+// was taken (lanes >= k: false).  Every lane runs the same steps.
+__device__ __forceinline__ bool warp_topp_keep(int lane, int k, float wv, double thr)
+{
+    bool taken = false;
+    double c = 0.0;
+    for (int n = 0; n < k; ++n) {
+        float best = (lane < k && !taken) ? wv : 0.f;
+        int bj = (lane < k && !taken) ? lane : 0x7fffffff;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+            const bool better = oj != 0x7fffffff && (bj == 0x7fffffff || ob > best || (ob == best && oj < bj));
+            if (better) { best = ob; bj = oj; }
+        }
+        if (lane == bj) taken = true;
+        c += (double)best;
+        if (c >= thr) break;
+    }
+    return taken;
 }
 
 }  // namespace qrx

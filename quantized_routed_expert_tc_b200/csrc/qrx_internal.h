@@ -32,6 +32,8 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
 // device status flag (one per device, in k_quant.cu)
 cudaError_t read_and_clear_device_flag(int *flag);
 
+cudaError_t launch_requant_fp8(const uint8_t *w8, int64_t rows, int64_t K, int64_t ld8, const float *bscale,
+                              int wbits, uint8_t *q, int64_t ldq, float *scale, int64_t lds, cudaStream_t st);
 cudaError_t launch_quantize_weights(const float *w, int64_t rows, int64_t K, int wbits,
                                     uint8_t *q, int64_t ldq, float *scale, int64_t lds,
                                     cudaStream_t st);
@@ -51,11 +53,15 @@ struct RouterArgs {
     float *logits;          // [T][E] scratch
     int32_t *idx;           // [T][k]
     float *w;               // [T][k]
+    double topp_thr;        // adaptive top-p: p * rsf; 0 = off
 };
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t st);
+cudaError_t launch_topp_prune(int32_t *idx, float *w, int T, int k, double thr, cudaStream_t st);
 
+// usage (may be null): per-expert counters [E], += this call's counts
 cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const qrx_perm &p,
-                           cudaStream_t st);
+                           cudaStream_t st, uint64_t *usage = nullptr);
+cudaError_t launch_usage_add(const int32_t *counts, int E, uint64_t *usage, cudaStream_t st);
 
 // expert FFN over the union (GEMV-shaped kernels)
 struct FfnArgs {

@@ -39,6 +39,21 @@ def activations(wl, T: int | None = None, batch: int = 0) -> np.ndarray:
     return synth.normal_f32(wl.seed, W.stream(W.K_X, batch), n).reshape(T, wl.hidden)
 
 
+def activations_correlated(wl, T: int, rho: float, batch: int = 0) -> np.ndarray:
+    """A verify batch whose T tokens share router input structure: token i is
+    sqrt(rho) * z + sqrt(1 - rho) * z_i with z common to the batch and z_i its own
+    (all N(0,1) draws; pairwise correlation rho per coordinate), formed in double
+    and rounded to f32 (bf16 workloads: then to bf16, nearest-even).  rho = 0 gives
+    independent tokens, rho = 1 identical ones."""
+    n = wl.hidden
+    z = synth.normal_f32(wl.seed, W.stream(W.K_XC, batch), n).astype(np.float64)
+    zi = synth.normal_f32(wl.seed, W.stream(W.K_X, batch), T * n).reshape(T, n).astype(np.float64)
+    x = (np.sqrt(rho) * z[None, :] + np.sqrt(1.0 - rho) * zi).astype(np.float32)
+    if wl.afmt == W.A_BF16:
+        return torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    return x
+
+
 def to_device_act(wl, x: np.ndarray, device="cuda") -> torch.Tensor:
     """Activation array -> device tensor of the workload's dtype (f32 or bf16)."""
     if wl.afmt == W.A_BF16:

@@ -44,6 +44,11 @@ class CExperts(ctypes.Structure):
                 ("s2", ctypes.c_void_p)]
 
 
+class COpts(ctypes.Structure):
+    """qrx_moe_opts."""
+    _fields_ = [("expert_top_p", ctypes.c_float), ("usage", ctypes.c_void_p)]
+
+
 class CPerm(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("counts", "offsets", "sorted", "inv", "union_ids", "n_union")]
@@ -65,9 +70,12 @@ _SIGS = {
     "qrx_strerror": ([ctypes.c_int], ctypes.c_char_p),
     "qrx_quantize_weights": ([vp, i64, i64, i32, vp, i64, vp, i64, vp], ctypes.c_int),
     "qrx_quantize_act_q8": ([vp, i64, i64, vp, vp, vp], ctypes.c_int),
+    "qrx_requant_fp8": ([vp, i64, i64, i64, vp, i32, vp, i64, vp, i64, vp], ctypes.c_int),
     "qrx_block_dots_q8": ([i32, vp, i64, i64, vp, vp, vp], ctypes.c_int),
     "qrx_route": ([P(Cfg), vp, i32, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
     "qrx_permute": ([P(Cfg), vp, i32, P(CPerm), vp], ctypes.c_int),
+    "qrx_topp_prune": ([P(Cfg), vp, vp, i32, ctypes.c_float, vp], ctypes.c_int),
+    "qrx_usage_accumulate": ([P(Cfg), P(CPerm), vp, vp], ctypes.c_int),
     "qrx_expert_ffn": ([P(Cfg), P(CExperts), P(CPerm), P(CAct), i32, vp, vp, vp, sz, vp],
                        ctypes.c_int),
     "qrx_expert_ffn_noalloc": ([P(Cfg), P(CExperts), P(CPerm), P(CAct), i32, vp, vp],
@@ -77,10 +85,12 @@ _SIGS = {
     "qrx_combine": ([P(Cfg), vp, vp, vp, vp, i32, vp, vp], ctypes.c_int),
     "qrx_moe_forward": ([P(Cfg), vp, i32, vp, vp, P(CExperts), P(CExperts), vp, vp, vp, vp, sz,
                          vp], ctypes.c_int),
+    "qrx_moe_forward_opts": ([P(Cfg), vp, i32, vp, vp, P(CExperts), P(CExperts), vp, vp, vp, vp,
+                              sz, P(COpts), vp], ctypes.c_int),
     "qrx_moe_forward_hostio": ([P(Cfg), vp, i32, vp, vp, P(CExperts), P(CExperts), vp, vp, sz,
                                 vp], ctypes.c_int),
     "qrx_moe_forward_profiled": ([P(Cfg), vp, i32, vp, vp, P(CExperts), P(CExperts), vp, vp, vp,
-                                  vp, sz, ctypes.POINTER(vp), i32, vp], ctypes.c_int),
+                                  vp, sz, ctypes.POINTER(vp), i32, P(COpts), vp], ctypes.c_int),
 }
 
 
@@ -282,15 +292,46 @@ def qrx_combine(cfg, y_sorted, y_sh, topk_w, inv, out, stream=None):
 
 
 def qrx_moe_forward(cfg, x, Wr, bias, routed: Experts, shared: Experts | None, topk_idx, topk_w,
-                    out, ws, stream=None):
+                    out, ws, stream=None, topp: float = 0.0, usage=None):
+    """The whole layer.  topp > 0 or a usage tensor (uint64/int64 [E] on the
+    device) go through qrx_moe_forward_opts."""
     sh = ctypes.byref(shared.c()) if shared is not None else None
+    if topp or usage is not None:
+        opts = COpts(float(topp), _p(usage))
+        _check("qrx_moe_forward_opts", lib().qrx_moe_forward_opts(
+            ctypes.byref(cfg), _p(x), x.shape[0], _p(Wr), _p(bias), ctypes.byref(routed.c()), sh,
+            _p(topk_idx), _p(topk_w), _p(out), _p(ws), ws.numel(), ctypes.byref(opts), _st(stream)))
+        return
     _check("qrx_moe_forward", lib().qrx_moe_forward(
         ctypes.byref(cfg), _p(x), x.shape[0], _p(Wr), _p(bias), ctypes.byref(routed.c()), sh,
         _p(topk_idx), _p(topk_w), _p(out), _p(ws), ws.numel(), _st(stream)))
 
 
+def qrx_requant_fp8(w8, bscale, wbits: int, q, scale, stream=None):
+    """FP8 e4m3 rows (uint8 [rows][K]) with 128x128 block scales -> packed codes q
+    [rows][K*wbits/8] and row scales [rows]."""
+    rows, K = w8.shape
+    if w8.stride(1) != 1 or not w8.is_cuda:
+        raise ValueError("w8 rows must be contiguous device memory (a row stride is allowed)")
+    _check("qrx_requant_fp8", lib().qrx_requant_fp8(w8.data_ptr(), rows, K, w8.stride(0), _p(bscale), wbits,
+                                                    _p(q), q.stride(0), _p(scale), 1, _st(stream)))
+
+
+def qrx_topp_prune(cfg, topk_idx, topk_w, p: float, stream=None):
+    """Adaptive expert top-p in place on a router output [T][k]."""
+    _check("qrx_topp_prune", lib().qrx_topp_prune(ctypes.byref(cfg), _p(topk_idx), _p(topk_w),
+                                                  topk_idx.shape[0], float(p), _st(stream)))
+
+
+def qrx_usage_accumulate(cfg, perm, usage, stream=None):
+    """usage[e] += perm.counts[e] (usage: uint64/int64 [E] device tensor)."""
+    _check("qrx_usage_accumulate", lib().qrx_usage_accumulate(ctypes.byref(cfg), ctypes.byref(perm.c()),
+                                                              _p(usage), _st(stream)))
+
+
 def qrx_moe_forward_profiled(cfg, x, Wr, bias, routed: Experts, shared: Experts | None,
-                             topk_idx, topk_w, out, ws, events, stream=None):
+                             topk_idx, topk_w, out, ws, events, stream=None, topp: float = 0.0,
+                             usage=None):
     """qrx_moe_forward recording 7 torch.cuda.Event objects between its stages."""
     sh = ctypes.byref(shared.c()) if shared is not None else None
     for ev in events:                     # torch creates the CUDA event on first record
@@ -299,7 +340,8 @@ def qrx_moe_forward_profiled(cfg, x, Wr, bias, routed: Experts, shared: Experts 
     arr = (vp * 7)(*[ev.cuda_event for ev in events])
     _check("qrx_moe_forward_profiled", lib().qrx_moe_forward_profiled(
         ctypes.byref(cfg), _p(x), x.shape[0], _p(Wr), _p(bias), ctypes.byref(routed.c()), sh,
-        _p(topk_idx), _p(topk_w), _p(out), _p(ws), ws.numel(), arr, len(events), _st(stream)))
+        _p(topk_idx), _p(topk_w), _p(out), _p(ws), ws.numel(), arr, len(events),
+        ctypes.byref(COpts(float(topp), _p(usage))), _st(stream)))
 
 
 def qrx_moe_forward_hostio(cfg, x_host, Wr, bias, routed: Experts, shared: Experts | None,

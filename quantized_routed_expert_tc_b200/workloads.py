@@ -29,7 +29,7 @@ A_F32, A_Q8, A_BF16 = 0, 1, 2
 AFMT_NAMES = {A_F32: "f32", A_Q8: "q8_0", A_BF16: "bf16"}
 
 # stream ids: (kind << 32) | index
-K_GATE, K_UP, K_DOWN, K_WR, K_BIAS, K_X = 1, 2, 3, 4, 5, 6
+K_GATE, K_UP, K_DOWN, K_WR, K_BIAS, K_X, K_XC = 1, 2, 3, 4, 5, 6, 7
 W_STD = 0.02
 
 

@@ -66,7 +66,7 @@ def check_routing(r, idx_gpu, w_gpu):
     return ties
 
 
-def gpu_layer(glay, wl, x_np, bias=None, bits=None):
+def gpu_layer(glay, wl, x_np, bias=None, bits=None, topp=0.0, usage=None):
     """Whole layer through qrx_moe_forward; returns (idx, w, out) on the host."""
     bits = wl.wbits if bits is None else bits
     cfg = qrx.cfg_of(wl.with_(wbits=bits))
@@ -77,7 +77,7 @@ def gpu_layer(glay, wl, x_np, bias=None, bits=None):
     out = torch.empty((T, wl.hidden), dtype=torch.float32, device="cuda")
     ws = qrx.workspace(cfg, T)
     qrx.qrx_moe_forward(cfg, x, glay.Wr, glay.bias if bias is None else bias,
-                        glay.routed[bits], glay.shared[bits], idx, w, out, ws)
+                        glay.routed[bits], glay.shared[bits], idx, w, out, ws, topp=topp, usage=usage)
     torch.cuda.synchronize()
     assert qrx.qrx_last_error() == qrx.QRX_OK
     return np_(idx), np_(w), np_(out)
@@ -110,13 +110,13 @@ def gpu_staged(glay, wl, x_np, idx_np, w_np, bits=None):
     return np_(out)
 
 
-def check_layer(glay, olay, wl, x_np, tokens, bits=None, bias_np=None):
+def check_layer(glay, olay, wl, x_np, tokens, bits=None, bias_np=None, topp=0.0):
     """Whole-layer parity on the listed tokens (near-ties resolved by the oracle)."""
     bits = wl.wbits if bits is None else bits
     wlb = wl.with_(wbits=bits)
     bias_np = router_weights(wl)[1] if bias_np is None else bias_np
-    idx, w, out = gpu_layer(glay, wlb, x_np, bias=cu(bias_np), bits=bits)
-    r, ref = olay.forward_tokens(wlb, x_np, tokens, bias=bias_np)
+    idx, w, out = gpu_layer(glay, wlb, x_np, bias=cu(bias_np), bits=bits, topp=topp)
+    r, ref = olay.forward_tokens(wlb, x_np, tokens, bias=bias_np, topp=topp)
     ties = check_routing(r, idx, w)
     got = out[list(tokens)]
     if ties:
@@ -372,6 +372,109 @@ def test_small_bf16_tensor_cores_stages(small_tc):
     assert rel_err(np_(yd), y_o) <= TOL
 
 
+# ------------------------------------------------------------------ adaptive top-p, usage
+@pytest.mark.parametrize("p", [0.3, 0.5, 0.7, 0.9])
+def test_topp_prune_bitexact(tiny, p):
+    """qrx_topp_prune on the oracle router's output: idx and w bit-exact."""
+    glay, olay = tiny
+    wl = W.TINY.with_(T=300)
+    x = activations(wl, 300, batch=11)
+    _, bias = router_weights(wl)
+    r = oracle.router(wl, x, olay.Wr, bias)
+    i_ref, w_ref, _ = oracle.topp_prune(r["idx"], r["w"], p, wl.rsf)
+    idx, w = cu(r["idx"]), cu(r["w"])
+    qrx.qrx_topp_prune(qrx.cfg_of(wl), idx, w, p)
+    torch.cuda.synchronize()
+    assert qrx.qrx_last_error() == qrx.QRX_OK
+    assert np.array_equal(np_(idx), i_ref)
+    assert np.array_equal(np_(w).view(np.uint32), w_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("afmt", [W.A_F32, W.A_Q8])
+def test_tiny_layer_topp(tiny, afmt):
+    """The whole layer with top-p 0.7 fused into the router: every token."""
+    glay, olay = tiny
+    wl = W.TINY.with_(T=40, afmt=afmt)
+    res = check_layer(glay, olay, wl, activations(wl, 40, batch=12), range(40), topp=0.7)
+    dropped = int((res["idx"] < 0).sum())
+    assert 0 < dropped < 40 * wl.top_k
+
+
+def test_small_tc_layer_topp(small_tc):
+    """Top-p on the tensor-core engine: fewer positions than T*k in every expert tile."""
+    glay, olay = small_tc
+    wl = W.SMALL_TC
+    check_layer(glay, olay, wl, activations(wl, 300, batch=13), range(0, 300, 7), topp=0.7)
+
+
+def test_usage_counters(tiny):
+    """Usage counters from the fused permutation equal the routed assignments per
+    expert, summed over calls; qrx_usage_accumulate adds a permutation's counts."""
+    glay, olay = tiny
+    wl = W.TINY.with_(T=50)
+    usage = torch.zeros(wl.n_experts, dtype=torch.int64, device="cuda")
+    ref = np.zeros(wl.n_experts, np.uint64)
+    for b, p in enumerate([0.0, 0.7, 0.0]):
+        x = activations(wl, 50, batch=20 + b)
+        idx, _, _ = gpu_layer(glay, wl, x, topp=p, usage=usage)
+        ref += oracle.usage(idx, wl.n_experts)
+    torch.cuda.synchronize()
+    assert np.array_equal(np_(usage).astype(np.uint64), ref)
+    # the stage entry point
+    c = qrx.cfg_of(wl)
+    perm = qrx.Perm.empty(50, wl.top_k, wl.n_experts)
+    qrx.qrx_permute(c, cu(idx), perm)
+    u2 = torch.zeros(wl.n_experts, dtype=torch.int64, device="cuda")
+    qrx.qrx_usage_accumulate(c, perm, u2)
+    qrx.qrx_usage_accumulate(c, perm, u2)
+    torch.cuda.synchronize()
+    assert np.array_equal(np_(u2).astype(np.uint64), 2 * oracle.usage(idx, wl.n_experts))
+
+
+@pytest.mark.parametrize("bits", [8, 4, 2])
+def test_requant_fp8_bitexact(dev, bits):
+    """FP8 (128x128 block scales) -> packed per-row codes: every byte value (NaN and
+    subnormal codes included), ragged blocks (300 x 224), a padded row stride, and one
+    GLM down-projection matrix (6144 x 2048); codes and scales bit-exact."""
+    rng = np.random.default_rng(40 + bits)
+    for rows, K, ld in ((300, 224, 224), (300, 224, 260), (6144, 2048, 2048)):
+        w8 = rng.integers(0, 256, size=(rows, ld), dtype=np.uint8)
+        bs = (rng.random(((rows + 127) // 128, (K + 127) // 128)) * 0.01 + 1e-4).astype(np.float32)
+        q_ref, s_ref = oracle.requant_fp8(np.ascontiguousarray(w8[:, :K]), bs, bits)
+        w8_d = cu(w8)[:, :K]
+        q = torch.zeros((rows, K * bits // 8), dtype=torch.uint8, device="cuda")
+        sc = torch.zeros(rows, dtype=torch.float32, device="cuda")
+        qrx.qrx_requant_fp8(w8_d, cu(bs), bits, q, sc)
+        torch.cuda.synchronize()
+        assert qrx.qrx_last_error() == qrx.QRX_OK
+        assert np.array_equal(np_(q), q_ref), (rows, K, ld)
+        assert np.array_equal(np_(sc).view(np.uint32), s_ref.view(np.uint32)), (rows, K, ld)
+
+
+@pytest.mark.parametrize("rho", [0.0, 0.6, 0.95])
+def test_verify_batch_union(glm, rho):
+    """Union size of correlated verify batches through the library's router and
+    permutation equals the oracle's (batches without router near-ties)."""
+    from quantized_routed_expert_tc_b200.layer import activations_correlated
+    glay, olay = glm
+    for T in (2, 4, 16):
+        wl = W.GLM_DECODE_T1.with_(T=T)
+        c = qrx.cfg_of(wl)
+        x = activations_correlated(wl, T, rho, batch=7)
+        r = oracle.router(wl, x, olay.Wr, olay.bias)
+        nu_ref = oracle.permute(r["idx"], wl.n_experts)["n_union"]
+        idx = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+        ws = qrx.workspace(c, T)
+        qrx.qrx_route(c, to_device_act(wl, x), glay.Wr, glay.bias, idx, w, ws)
+        perm = qrx.Perm.empty(T, wl.top_k, wl.n_experts)
+        qrx.qrx_permute(c, idx, perm)
+        torch.cuda.synchronize()
+        assert qrx.qrx_last_error() == qrx.QRX_OK
+        if not r["ties"].any():
+            assert int(perm.n_union.item()) == nu_ref, (T, rho)
+
+
 # ------------------------------------------------------------------ GLM-shaped layer, full size
 def test_glm_decode_t1(glm):
     glay, olay = glm
@@ -386,6 +489,17 @@ def test_glm_decode_t32_q8(glm):
     res = check_layer(glay, olay, wl, activations(wl), [0, 13, 31])
     n_union = len(np.unique(res["idx"]))
     assert n_union < 256                       # skewed bias: the union is below E
+
+
+def test_glm_decode_t32_q8_topp(glm):
+    """Top-p 0.7 at the GLM shape: sampled tokens match, and the union shrinks."""
+    glay, olay = glm
+    wl = W.GLM_DECODE_T32_Q8
+    x = activations(wl)
+    res = check_layer(glay, olay, wl, x, [0, 13, 31], topp=0.7)
+    idx0, _, _ = gpu_layer(glay, wl, x)
+    nu_p = len(np.unique(res["idx"][res["idx"] >= 0]))
+    assert nu_p < len(np.unique(idx0))
 
 
 def test_glm_verify_t4_bf16(glm):

@@ -589,3 +589,27 @@ def test_requant_power_of_two_scales():
             q2, s2 = oracle.requant_fp8(w8, bs * np.float32(2.0 ** m), bits)
             assert np.array_equal(q, q2)
             assert np.array_equal(s2, s * np.float32(2.0 ** m))
+
+
+# --------------------------------------------------------------------------- verify-batch union
+def test_union_of_correlated_batches():
+    """Union size of a verify batch (README "JustVugg/colibri", "已实现的功能": MTP
+    verification routes extra experts): identical tokens (rho = 1) route to exactly k
+    experts; independent tokens (rho = 0) are the plain draws; the union never exceeds
+    min(E, T*k) and grows with T."""
+    from quantized_routed_expert_tc_b200.layer import activations_correlated, router_weights
+    wl = W.TINY
+    Wr, bias = router_weights(wl)
+    x1 = activations_correlated(wl, 6, 1.0, batch=3)
+    assert (x1 == x1[0]).all()
+    r = oracle.router(wl, x1, Wr, bias)
+    assert oracle.permute(r["idx"], wl.n_experts)["n_union"] == wl.top_k
+    x0 = activations_correlated(wl, 6, 0.0, batch=3)
+    from quantized_routed_expert_tc_b200 import synth as S
+    assert np.array_equal(x0, S.normal_f32(wl.seed, W.stream(W.K_X, 3), 6 * wl.hidden).reshape(6, -1))
+    last = 0
+    for T in (1, 2, 4, 8):
+        x = activations_correlated(wl, T, 0.5, batch=4)
+        nu = oracle.permute(oracle.router(wl, x, Wr, bias)["idx"], wl.n_experts)["n_union"]
+        assert wl.top_k <= nu <= min(wl.n_experts, T * wl.top_k) and nu >= last
+        last = nu
