@@ -227,8 +227,9 @@ struct GvSmem {
 };
 
 // Shared memory: `stages` ring stages (weights, then the block's row scales),
-// their mbarriers and arrival counters, the token group's digit records,
-// per-stage partial sums [ts][tpc][wpt][R], token rows, the slot cost prefix.
+// their mbarriers and arrival counters, staged digit records (recb = 0: the
+// kernel reads them from global memory), per-stage partial sums
+// [ts][tpc][wpt][R], token rows, the slot cost prefix.
 __host__ __device__ inline GvSmem gv_smem(int stages, int ts, int recb, int rb, int tpc, int wpt,
                                           int R, int maxslots)
 {
@@ -346,6 +347,42 @@ struct LaneDig {
 #pragma unroll
             for (int pl = 0; pl < NDIG; ++pl) corr[bc][pl] = WB == 8 ? 0 : co[sb * NDIG + pl];
         }
+    }
+
+    // The same dot product on a weight chunk already unpacked (u[word][vector]):
+    // the unpack is shared by every token that meets the chunk.
+    __device__ __forceinline__ float dot_u(const uint32_t (&u)[4][Fmt<WB>::UPW]) const
+    {
+        int acc[NBC][NDIG][2];
+#pragma unroll
+        for (int bc = 0; bc < NBC; ++bc)
+#pragma unroll
+            for (int pl = 0; pl < NDIG; ++pl) {
+                acc[bc][pl][0] = corr[bc][pl];
+                acc[bc][pl][1] = 0;
+            }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int bc = WB == 2 ? (i >> 1) : 0;
+#pragma unroll
+            for (int j = 0; j < Fmt<WB>::UPW; ++j)
+#pragma unroll
+                for (int pl = 0; pl < NDIG; ++pl)
+                    acc[bc][pl][i & 1] = dp4a(u[i][j], w[pl][i * Fmt<WB>::UPW + j], acc[bc][pl][i & 1]);
+        }
+        float v = 0.f;
+#pragma unroll
+        for (int bc = 0; bc < NBC; ++bc) {
+            float cv;
+            if constexpr (NDIG == 3)
+                cv = fmaf(__int2float_rn(acc[bc][2][0] + acc[bc][2][1]), 65536.f,
+                          __int2float_rn((acc[bc][0][0] + acc[bc][0][1]) +
+                                         256 * (acc[bc][1][0] + acc[bc][1][1])));
+            else
+                cv = __int2float_rn(acc[bc][0][0] + acc[bc][0][1]);
+            v = fmaf(sig[bc], cv, v);
+        }
+        return v;
     }
 
     // The lane's share of one row's dot product: exact int32 per block, then f32.
@@ -485,10 +522,7 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
     uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + M.mbar);
     int *cnt = reinterpret_cast<int *>(smem + M.cnt);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + M.abort);
-    unsigned char *dig = smem + M.dig;
     float *red = reinterpret_cast<float *>(smem + M.red);
-    int *tin = reinterpret_cast<int *>(smem + M.tin);
-    int *tout = reinterpret_cast<int *>(smem + M.tout);
     int64_t *pre = reinterpret_cast<int64_t *>(smem + M.pre);
 
     const int tid = threadIdx.x, lane = tid & 31;
@@ -595,9 +629,15 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
     }
 
     int n = 0, cur_s = -1, cur_j = -1;
-    int p0 = 0, tout1 = 0;
+    int p0 = 0, tout1 = 0, tg = 0;
     bool is_routed = false;
     LD dreg;
+    // token i of the current slot: its activation record row and its output row
+    auto row_in_of = [&](int i) -> int {
+        if (is_routed) return GATEUP ? p.sorted[p0 + i] / p.k : p0 + i;
+        return GATEUP ? i : (int)p.sh_in_row0 + i;
+    };
+    auto row_out_of = [&](int i) -> int { return is_routed ? p0 + i : (int)p.sh_out_row0 + i; };
     while (cu.valid) {
         const int nt = cu.nt;
         if (cu.s != cur_s || cu.j != cur_j) {
@@ -611,40 +651,10 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
                     p0 = 0;
                 }
             }
-            const int tg = cu.j * p.ts;
+            tg = cu.j * p.ts;
             if constexpr (TP == 1) {               // one token: its record straight from global
-                int row_in;
-                if (is_routed) {
-                    const int pos = p0 + tg;
-                    row_in = GATEUP ? p.sorted[pos] / p.k : pos;
-                    tout1 = pos;
-                } else {
-                    row_in = GATEUP ? tg : (int)p.sh_in_row0 + tg;
-                    tout1 = (int)p.sh_out_row0 + tg;
-                }
-                dreg.load(p.xrec + (size_t)row_in * RL.bytes, RL, c, K);
-            } else {
-                __syncthreads();                   // earlier readers of dig, tin, tout are done
-                if (*abort_flag) break;
-                if (tid < nt) {
-                    const int i = tg + tid;
-                    if (is_routed) {
-                        const int pos = p0 + i;
-                        tin[tid] = GATEUP ? p.sorted[pos] / p.k : pos;
-                        tout[tid] = pos;
-                    } else {
-                        tin[tid] = GATEUP ? i : (int)p.sh_in_row0 + i;
-                        tout[tid] = (int)p.sh_out_row0 + i;
-                    }
-                }
-                __syncthreads();
-                const int n16 = RL.bytes / 16;     // copy the group's records
-                for (int i = tid; i < nt * n16; i += NT) {
-                    const int t = i / n16, q = i % n16;
-                    reinterpret_cast<uint4 *>(dig + (size_t)t * RL.bytes)[q] =
-                        reinterpret_cast<const uint4 *>(p.xrec + (size_t)tin[t] * RL.bytes)[q];
-                }
-                __syncthreads();
+                dreg.load(p.xrec + (size_t)row_in_of(tg) * RL.bytes, RL, c, K);
+                tout1 = row_out_of(tg);
             }
             cur_s = cu.s;
             cur_j = cu.j;
@@ -660,28 +670,50 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
         float *rst = red + (size_t)stage * M.red_stage;
         for (int t0 = 0; t0 < nt; t0 += TP) {
             float part[V];
+            if constexpr (TP == 1) {
+                uint4 wv[R];
 #pragma unroll
-            for (int tt = 0; tt < TP; ++tt) {
-                if (t0 + tt < nt) {
-                    if constexpr (TP == 1) {
-                        uint4 wv[R];
+                for (int r = 0; r < R; ++r)
+                    wv[r] = *reinterpret_cast<const uint4 *>(blk + (size_t)r * p.row_bytes);
 #pragma unroll
-                        for (int r = 0; r < R; ++r)
-                            wv[r] = *reinterpret_cast<const uint4 *>(blk + (size_t)r * p.row_bytes);
+                for (int r = 0; r < R; ++r) part[r] = dreg.dot(wv[r]);
+            } else if constexpr (WB == 2) {
+                // int2: the unpacked chunk (16 words) does not fit beside TP tokens'
+                // digits, so each token re-reads and unpacks the chunk
 #pragma unroll
-                        for (int r = 0; r < R; ++r) part[r] = dreg.dot(wv[r]);
-                    } else {
+                for (int tt = 0; tt < TP; ++tt) {
+                    if (t0 + tt < nt) {
                         LD d;
-                        d.load(dig + (size_t)(t0 + tt) * RL.bytes, RL, c, K);
+                        d.load(p.xrec + (size_t)row_in_of(tg + t0 + tt) * RL.bytes, RL, c, K);
 #pragma unroll
                         for (int r = 0; r < R; ++r)
                             part[r * TP + tt] =
                                 d.dot(*reinterpret_cast<const uint4 *>(blk + (size_t)r * p.row_bytes));
-                    }
-                } else {
+                    } else {
 #pragma unroll
-                    for (int r = 0; r < R; ++r) part[r * TP + tt] = 0.f;
+                        for (int r = 0; r < R; ++r) part[r * TP + tt] = 0.f;
+                    }
                 }
+            } else {
+                // the pass's tokens (a missing one repeats the last, its sums discarded)
+                LD d[TP];
+#pragma unroll
+                for (int tt = 0; tt < TP; ++tt)
+                    d[tt].load(p.xrec + (size_t)row_in_of(tg + min(t0 + tt, nt - 1)) * RL.bytes, RL, c, K);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const uint4 wv = *reinterpret_cast<const uint4 *>(blk + (size_t)r * p.row_bytes);
+                    uint32_t u[4][Fmt<WB>::UPW];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) unpack_word<WB>(word_of(wv, i), u[i]);
+#pragma unroll
+                    for (int tt = 0; tt < TP; ++tt) part[r * TP + tt] = d[tt].dot_u(u);
+                }
+#pragma unroll
+                for (int tt = 0; tt < TP; ++tt)
+                    if (t0 + tt >= nt)
+#pragma unroll
+                        for (int r = 0; r < R; ++r) part[r * TP + tt] = 0.f;
             }
             // warp partials of this pass -> rst[token][team][wit][row]
             if (cpr >= 32) {
@@ -726,7 +758,7 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
                         G += src[w2 * R + 2 * q];
                         U += src[w2 * R + 2 * q + 1];
                     }
-                    const int orow = TP == 1 ? tout1 : tout[t];
+                    const int orow = TP == 1 ? tout1 : row_out_of(tg + t);
                     p.out[(int64_t)orow * p.out_ld + (row_g >> 1)] =
                         silu_mul(scl[lrow] * G, scl[lrow + 1] * U);
                 }
@@ -740,7 +772,7 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
                     const float *src = rst + ((t * p.tpc + tf) * p.wpt) * R;
                     float Y = 0.f;
                     for (int w2 = 0; w2 < p.wpt; ++w2) Y += src[w2 * R + r];
-                    const int orow = TP == 1 ? tout1 : tout[t];
+                    const int orow = TP == 1 ? tout1 : row_out_of(tg + t);
                     p.out[(int64_t)orow * p.out_ld + row] = scl[lrow] * Y;
                 }
             }
@@ -796,8 +828,10 @@ static inline bool gemv_plan(GemvPlan &pl, int wbits, int ndig, int K, int rows,
     const int tries[3] = {4, 3, 2};
     for (int i = (maxtok <= 1 ? 0 : 1); i < 3; ++i) {
         const int stages = tries[i];
+        // activation records are read from global memory (L2), not staged: a
+        // token group is bounded only by the per-stage partial sums
         auto total = [&](int ts) {
-            return gv_smem(stages, ts, p.rec.bytes, p.rb, p.tpc, p.wpt, R, maxslots).total;
+            return gv_smem(stages, ts, 0, p.rb, p.tpc, p.wpt, R, maxslots).total;
         };
         if (total(1) > GV_SMEM_MAX) continue;
         int ts = maxtok;
@@ -806,7 +840,7 @@ static inline bool gemv_plan(GemvPlan &pl, int wbits, int ndig, int K, int rows,
         while (ts > 1 && total(ts) > GV_SMEM_MAX) --ts;
         p.stages = stages;
         p.ts = ts;
-        p.sm = gv_smem(stages, ts, p.rec.bytes, p.rb, p.tpc, p.wpt, R, maxslots);
+        p.sm = gv_smem(stages, ts, 0, p.rb, p.tpc, p.wpt, R, maxslots);
         pl.smem = (size_t)p.sm.total;
         return true;
     }
