@@ -126,7 +126,8 @@ size_t qrx_workspace_bytes(const qrx_cfg *cfg, int32_t T);
  *   QRX_ENGINE_GEMV  the HBM-streaming integer-digit GEMV (any format);
  *   QRX_ENGINE_TC    grouped GEMMs on the tcgen05 tensor cores: bf16
  *                    activations, int4 weights, T >= 256, H and I multiples
- *                    of 256.
+ *                    of 256, and a CUDA driver that provides tensor-map
+ *                    encoding (without one, every shape reports the GEMV).
  * Returns QRX_EINVAL for an invalid configuration or T <= 0.  The
  * allocation-free entry point always uses the GEMV. */
 #define QRX_ENGINE_GEMV 0

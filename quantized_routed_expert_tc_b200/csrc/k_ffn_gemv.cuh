@@ -223,15 +223,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity)
 
 // ---------------------------------------------------------------- kernel
 struct GvSmem {
-    int stage_bytes, scales_off, mbar, cnt, abort, dig, red, red_stage, tin, tout, pre, total;
+    int stage_bytes, scales_off, mbar, cnt, abort, red, red_stage, pre, total;
 };
 
 // Shared memory: `stages` ring stages (weights, then the block's row scales),
-// their mbarriers and arrival counters, staged digit records (recb = 0: the
-// kernel reads them from global memory), per-stage partial sums
-// [ts][tpc][wpt][R], token rows, the slot cost prefix.
-__host__ __device__ inline GvSmem gv_smem(int stages, int ts, int recb, int rb, int tpc, int wpt,
-                                          int R, int maxslots)
+// their mbarriers and arrival counters, per-stage partial sums
+// [ts][tpc][wpt][R], the slot cost prefix.  Activation records stay in global
+// memory (L2): every lane reads its chunk's digit words from there.
+__host__ __device__ inline GvSmem gv_smem(int stages, int ts, int rb, int tpc, int wpt, int R,
+                                          int maxslots)
 {
     GvSmem m;
     m.scales_off = GV_BLK;
@@ -243,15 +243,9 @@ __host__ __device__ inline GvSmem gv_smem(int stages, int ts, int recb, int rb, 
     o += stages * 4;
     m.abort = o;
     o = align16(o + 4);
-    m.dig = o;
-    o += ts * recb;
     m.red = o;
     m.red_stage = ts * tpc * wpt * R;         // floats
     o += stages * m.red_stage * 4;
-    m.tin = o;
-    o += ts * 4;
-    m.tout = o;
-    o += ts * 4;
     o = (o + 7) & ~7;
     m.pre = o;
     o += (maxslots + 2) * 8;
@@ -831,7 +825,7 @@ static inline bool gemv_plan(GemvPlan &pl, int wbits, int ndig, int K, int rows,
         // activation records are read from global memory (L2), not staged: a
         // token group is bounded only by the per-stage partial sums
         auto total = [&](int ts) {
-            return gv_smem(stages, ts, 0, p.rb, p.tpc, p.wpt, R, maxslots).total;
+            return gv_smem(stages, ts, p.rb, p.tpc, p.wpt, R, maxslots).total;
         };
         if (total(1) > GV_SMEM_MAX) continue;
         int ts = maxtok;
@@ -840,7 +834,7 @@ static inline bool gemv_plan(GemvPlan &pl, int wbits, int ndig, int K, int rows,
         while (ts > 1 && total(ts) > GV_SMEM_MAX) --ts;
         p.stages = stages;
         p.ts = ts;
-        p.sm = gv_smem(stages, ts, 0, p.rb, p.tpc, p.wpt, R, maxslots);
+        p.sm = gv_smem(stages, ts, p.rb, p.tpc, p.wpt, R, maxslots);
         pl.smem = (size_t)p.sm.total;
         return true;
     }

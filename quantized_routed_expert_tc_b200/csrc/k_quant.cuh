@@ -62,16 +62,37 @@ __global__ void __launch_bounds__(256) k_quantize_weights(const float *__restric
 // dequantises with 128x128 block scales and requantises into the per-row
 // container).  One warp per row; each value is f32(fp8) * block scale (a NaN
 // code counts as 0), recomputed in pass 2 instead of kept: the row's FP8
-// bytes are re-read from L2.  Pass 1: absmax; pass 2: codes as
-// k_quantize_weights.  Lanes read 4 bytes at a time: K % 32 == 0, rows
-// 4-byte aligned.
-__device__ __forceinline__ float fp8_value(uint32_t byte, float scale)
+// bytes are re-read from L2.  Pass 1: absmax; pass 2: codes
+// round-half-away(fl(x / s)).  Lanes read 4 codes at a time (K % 32 == 0,
+// rows 4-byte aligned) and decode them in pairs.
+//
+// The quotient: t = x * (1/s) is within ~3 * 2^-24 (relative) of the
+// correctly rounded fl(x / s), so when t is farther than 1e-6 * |t| from a
+// half-integer both round to the same integer; only near a half-integer (or
+// when 1/s is not finite) is the division itself computed.
+__device__ __forceinline__ void fp8x4_values(uint32_t v, float sc, float (&f)[4])
 {
-    __nv_fp8_e4m3 f8;
-    f8.__x = (__nv_fp8_storage_t)byte;
-    float f = static_cast<float>(f8);
-    if (f != f) f = 0.f;
-    return __fmul_rn(f, scale);
+    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(v & 0xFFFFu), __NV_E4M3);
+    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(v >> 16), __NV_E4M3);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (f[j] != f[j]) f[j] = 0.f;
+        f[j] = __fmul_rn(f[j], sc);
+    }
+}
+
+__device__ __forceinline__ int requant_code(float x, float s, float inv, bool inv_ok, int qmin, int qmax)
+{
+    float r;
+    const float t = __fmul_rn(x, inv);
+    const float d = fabsf(t - floorf(t) - 0.5f);
+    if (inv_ok && d > 1e-6f * fabsf(t)) r = t;
+    else r = __fdiv_rn(x, s);
+    int c = (int)roundf(r);
+    return c > qmax ? qmax : (c < qmin ? qmin : c);
 }
 
 template <int WB>
@@ -92,13 +113,15 @@ __global__ void __launch_bounds__(256) k_requant_fp8(const uint8_t *__restrict__
     const float *bs = bscale + (r / 128) * ((K + 127) / 128);
     float amax = 0.f;
     for (int64_t i = lane * 4; i < K; i += 128) {
-        const uint32_t v = *reinterpret_cast<const uint32_t *>(wr + i);
-        const float sc = bs[i / 128];       // 4 consecutive columns share a block
+        float f[4];
+        fp8x4_values(*reinterpret_cast<const uint32_t *>(wr + i), bs[i / 128], f);   // 4 columns, one block
 #pragma unroll
-        for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fabsf(fp8_value((v >> (8 * j)) & 0xFFu, sc)));
+        for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fabsf(f[j]));
     }
     amax = warp_max(amax);
     const float s = __fdiv_rn(amax, (float)QMAX);
+    const float inv = s != 0.f ? __frcp_rn(s) : 0.f;
+    const bool inv_ok = s != 0.f && isfinite(inv);
     if (lane == 0) scale[r * lds] = s;
     uint32_t *qr = reinterpret_cast<uint32_t *>(q + r * ldq);
     const int64_t nwords = K / EPW;
@@ -107,16 +130,11 @@ __global__ void __launch_bounds__(256) k_requant_fp8(const uint8_t *__restrict__
         uint32_t word = 0;
 #pragma unroll
         for (int i = 0; i < EPW; i += 4) {
-            const uint32_t v = *reinterpret_cast<const uint32_t *>(wr + c0 + i);
-            const float sc = bs[(c0 + i) / 128];
+            float f[4];
+            fp8x4_values(*reinterpret_cast<const uint32_t *>(wr + c0 + i), bs[(c0 + i) / 128], f);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const float x = fp8_value((v >> (8 * j)) & 0xFFu, sc);
-                int c = 0;
-                if (s != 0.f) {
-                    c = (int)roundf(__fdiv_rn(x, s));
-                    c = c > QMAX ? QMAX : (c < QMIN ? QMIN : c);
-                }
+                const int c = s != 0.f ? requant_code(f[j], s, inv, inv_ok, QMIN, QMAX) : 0;
                 word |= ((uint32_t)c & ((1u << WB) - 1u)) << (WB * (i + j));
             }
         }

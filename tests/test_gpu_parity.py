@@ -451,6 +451,26 @@ def test_requant_fp8_bitexact(dev, bits):
         assert np.array_equal(np_(sc).view(np.uint32), s_ref.view(np.uint32)), (rows, K, ld)
 
 
+def test_requant_fp8_exact_halves(dev):
+    """Values whose quotient by the row scale lands on (or next to) a half-integer:
+    e4m3 7.0 (0x4E) sets the row maximum, 3.5 / -3.5 / 2.5 / 0.5 (0x46 / 0xC6 / 0x42 /
+    0x30) divide to exact halves at int4 (s = 1) and to near-halves at int8 and int2."""
+    rows, K = 128, 256
+    pattern = np.array([0x4E, 0x46, 0xC6, 0x42, 0x30, 0xB0, 0x00, 0x38], np.uint8)
+    w8 = np.tile(pattern, (rows, K // pattern.size))
+    w8[::3, 0] = 0x46                        # rows whose maximum is 3.5 instead
+    bs = np.ones((1, 2), np.float32)
+    bs[0, 1] = 0.5
+    for bits in (8, 4, 2):
+        q_ref, s_ref = oracle.requant_fp8(w8, bs, bits)
+        q = torch.zeros((rows, K * bits // 8), dtype=torch.uint8, device="cuda")
+        sc = torch.zeros(rows, dtype=torch.float32, device="cuda")
+        qrx.qrx_requant_fp8(cu(w8), cu(bs), bits, q, sc)
+        torch.cuda.synchronize()
+        assert np.array_equal(np_(q), q_ref), bits
+        assert np.array_equal(np_(sc).view(np.uint32), s_ref.view(np.uint32)), bits
+
+
 @pytest.mark.parametrize("rho", [0.0, 0.6, 0.95])
 def test_verify_batch_union(glm, rho):
     """Union size of correlated verify batches through the library's router and
