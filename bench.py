@@ -75,6 +75,18 @@ FALLBACK_BF16_TFLOPS = 1590.0
 TC_MIN_T = 256          # tokens from which bf16 x int4 batches run on the tensor cores
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest value of x over all ranks (the slowest rank's time); x itself on
+    one rank.  device: where the collective's tensor lives (cuda for NCCL)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def uses_tensor_cores(wl) -> bool:
     """Whether the library takes the tcgen05 path for this workload's expert FFN."""
     return wl.afmt == 2 and wl.wbits == 4 and wl.T >= TC_MIN_T
@@ -400,11 +412,7 @@ def run_qrx(args, wl, rank, world, local_rank):
         dist.barrier()
     clocks = sampler.stop()
     total = np.array([a.elapsed_time(z) for a, z in evs])        # ms per step
-    ms_step = float(total.mean())
-    if world > 1:
-        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = max_over_ranks(float(total.mean()), world, dev)
     rc = qrx.qrx_last_error()
     if rc != qrx.QRX_OK:
         raise RuntimeError(f"device error during timing: {qrx.qrx_strerror(rc)}")
@@ -456,10 +464,7 @@ def run_qrx(args, wl, rank, world, local_rank):
             es[i][1].record(stream)
         torch.cuda.synchronize(dev)
         e_ms = float(np.mean([a.elapsed_time(z) for a, z in es]))
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e_ms, world, dev)
         xbytes = T * H * (2 if wl.afmt == 2 else 4)
         e2e = {"value": T * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": xbytes,
                "d2h_bytes_per_step": T * H * 4, "ms_per_step": e_ms}

@@ -27,6 +27,7 @@
 // results are deterministic.  For gate/up the matrix rows are interleaved
 // (gate row i, up row i) so the SwiGLU is applied where both sums meet.
 #pragma once
+#include <atomic>
 #include "qrx_dev.cuh"
 
 namespace qrx {
@@ -845,14 +846,14 @@ template <int WB, int NDIG, int TP, bool GU>
 static cudaError_t gemv_go(const GemvPlan &pl, int grid, cudaStream_t st)
 {
     auto kern = k_ffn_gemv<WB, NDIG, TP, GU>;
-    static unsigned long long configured = 0;   // bit per device: max dynamic smem set
+    static std::atomic<unsigned long long> configured{0};   // bit per device: max dynamic smem set
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    if (dev >= 64 || !(configured >> dev & 1ull)) {
+    if (dev >= 64 || !(configured.load(std::memory_order_acquire) >> dev & 1ull)) {
         err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_MAX);
         if (err != cudaSuccess) return err;
-        if (dev < 64) configured |= 1ull << dev;
+        if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_release);
     }
     return launch_k(kern, dim3(grid), dim3(GvShape<WB, NDIG>::NT), pl.smem, st, pl.p);
 }

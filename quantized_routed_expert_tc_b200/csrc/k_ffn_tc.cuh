@@ -41,6 +41,7 @@
 // status flag, every role leaves its loops, the producer waits (bounded) for
 // the copies it started, and only then is TMEM freed.
 #pragma once
+#include <atomic>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <mutex>
@@ -727,14 +728,14 @@ static cudaError_t tc_go(TcP &p, const void *w, const void *w_sh, int64_t w_stri
     if (!ok) return cudaErrorInvalidValue;
     const int smem = tc_smem_bytes(maxslots);
     if (smem > GV_SMEM_MAX) return cudaErrorInvalidValue;
-    static unsigned long long configured = 0;
+    static std::atomic<unsigned long long> configured{0};   // bit per device: max dynamic smem set
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    if (dev >= 64 || !(configured >> dev & 1ull)) {
+    if (dev >= 64 || !(configured.load(std::memory_order_acquire) >> dev & 1ull)) {
         err = cudaFuncSetAttribute(k_ffn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_MAX);
         if (err != cudaSuccess) return err;
-        if (dev < 64) configured |= 1ull << dev;
+        if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_release);
     }
     return launch_k(k_ffn_tc, dim3(num_sms), dim3(TC_THREADS), (size_t)smem, st, mw, mwsh, mb, p);
 }
