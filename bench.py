@@ -102,14 +102,23 @@ def tensor_peak():
     return FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """Source text without // comments, /* */ comments and blank lines: edits to the
+    comments leave the compiled kernel, and so its measured traffic, unchanged."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln.strip())
+
+
 def kernel_source_hash(kernel: str = "k_ffn_gemv_gateup") -> str:
-    """Hash of a kernel's source: traffic figures apply only to this version."""
+    """Hash of a kernel's code (comments excluded): traffic figures apply only to it."""
     h = hashlib.sha256()
     files = ("k_ffn_tc.cuh", "qrx_dev.cuh") if kernel.startswith("k_ffn_tc") else \
         ("k_ffn_gemv.cuh", "qrx_dev.cuh")
     for f in files:
-        with open(os.path.join(ROOT, "quantized_routed_expert_tc_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "quantized_routed_expert_tc_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

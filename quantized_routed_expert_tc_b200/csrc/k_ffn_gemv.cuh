@@ -20,9 +20,13 @@
 // a "team" of CPR threads covers one row (thread c reads 16-byte chunk c) and
 // handles R = 8 consecutive rows of a block.  Activations enter as digit
 // planes (qrx_dev.cuh) prepared once per row by k_act_digits (tokens, for
-// gate/up) and k_h_digits (h rows, for down).  With one token per slot each
-// thread loads its chunk's digits straight from that record; with more, the
-// slot's token group is staged in shared memory.  Reductions
+// gate/up) and k_h_digits (h rows, for down); every thread loads its chunk's
+// digit words straight from those records (L2-resident).  With several
+// tokens per slot a pass takes TP tokens' digits into registers and reads and
+// unpacks each weight chunk once for all of them (int2, whose unpacked chunk
+// does not fit beside them, re-reads it per token); a token group is bounded
+// only by the per-stage partial sums (64 tokens at the GLM shape), so each
+// expert's weights stream once per call at decode batch sizes.  Reductions
 // are fixed-order (warp butterflies, then warp partials in index order), so
 // results are deterministic.  For gate/up the matrix rows are interleaved
 // (gate row i, up row i) so the SwiGLU is applied where both sums meet.
