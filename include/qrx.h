@@ -11,7 +11,10 @@
  *     expert of a batch read once, applied to every position routed to it);
  *   - blog "GLM-5.2 on slow computers", section "让它变得可以忍受的那些装置":
  *     the same expert in a batch is read only once; int4 container with
- *     per-row scale, dequant-on-use.
+ *     per-row scale, dequant-on-use;
+ *   - README sections "快速开始" and "如何测试，按顺序": adaptive expert top-p
+ *     (--topp) and the per-expert usage record; "已实现的功能": the FP8
+ *     (128x128 block scales) -> int4 converter.
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers owned by the caller (for
@@ -31,7 +34,8 @@
  * Tensor layouts (row-major, C order):
  *   x        [T][H]      f32 (QRX_A_F32, QRX_A_Q8_0) or bf16 (QRX_A_BF16)
  *   W_router [E][H]      f32;  bias [E] f32 (score-correction bias)
- *   topk_idx [T][k]      int32; topk_w [T][k] f32
+ *   topk_idx [T][k]      int32 (-1: a slot dropped by adaptive top-p);
+ *   topk_w   [T][k]      f32 (0 for a dropped slot)
  *   Expert weights, `n` experts back to back (n = E routed, 1 shared):
  *     w13 [n][2I][H*b/8] uint8: row 2i is gate row i, row 2i+1 is up row i
  *     s13 [n][2I]        f32 row scales of w13

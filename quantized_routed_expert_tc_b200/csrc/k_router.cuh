@@ -12,7 +12,9 @@
 // four warps that keep their quarter of the row in registers and run every
 // token over it.  More tokens: k_router_tile, 32-token x 64-expert tiles
 // staged in shared memory.  Then k_router_select, one warp per token: sigmoid,
-// bias, group scores, group choice, top-k and weights.
+// bias, group scores, group choice, top-k and weights, and (when asked)
+// adaptive expert top-p on the result (README, "快速开始": the --topp knob),
+// which k_topp_prune also applies on its own to a router output in memory.
 #pragma once
 #include "qrx_dev.cuh"
 
