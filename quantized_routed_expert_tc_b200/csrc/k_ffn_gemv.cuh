@@ -32,6 +32,7 @@
 // (gate row i, up row i) so the SwiGLU is applied where both sums meet.
 #pragma once
 #include <atomic>
+#include <cuda/atomic>
 #include "qrx_dev.cuh"
 
 namespace qrx {
@@ -731,16 +732,18 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
                 }
             }
         }
-        // ---- arrive; the last warp of this unit finalizes it and refills the stage
+        // ---- arrive; the last warp of this unit finalizes it and refills the stage.
+        // __syncwarp orders the warp's partial sums before lane 0's release; the
+        // last warp's acquire, then __syncwarp, orders its reads after everyone's.
         __syncwarp();
         int last = 0;
         if (lane == 0) {
-            __threadfence_block();
-            last = atomicAdd(&cnt[stage], 1) == NWARPS - 1;
+            cuda::atomic_ref<int, cuda::thread_scope_block> arrivals(cnt[stage]);
+            last = arrivals.fetch_add(1, cuda::memory_order_acq_rel) == NWARPS - 1;
         }
         last = __shfl_sync(0xffffffffu, last, 0);
         if (last) {
-            __threadfence_block();
+            __syncwarp();
             const float *scl = reinterpret_cast<const float *>(sbase + M.scales_off);
             const int rblk = (int)cu.b;
             if constexpr (GATEUP) {
