@@ -7,9 +7,9 @@ does.  It shares no code with the CUDA library.
 
 Parity status: every function below is pinned by tests/test_oracle_pins.py to
 something other than itself (hand-worked fixtures in tests/golden, brute force,
-closed forms, numpy/f64 recomputation).  The composition of the whole layer
-has no printed example on the colibri pages: parity unpinned at layer level,
-beyond the invariants the tests check.
+closed forms, numpy/f64 recomputation).  The colibri pages print no example of
+a whole layer; the layer composition is pinned by a closed form (structured
+tokens, router and expert rows under which every stage is a scalar expression).
 """
 from __future__ import annotations
 

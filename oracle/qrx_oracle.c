@@ -30,8 +30,10 @@
  * operations are single IEEE operations exactly as written.
  *
  * Parity pins (tests/test_oracle_pins.py) tie each function to something
- * other than itself; the layer as a whole has no printed example on the
- * pages, so "parity unpinned" applies to the layer-level composition only.
+ * other than itself.  The pages print no example of a whole layer; the layer
+ * composition is pinned by a closed form instead: one-hot tokens, chosen
+ * router logits and single-entry expert rows make every stage a scalar
+ * expression the test evaluates in double.
  */
 #include <math.h>
 #include <stdint.h>

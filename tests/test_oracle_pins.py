@@ -613,3 +613,74 @@ def test_union_of_correlated_batches():
         nu = oracle.permute(oracle.router(wl, x, Wr, bias)["idx"], wl.n_experts)["n_union"]
         assert wl.top_k <= nu <= min(wl.n_experts, T * wl.top_k) and nu >= last
         last = nu
+
+
+# --------------------------------------------------------------------------- layer closed form
+def test_layer_closed_form():
+    """The whole layer against a closed form.  Structured inputs make every stage
+    collapse to a few scalar operations:
+    - token t is one-hot at input column t (values 1, 2, -0.5), so each logit is one
+      chosen router entry times that value (exact);
+    - the logits are chosen so that each token's kept groups and top-4 experts follow
+      by hand (well separated: no near-ties);
+    - every gate/up/down row has one nonzero entry, 7 * (e + 1) / 2^m times a sign,
+      which int4 per-row quantisation represents exactly (scale (e + 1) / 2^m, code 7).
+    Expected values are formed here in double from those constants."""
+    import math
+    wl = W.TINY.with_(T=3, bias_std=0.0)                       # H 256, E 16, I 128, G 4, Gk 2, k 4
+    H, E, I, k, rsf = wl.hidden, wl.n_experts, wl.inter, wl.top_k, wl.rsf
+    xv = [1.0, 2.0, -0.5]
+    x = np.zeros((3, H), np.float32)
+    for t in range(3):
+        x[t, t] = xv[t]
+    # wanted logits per token (unlisted experts: -4, far below)
+    want = [{0: 3.0, 1: 2.5, 2: 2.0, 3: 1.5, 4: 1.0, 5: 0.5, 6: 0.0, 7: -0.5},
+            {15: 3.0, 14: 2.0, 11: 2.5, 8: 1.0},
+            {5: 4.0, 0: 1.0, 6: 0.5, 2: 0.25}]
+    Wr = np.zeros((E, H), np.float32)
+    for t in range(3):
+        for e in range(E):
+            Wr[e, t] = want[t].get(e, -4.0) / xv[t]
+    bias = np.zeros(E, np.float32)
+    sel = [[0, 1, 2, 3], [15, 11, 14, 8], [5, 0, 6, 2]]          # by hand from the logits above
+
+    def val(e, r, m):              # the one nonzero of row r of a matrix of expert e
+        return (1 if (r + e) % 2 == 0 else -1) * 7.0 * (e + 1) / 2.0 ** m
+
+    ex = {}
+    for e in range(E + 1):         # e == E: the shared expert
+        g = np.zeros((I, H), np.float32)
+        u = np.zeros((I, H), np.float32)
+        d = np.zeros((H, I), np.float32)
+        for i in range(I):
+            g[i, i % 3] = val(e, i, 6)
+            u[i, i % 3] = val(e, i + 1, 7)
+        for r in range(H):
+            d[r, r % I] = val(e, r, 8)
+        ex[e] = oracle.quantize_expert(g, u, d, 4)
+    shared = ex.pop(E)
+    idx, wt, out = oracle.moe_forward(wl, x, Wr, bias, ex, shared)
+
+    sig = lambda z: 1.0 / (1.0 + math.exp(-z))
+    for t in range(3):
+        assert idx[t].tolist() == sel[t]
+        s = [sig(want[t][e]) for e in sel[t]]
+        for j in range(k):
+            assert abs(wt[t, j] - s[j] / sum(s) * rsf) <= 1e-6 * rsf
+
+    def expert_out(e, t):          # y[r] of expert e for token t, in double
+        h = np.zeros(I)
+        for i in range(I):
+            if i % 3 == t:
+                gi, ui = val(e, i, 6) * xv[t], val(e, i + 1, 7) * xv[t]
+                h[i] = gi * sig(gi) * ui
+        return np.array([val(e, r, 8) * h[r % I] for r in range(H)])
+
+    for t in range(3):
+        ref = expert_out(E, t)
+        for j, e in enumerate(sel[t]):
+            s = [sig(want[t][q]) for q in sel[t]]
+            ref = ref + (s[j] / sum(s) * rsf) * expert_out(e, t)
+        scale = np.abs(ref).max()
+        assert scale > 0
+        assert np.abs(out[t].astype(np.float64) - ref).max() <= 1e-6 * scale, t
