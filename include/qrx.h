@@ -287,7 +287,9 @@ int qrx_expert_ffn_noalloc(const qrx_cfg *cfg, const qrx_experts *routed,
 /* ---- the whole layer --------------------------------------------------- */
 
 /* activation records -> route -> permute -> routed + shared FFN -> combine,
- * all on `stream` with no host synchronisation (capturable in a CUDA graph).
+ * all on `stream` with no host synchronisation.  (Capture into a CUDA graph
+ * is not tested; the first call on a device also raises kernels' shared-memory
+ * limits, so make one call before capturing.)
  * The kernels after the first are chained with programmatic dependent launch:
  * each may start while its predecessor drains and waits for it only where it
  * reads its output (the down kernel starts streaming its weights first).
