@@ -684,3 +684,132 @@ def test_layer_closed_form():
         scale = np.abs(ref).max()
         assert scale > 0
         assert np.abs(out[t].astype(np.float64) - ref).max() <= 1e-6 * scale, t
+
+
+def _bf16_rne(v: float) -> tuple[float, float]:
+    """v rounded to bf16 (8 significant bits, ties to even), and the distance of
+    v's scaled mantissa from the nearest rounding tie."""
+    import math
+    if v == 0.0:
+        return 0.0, 0.5
+    m, ex = math.frexp(v)                      # |m| in [0.5, 1)
+    z = m * 256.0
+    return math.ldexp(round(z), ex - 8), abs(abs(z - math.trunc(z)) - 0.5)
+
+
+@pytest.mark.parametrize("afmt", [W.A_F32, W.A_Q8, W.A_BF16])
+def test_layer_closed_form_h_rounding(afmt):
+    """The whole layer in each activation mode against a closed form that includes
+    the rounding of h before the down projection (Q8_0 re-quantisation per
+    32-block, or bf16 nearest-even).
+    - Tokens are one-hot (values 1, 2, -0.5), routed as in test_layer_closed_form.
+    - Each gate/up row has one nonzero, in a column that belongs to one token, so
+      token t's h has three nonzeros of different sizes in every 32-block of I
+      (rows 32b + t, +3, +6); every int4 row is exact (scale c, code 7).
+    - Q8_0: x's block is one-hot, so its code is +-127 and d = f32(|x|/127);
+      h's blocks hold three values, so two of them move by the quantisation.
+    The closed form checks its own guards: no value near a rounding tie, and the
+    rounding of h must change the result by far more than the tolerance."""
+    import math
+    wl = W.TINY.with_(T=3, bias_std=0.0, afmt=afmt)
+    H, E, I, k, rsf = wl.hidden, wl.n_experts, wl.inter, wl.top_k, wl.rsf
+    xv = [1.0, 2.0, -0.5]
+    x = np.zeros((3, H), np.float32)
+    for t in range(3):
+        x[t, t] = xv[t]
+    want = [{0: 3.0, 1: 2.5, 2: 2.0, 3: 1.5, 4: 1.0, 5: 0.5, 6: 0.0, 7: -0.5},
+            {15: 3.0, 14: 2.0, 11: 2.5, 8: 1.0},
+            {5: 4.0, 0: 1.0, 6: 0.5, 2: 0.25}]
+    Wr = np.zeros((E, H), np.float32)
+    for t in range(3):
+        for e in range(E):
+            Wr[e, t] = want[t].get(e, -4.0) / xv[t]
+    bias = np.zeros(E, np.float32)
+    sel = [[0, 1, 2, 3], [15, 11, 14, 8], [5, 0, 6, 2]]
+
+    def val(e, r, m):              # the one nonzero of row r: +-7 * (e + 1) * mag / 2^m
+        mag = 1 + (r + r // 32 + r // 128) % 4
+        return (1 if (r + e) % 2 == 0 else -1) * 7.0 * (e + 1) * mag / 2.0 ** m
+
+    def col(i):                    # input column of gate/up row i; columns >= 3 are zero in x
+        j = i % 32
+        return j % 3 if j < 9 else 3 + i % 5
+
+    ex = {}
+    for e in range(E + 1):
+        g = np.zeros((I, H), np.float32)
+        u = np.zeros((I, H), np.float32)
+        d = np.zeros((H, I), np.float32)
+        for i in range(I):
+            g[i, col(i)] = val(e, i, 6)
+            u[i, col(i)] = val(e, i + 1, 7)
+        for r in range(H):
+            d[r, r % I] = val(e, r, 8)
+        ex[e] = oracle.quantize_expert(g, u, d, 4)
+    shared = ex.pop(E)
+    act = x
+    if afmt == W.A_BF16:           # 1, 2 and -0.5 are exact in bf16: the top half of the f32
+        act = (x.view(np.uint32) >> 16).astype(np.uint16)
+    idx, wt, out = oracle.moe_forward(wl, act, Wr, bias, ex, shared)
+
+    sig = lambda z: 1.0 / (1.0 + math.exp(-z))
+    if afmt == W.A_Q8:             # one-hot block: code +-127, d = f32(|v| / 127)
+        xe = [math.copysign(127.0 * float(np.float32(abs(v)) / np.float32(127.0)), v) for v in xv]
+    else:
+        xe = xv
+    guard = []                     # distances from a rounding tie
+
+    def h_of(e, t):
+        h = np.zeros(I)
+        for i in range(I):
+            if col(i) == t:
+                gi, ui = val(e, i, 6) * xe[t], val(e, i + 1, 7) * xe[t]
+                h[i] = gi * sig(gi) * ui
+        return h
+
+    def h_rounded(h):
+        if afmt == W.A_F32:
+            return h
+        hr = np.zeros(I)
+        if afmt == W.A_BF16:
+            for i in range(I):
+                hr[i], dist = _bf16_rne(h[i])
+                if h[i] != 0.0:
+                    guard.append(dist)
+            return hr
+        for b in range(I // 32):   # Q8_0 per 32-block of I
+            blk = h[b * 32:(b + 1) * 32]
+            amax = np.abs(blk).max()
+            dq = float(np.float32(amax) / np.float32(127.0))
+            for j, v in enumerate(blk):
+                z = v * 127.0 / amax
+                guard.append(abs(abs(z - math.trunc(z)) - 0.5))
+                hr[b * 32 + j] = math.copysign(math.floor(abs(z) + 0.5), z) * dq
+        return hr
+
+    def layer(t, rounded):
+        s = [sig(want[t][q]) for q in sel[t]]
+        def y(e):
+            h = h_of(e, t)
+            h = h_rounded(h) if rounded else h
+            return np.array([val(e, r, 8) * h[r % I] for r in range(H)])
+        ref = y(E)
+        for j, e in enumerate(sel[t]):
+            ref = ref + (s[j] / sum(s) * rsf) * y(e)
+        return ref, s
+
+    for t in range(3):
+        assert idx[t].tolist() == sel[t]
+        ref, s = layer(t, True)
+        for j in range(k):
+            assert abs(wt[t, j] - s[j] / sum(s) * rsf) <= 1e-6 * rsf
+        scale = np.abs(ref).max()
+        assert scale > 0
+        assert np.abs(out[t].astype(np.float64) - ref).max() <= 1e-6 * scale, t
+        if afmt != W.A_F32:        # the rounding of h is visible at this tolerance
+            plain, _ = layer(t, False)
+            assert np.abs(plain - ref).max() > 100 * 1e-6 * scale, t
+    if afmt != W.A_F32:            # the oracle's f32 h is within a few ulps (~2.4e-7 relative)
+        # of the double h here, which moves a scaled mantissa (< 256) or a Q8_0 ratio
+        # (<= 127) by < 7e-5: a tie distance of 2e-4 leaves every rounding decided alike
+        assert min(guard) > 2e-4, min(guard)
