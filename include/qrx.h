@@ -250,7 +250,9 @@ int qrx_shared_ffn(const qrx_cfg *cfg, const qrx_experts *shared, const qrx_act 
                    void *stream);
 
 /* Weighted combine: out[t] = y_sh[t] + sum_j topk_w[t][j] * y_sorted[inv[t*k+j]]
- * in fixed j order.  y_sh may be NULL (no shared term).  out [T][H] f32. */
+ * in fixed j order.  y_sh may be NULL (no shared term).  A slot with
+ * inv < 0 (dropped by adaptive top-p) contributes nothing, whatever its
+ * weight.  out [T][H] f32. */
 int qrx_combine(const qrx_cfg *cfg, const float *y_sorted, const float *y_sh,
                 const float *topk_w, const int32_t *inv, int32_t T, float *out,
                 void *stream);

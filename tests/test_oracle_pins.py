@@ -454,6 +454,44 @@ def test_combine_and_layer():
     assert not out0.any()
 
 
+def test_combine_stage_properties():
+    """The combine stage alone (README "JustVugg/colibri", "已实现的功能": routed
+    experts plus the shared expert), by properties that fix it:
+    - one-hot weights (1 on one slot) with no shared term return that slot's row;
+    - a dropped slot (inv -1) counts as nothing, whatever its weight: it equals
+      the same call with that slot kept at weight 0;
+    - every slot dropped leaves the shared term;
+    - relabelling the sorted positions (rows moved, inv remapped) changes nothing."""
+    rng = np.random.default_rng(5)
+    wl = W.TINY
+    T, k, H = 5, wl.top_k, wl.hidden
+    A = T * k
+    ys = rng.standard_normal((A, H)).astype(np.float32)
+    ysh = rng.standard_normal((T, H)).astype(np.float32)
+    wt = rng.uniform(0.1, 1.0, (T, k)).astype(np.float32)
+    inv = rng.permutation(A).astype(np.int32)
+    out = oracle.combine(wl, ys, ysh, wt, inv)
+    for t in range(T):
+        for j in range(k):
+            oh = np.zeros((T, k), np.float32)
+            oh[t, j] = 1.0
+            sel = oracle.combine(wl, ys, None, oh, inv)
+            assert np.array_equal(sel[t], ys[inv[t * k + j]])
+            assert not np.delete(sel, t, axis=0).any()
+    drop = inv.copy()
+    dropped = [1, 6, 7, 12]
+    drop[dropped] = -1
+    w0 = wt.copy().ravel()
+    w0[dropped] = 0.0
+    assert np.array_equal(oracle.combine(wl, ys, ysh, wt, drop),
+                          oracle.combine(wl, ys, ysh, w0.reshape(T, k), inv))
+    assert np.array_equal(oracle.combine(wl, ys, ysh, wt, np.full(A, -1, np.int32)), ysh)
+    relabel = rng.permutation(A)                    # row p moves to relabel[p]
+    ys2 = np.empty_like(ys)
+    ys2[relabel] = ys
+    assert np.array_equal(oracle.combine(wl, ys2, ysh, wt, relabel[inv].astype(np.int32)), out)
+
+
 # --------------------------------------------------------------------------- adaptive top-p
 def test_topp_fixture():
     """Hand-derived cases: README "JustVugg/colibri", "快速开始" (--topp)."""
