@@ -92,6 +92,19 @@ def uses_tensor_cores(wl) -> bool:
     return wl.afmt == 2 and wl.wbits == 4 and wl.T >= TC_MIN_T
 
 
+def gateup_weight_bytes(wl, n_union):
+    """Algorithmic bytes of one gate/up launch: each union expert and the shared
+    expert read once, 2I rows of H codes plus one f32 scale each."""
+    return (n_union + 1) * (2 * wl.inter * (wl.hidden * wl.wbits // 8 + 4))
+
+
+def tc_gateup_flops(wl, T: int) -> float:
+    """Algorithmic flops of one tensor-core gate/up launch: 2 per weight x token
+    product, over every assignment plus the shared expert's T tokens, for the
+    2I gate and up rows of H inputs."""
+    return 2.0 * (T * wl.top_k + T) * (2 * wl.inter) * wl.hidden
+
+
 def tensor_peak():
     """Dense bf16 tensor peak (burst: the kernel is timed between its own events)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -454,17 +467,13 @@ def run_qrx(args, wl, rank, world, local_rank):
     # algorithmic bytes: each union expert and the shared expert read once
     nu = np.array([unions[i % npool] for i in range(nprof)], dtype=np.float64)
     exp_bytes = wl.expert_bytes()
-    I, b = wl.inter, wl.wbits
-    gateup_bytes = (nu + 1) * (2 * I * (H * b // 8 + 4))
-    layer_bytes = (nu + 1) * exp_bytes
+    gateup_bytes = gateup_weight_bytes(wl, nu)
     gu_ms = per[:, 3]          # the gate/up kernel alone (stage 3)
     achieved = float((gateup_bytes / (gu_ms / 1e3)).mean() / 1e9)
     peak, peak_kind = peaks()
     tc = uses_tensor_cores(wl)
     if tc:
-        # tensor-core path: 2 flops per weight x token product, every assignment
-        # plus the shared expert's T tokens, gate and up rows (2I x H)
-        gateup_flops = 2.0 * (T * k + T) * (2 * I) * H
+        gateup_flops = tc_gateup_flops(wl, T)
         tc_achieved = gateup_flops / float(gu_ms.mean() / 1e3) / 1e12
         tc_peak, tc_peak_kind = tensor_peak()
     nu_all = np.array([unions[i % npool] for i in range(args.steps)], dtype=np.float64)

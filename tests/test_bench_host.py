@@ -84,3 +84,23 @@ def test_reference_arm_other_ranks_print_nothing():
                     "--warmup", "1"], env_extra={"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0
     assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_algorithmic_figures():
+    """The roofline's algorithmic bytes and flops, against figures worked out by
+    hand for the GLM-shaped layer (H 6144, I 2048, top-8, int4)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from quantized_routed_expert_tc_b200 import workloads as W
+    wl = W.GLM_DECODE_T1
+    # one expert: gate + up = 4096 rows x (3072 code bytes + 4 scale bytes),
+    # down = 6144 rows x (1024 + 4)
+    assert wl.expert_bytes() == 4096 * 3076 + 6144 * 1028 == 18_915_328
+    # T = 1: 8 routed experts + the shared one, gate/up rows only
+    assert bench.gateup_weight_bytes(wl, 8) == 9 * 4096 * 3076 == 113_393_664
+    assert bench.gateup_weight_bytes(wl.with_(wbits=8), 8) == 9 * 4096 * 6148
+    assert bench.gateup_weight_bytes(wl.with_(wbits=2), 8) == 9 * 4096 * 1540
+    # 2048-token prefill: (2048 * 8 + 2048) rows of tokens x 4096 weight rows x 6144 inputs, 2 flops each
+    pf = W.GLM_PREFILL_T2048_BF16
+    assert bench.tc_gateup_flops(pf, 2048) == 2 * 18432 * 4096 * 6144 == 927_712_935_936
+    assert bench.uses_tensor_cores(pf) and not bench.uses_tensor_cores(wl)
