@@ -124,12 +124,16 @@ def tensor_peak():
 
 
 def _code_only(text: str) -> str:
-    """Source text without // comments, /* */ comments and blank lines: edits to the
-    comments leave the compiled kernel, and so its measured traffic, unchanged."""
+    """The code the measured (default) build compiles: the source without // and
+    /* */ comments, blank lines, and the lines that exist only for bounds-checked
+    builds (QRX_CHECK_OR / QRX_CHECK_ONLY and the qrx_check.cuh include, which
+    expand to nothing without -DQRX_CHECK).  Edits to any of those leave the
+    compiled kernel, and so its measured traffic, unchanged."""
     import re
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     lines = (re.sub(r"//.*", "", ln).rstrip() for ln in text.splitlines())
-    return "\n".join(ln for ln in lines if ln.strip())
+    return "\n".join(ln for ln in lines
+                     if ln.strip() and not re.search(r"qrx_check", ln, flags=re.I))
 
 
 def kernel_source_hash(kernel: str = "k_ffn_gemv_gateup") -> str:

@@ -4,6 +4,7 @@
 // experts plus a shared expert; weights from the router).
 #pragma once
 #include "qrx_dev.cuh"
+#include "qrx_check.cuh"
 
 namespace qrx {
 
@@ -26,6 +27,7 @@ __global__ void __launch_bounds__(256) k_combine(const float *__restrict__ y, co
         const float wj = w[a];
         const int p = inv[a];
         if (p < 0) continue;
+        QRX_CHECK_OR(p < (int64_t)T * k, continue);
         const float4 v = *reinterpret_cast<const float4 *>(y + (int64_t)p * H + h);
         acc.x = fmaf(wj, v.x, acc.x);
         acc.y = fmaf(wj, v.y, acc.y);

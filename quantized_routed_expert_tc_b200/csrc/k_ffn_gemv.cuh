@@ -34,6 +34,7 @@
 #include <atomic>
 #include <cuda/atomic>
 #include "qrx_dev.cuh"
+#include "qrx_check.cuh"
 
 namespace qrx {
 
@@ -540,6 +541,9 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
     // has ceil(ntok/TS) groups (all full but the last): nblk * (BWU*groups + ntok).
     const int nu = p.routed ? *p.n_union : 0;
     const int nslots = nu + (p.shared ? 1 : 0);
+    QRX_CHECK_ONLY(const int64_t n_pos = p.routed ? (int64_t)p.T * p.k : 0;)   // routed positions
+    QRX_CHECK_ONLY(const int64_t n_in = GATEUP ? (int64_t)p.T : max(n_pos, p.shared ? p.sh_in_row0 + p.T : (int64_t)0);)
+    QRX_CHECK_ONLY(const int64_t n_out = max(n_pos, p.shared ? p.sh_out_row0 + p.T : (int64_t)0);)
     if (tid < 32) {
         int64_t run = 0;
         for (int s0 = 0; s0 < nslots; s0 += 32) {
@@ -634,6 +638,8 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
     LD dreg;
     // token i of the current slot: its activation record row and its output row
     auto row_in_of = [&](int i) -> int {
+        QRX_CHECK_OR(!is_routed || (int64_t)p0 + i < n_pos, return 0);
+        QRX_CHECK_OR(!is_routed || !GATEUP || (p.sorted[p0 + i] >= 0 && p.sorted[p0 + i] / p.k < n_in), return 0);
         if (is_routed) return GATEUP ? p.sorted[p0 + i] / p.k : p0 + i;
         return GATEUP ? i : (int)p.sh_in_row0 + i;
     };
@@ -761,6 +767,7 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
                         U += src[w2 * R + 2 * q + 1];
                     }
                     const int orow = TP == 1 ? tout1 : row_out_of(tg + t);
+                    QRX_CHECK_OR(orow >= 0 && orow < n_out, continue);
                     p.out[(int64_t)orow * p.out_ld + (row_g >> 1)] =
                         silu_mul(scl[lrow] * G, scl[lrow + 1] * U);
                 }
@@ -775,6 +782,7 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
                     float Y = 0.f;
                     for (int w2 = 0; w2 < p.wpt; ++w2) Y += src[w2 * R + r];
                     const int orow = TP == 1 ? tout1 : row_out_of(tg + t);
+                    QRX_CHECK_OR(orow >= 0 && orow < n_out, continue);
                     p.out[(int64_t)orow * p.out_ld + row] = scl[lrow] * Y;
                 }
             }

@@ -46,6 +46,7 @@
 #include <cudaTypedefs.h>
 #include <mutex>
 #include "qrx_dev.cuh"
+#include "qrx_check.cuh"
 
 namespace qrx {
 
@@ -493,6 +494,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     } else if (warp >= TC_EPI0 && warp < TC_EPI0 + 4) {
         // ================= epilogue (warps 4..7) =================
         const int q4 = warp & 3;                   // TMEM lane quarter of this warp
+        QRX_CHECK_ONLY(const int64_t n_out = max(p.routed ? (int64_t)p.T * p.k : (int64_t)0, p.shared ? p.sh_out_row0 + p.T : (int64_t)0);)
         int local = 0;
         for (int64_t it = blockIdx.x; it < nitems && !*abort_flag; it += gridDim.x, ++local) {
             const TcItem d = tc_decode(p, pre, nslots, nu, it);
@@ -532,6 +534,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                             // gate on even rows, up on the odd row after it
                             const float other = __shfl_xor_sync(0xffffffffu, acc, 1);
                             if ((lane & 1) || n >= d.nv) continue;
+                            QRX_CHECK_OR(orow >= 0 && orow < n_out, continue);
                             const int pair = rowg >> 1;
                             const float h = silu_mul(acc, other);
                             if (p.out) p.out[orow * p.out_ld + pair] = h;
@@ -540,6 +543,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                     __float2bfloat16_rn(h);
                         } else {
                             if (n >= d.nv) continue;
+                            QRX_CHECK_OR(orow >= 0 && orow < n_out, continue);
                             p.out[orow * p.out_ld + rowg] = acc;
                         }
                     }
@@ -624,6 +628,7 @@ __global__ void __launch_bounds__(256) k_gather_x(const __nv_bfloat16 *__restric
     int64_t t = r - A;
     if (r < A) {
         const int32_t a = sorted[r];
+        QRX_CHECK_OR(a >= 0 && a < A, (void)0);      // an invalid position is zero-filled
         t = (a >= 0 && a < A) ? a / k : -1;
     }
     uint4 v = make_uint4(0u, 0u, 0u, 0u);

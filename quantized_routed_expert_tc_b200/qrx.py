@@ -95,7 +95,10 @@ _SIGS = {
 
 
 def lib_path() -> str:
-    return _build.LIB
+    """libqrx.so, or with QRX_CHECK=1 in the environment the bounds-checked
+    libqrx_check.so (same entry points and results; misses are reported by
+    qrx_last_error)."""
+    return _build.CHECK_LIB if os.environ.get("QRX_CHECK") == "1" else _build.LIB
 
 
 def lib():

@@ -104,3 +104,13 @@ def test_algorithmic_figures():
     pf = W.GLM_PREFILL_T2048_BF16
     assert bench.tc_gateup_flops(pf, 2048) == 2 * 18432 * 4096 * 6144 == 927_712_935_936
     assert bench.uses_tensor_cores(pf) and not bench.uses_tensor_cores(wl)
+
+
+def test_code_hash_covers_the_default_build_only():
+    """The kernel hash that keys recorded traffic ignores comments and the lines
+    that exist only in bounds-checked builds, and nothing else."""
+    sys.path.insert(0, ROOT)
+    import bench
+    src = "int a = 1;  // note\n/* block */\nQRX_CHECK_OR(a < 2, return);\n#include \"qrx_check.cuh\"\n\nint b = a;\n"
+    assert bench._code_only(src) == "int a = 1;\nint b = a;"
+    assert bench._code_only("int a = 2;\nint b = a;") != bench._code_only(src)
