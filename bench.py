@@ -538,7 +538,7 @@ def run_qrx(args, wl, rank, world, local_rank):
             "weight_gbs_frac_of_measured_hbm": weight_gbs / peak,
             "weight_gbs_frac_of_8tbs": weight_gbs / SPEC_HBM_GBS,
             "n_union_mean": float(nu.mean()),
-            # assignments served per routed expert read: T*k / n_union
+            # routed slots per routed expert read, T*k / n_union (slots dropped by top-p counted)
             "reuse_ratio": float(np.mean(T * k / nu)),
             "stage_us": {s: float(per[:, j].mean() * 1e3) for j, s in enumerate(stages)},
             "stage_note": "from qrx_moe_forward_profiled: events between kernels disable the "
