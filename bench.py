@@ -358,7 +358,11 @@ def oracle_slice(wl):
     return wl.T if wl.T <= ORACLE_SLICE else ORACLE_SLICE
 
 
-def cpu_baseline(wl, seconds: float, topp: float = 0.0):
+def cpu_baseline(wl, seconds: float, topp: float = 0.0, first=None):
+    """The oracle timed on the host cores over two batches (or their first
+    oracle_slice(wl) tokens).  `first`, when given, is the first batch (the GPU
+    arm's batch 0); the oracle's result on it is returned beside the timing, as
+    (idx, w, out), for the parity sample."""
     import numpy as np
     import oracle
     from quantized_routed_expert_tc_b200.layer import activations, expert_f32, router_weights
@@ -366,16 +370,20 @@ def cpu_baseline(wl, seconds: float, topp: float = 0.0):
     Wr, bias = router_weights(wl)
     ts = oracle_slice(wl)
     xs = [activations(wl, batch=1000 + b)[:ts] for b in range(2)]
+    if first is not None:
+        xs[0] = first[:ts]
     needed = set()
     for x in xs:
         needed.update(int(e) for e in np.unique(oracle.router(wl, x, Wr, bias)["idx"]))
     experts = {e: oracle.quantize_expert(*expert_f32(wl, e), wl.wbits) for e in sorted(needed)}
     shared = oracle.quantize_expert(*expert_f32(wl, wl.n_experts), wl.wbits)
-    n, t_total = 0, 0.0
+    n, t_total, ref = 0, 0.0, None
     while t_total < seconds or n < 2:
         t0 = time.perf_counter()
-        oracle.moe_forward(wl, xs[n % 2], Wr, bias, experts, shared, topp=topp)
+        res = oracle.moe_forward(wl, xs[n % 2], Wr, bias, experts, shared, topp=topp)
         t_total += time.perf_counter() - t0
+        if n == 0:
+            ref = res
         n += 1
         if n >= 200:
             break
@@ -384,7 +392,26 @@ def cpu_baseline(wl, seconds: float, topp: float = 0.0):
     return {"value": n * ts / t_total, "unit": "tokens/s", "cores": oracle.max_threads(),
             "kind": "oracle",
             "sample": f"{n} layer forwards of {what} over 2 distinct batches "
-                      f"({t_total:.1f} s of CPU time)"}
+                      f"({t_total:.1f} s of CPU time)"}, ref
+
+
+def parity_sample(ref, idx_gpu, out_gpu, tol: float = 1e-3) -> dict:
+    """The timed configuration against the oracle on one batch: `ref` = the
+    oracle's (idx, w, out) on the batch's first tokens, `idx_gpu` / `out_gpu` the
+    GPU layer's result on the whole batch (a token's output depends on that token
+    alone).  Tokens whose expert selection differs (a near-tie resolved the other
+    way) are counted and left out of the error."""
+    import numpy as np
+    idx_o, _, out_o = ref
+    ts = idx_o.shape[0]
+    same = np.all(np.asarray(idx_gpu)[:ts] == idx_o, axis=1)
+    got = np.asarray(out_gpu, dtype=np.float64)[:ts][same]
+    want = out_o.astype(np.float64)[same]
+    scale = float(np.abs(want).max()) if want.size else 0.0
+    err = float(np.abs(got - want).max() / scale) if scale > 0 else 0.0
+    return {"tokens": int(ts), "rows_compared": int(same.sum()),
+            "selection_differs": int((~same).sum()), "max_err_ratio": err, "tolerance": tol,
+            "ok": bool(err <= tol and same.any())}
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -515,9 +542,18 @@ def run_qrx(args, wl, rank, world, local_rank):
         e2e = {"value": T * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": xbytes,
                "d2h_bytes_per_step": T * H * 4, "ms_per_step": e_ms}
 
-    cpu = None
+    cpu = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, args.cpu_seconds, args.topp)
+        # the timed call once more on batch 0, checked against the oracle on its first tokens
+        qrx.qrx_moe_forward(cfg, xs[0], glay.Wr, glay.bias, glay.routed[wl.wbits],
+                            glay.shared[wl.wbits], idx, w, out, ws, stream, topp=args.topp)
+        torch.cuda.synchronize(dev)
+        rc = qrx.qrx_last_error()
+        if rc != qrx.QRX_OK:
+            raise RuntimeError(f"device error in the parity sample: {qrx.qrx_strerror(rc)}")
+        idx0, out0 = idx.cpu().numpy(), out.cpu().numpy()
+        cpu, ref = cpu_baseline(wl, args.cpu_seconds, args.topp, first=xs_np[0])
+        parity = parity_sample(ref, idx0, out0)
 
     if rank == 0:
         stages = ["act_records", "router", "permute", "gateup", "down", "combine"]
@@ -557,6 +593,7 @@ def run_qrx(args, wl, rank, world, local_rank):
                           "traffic": traffic, "timing": ROOFLINE_TIMING,
                           "algorithmic_bytes_per_launch": float(gateup_bytes.mean())}),
             "cpu_baseline": cpu,
+            "parity_sample": parity,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,

@@ -114,3 +114,42 @@ def test_code_hash_covers_the_default_build_only():
     src = "int a = 1;  // note\n/* block */\nQRX_CHECK_OR(a < 2, return);\n#include \"qrx_check.cuh\"\n\nint b = a;\n"
     assert bench._code_only(src) == "int a = 1;\nint b = a;"
     assert bench._code_only("int a = 2;\nint b = a;") != bench._code_only(src)
+
+
+def test_parity_sample_against_the_baseline_reference():
+    """The bench's parity sample: the CPU-baseline leg returns the oracle's result on
+    the GPU arm's first batch, and parity_sample compares the GPU rows with it."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+    from quantized_routed_expert_tc_b200 import workloads as W
+    from quantized_routed_expert_tc_b200.layer import activations, expert_f32, router_weights
+    wl = W.TINY
+    x0 = activations(wl, batch=0)
+    cpu, ref = bench.cpu_baseline(wl, 0.05, first=x0)
+    assert cpu["kind"] == "oracle" and cpu["value"] > 0
+    idx_o, w_o, out_o = ref
+    # the reference is the oracle's layer on that very batch
+    Wr, bias = router_weights(wl)
+    ex = {e: oracle.quantize_expert(*expert_f32(wl, e), wl.wbits) for e in range(wl.n_experts)}
+    sh = oracle.quantize_expert(*expert_f32(wl, wl.n_experts), wl.wbits)
+    i2, _, o2 = oracle.moe_forward(wl, x0, Wr, bias, ex, sh)
+    assert np.array_equal(i2, idx_o) and np.array_equal(o2, out_o)
+
+    same = bench.parity_sample(ref, idx_o, out_o)
+    assert same["ok"] and same["max_err_ratio"] == 0.0 and same["rows_compared"] == wl.T
+    # GPU rows beyond the oracle's slice are ignored
+    longer = np.vstack([out_o, np.full((5, wl.hidden), 1e9, np.float32)])
+    idx_longer = np.vstack([idx_o, np.zeros((5, wl.top_k), np.int32)])
+    assert bench.parity_sample(ref, idx_longer, longer)["ok"]
+    # an error above the tolerance fails
+    bad = out_o.copy()
+    bad[1, 3] += 0.01 * np.abs(out_o).max()
+    r = bench.parity_sample(ref, idx_o, bad)
+    assert not r["ok"] and 9e-3 < r["max_err_ratio"] < 1.1e-2
+    # a token whose selection differs is counted and left out
+    idx_bad = idx_o.copy()
+    idx_bad[1, 0] = (idx_bad[1, 0] + 1) % wl.n_experts
+    r = bench.parity_sample(ref, idx_bad, bad)
+    assert r["ok"] and r["selection_differs"] == 1 and r["rows_compared"] == wl.T - 1
