@@ -851,3 +851,49 @@ def test_layer_closed_form_h_rounding(afmt):
         # of the double h here, which moves a scaled mantissa (< 256) or a Q8_0 ratio
         # (<= 127) by < 7e-5: a tie distance of 2e-4 leaves every rounding decided alike
         assert min(guard) > 2e-4, min(guard)
+
+
+def test_layer_at_maximum_sizes():
+    """The largest configuration the library accepts: E = 1024 experts, top-32,
+    32 groups of 32 with 8 kept.  Each token gets 32 distinct experts, all inside
+    the 8 groups with the largest group scores (sum of the top-2 sc); the weights
+    sum to rsf; the permutation places every assignment once; and the layer equals
+    the dense per-token reference."""
+    E, k, G, Gk, H, I, T = 1024, 32, 32, 8, 64, 64, 3
+    wl = W.TINY.with_(hidden=H, inter=I, n_experts=E, n_group=G, topk_group=Gk, top_k=k, T=T)
+    ex = {}
+    for e in range(E + 1):
+        g = synth.normal_f32(61, W.stream(W.K_GATE, e), I * H, 0, 0.02).reshape(I, H)
+        u = synth.normal_f32(61, W.stream(W.K_UP, e), I * H, 0, 0.02).reshape(I, H)
+        d = synth.normal_f32(61, W.stream(W.K_DOWN, e), H * I, 0, 0.02).reshape(H, I)
+        ex[e] = oracle.quantize_expert(g, u, d, 4)
+    shared = ex.pop(E)
+    x = synth.normal_f32(62, 0, T * H).reshape(T, H)
+    Wr = synth.normal_f32(63, 0, E * H, 0, 0.1).reshape(E, H)
+    bias = synth.normal_f32(64, 0, E, 0, 0.1)
+    r = oracle.router(wl, x, Wr, bias)
+    gs = E // G
+    for t in range(T):
+        sel = r["idx"][t]
+        assert len(set(sel.tolist())) == k and sel.min() >= 0 and sel.max() < E
+        s = (1.0 / (1.0 + np.exp(-r["logits"][t].astype(np.float64)))).astype(np.float32)
+        sc = (s + bias).astype(np.float32)
+        top2 = np.sort(sc.reshape(G, gs), axis=1)[:, -2:]
+        gscore = (top2[:, 0] + top2[:, 1]).astype(np.float32)
+        best = set(np.argsort(-gscore.astype(np.float64), kind="stable")[:Gk].tolist())
+        assert set((sel // gs).tolist()) <= best
+        cand = np.array([e for e in range(E) if e // gs in best])
+        order = cand[np.lexsort((cand, -sc[cand].astype(np.float64)))]   # sc descending, then index
+        assert sel.tolist() == order[:k].tolist()
+        assert abs(float(r["w"][t].astype(np.float64).sum()) - wl.rsf) <= 1e-5 * wl.rsf
+    p = oracle.permute(r["idx"], E)
+    A = T * k
+    assert int(p["counts"].sum()) == A and sorted(p["sorted"].tolist()) == list(range(A))
+    assert all(p["sorted"][p["inv"][a]] == a for a in range(A))
+    idx, wt, out = oracle.moe_forward(wl, x, Wr, bias, ex, shared)
+    assert np.array_equal(idx, r["idx"])
+    for t in range(T):
+        acc = _dense_ffn(wl, shared, x[t])[1].astype(np.float64)
+        for j in range(k):
+            acc += float(wt[t, j]) * _dense_ffn(wl, ex[idx[t, j]], x[t])[1].astype(np.float64)
+        assert np.allclose(out[t], acc, rtol=1e-6, atol=1e-7 * np.abs(acc).max())
