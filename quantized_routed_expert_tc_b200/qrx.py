@@ -162,7 +162,17 @@ class Experts:
     s2: torch.Tensor     # [n, H] f32
 
     def c(self) -> CExperts:
-        return CExperts(_p(self.w13), _p(self.s13), _p(self.w2), _p(self.s2))
+        """The qrx_experts struct of these tensors, built once: a call passes it
+        without rebuilding it, and assigning any of the four tensors drops it."""
+        cs = self.__dict__.get("_cstruct")
+        if cs is None:
+            cs = CExperts(_p(self.w13), _p(self.s13), _p(self.w2), _p(self.s2))
+            self.__dict__["_cstruct"] = cs
+        return cs
+
+    def __setattr__(self, name, value):
+        self.__dict__.pop("_cstruct", None)
+        super().__setattr__(name, value)
 
     @staticmethod
     def empty(n: int, H: int, I: int, wbits: int, device="cuda") -> "Experts":
