@@ -6,6 +6,7 @@
 // union, run the experts' quantised SwiGLU FFNs over it, add the shared
 // expert, combine.  Every step runs in the kernels included below; the host
 // code only checks arguments, carves the caller's workspace and launches.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -36,16 +37,17 @@ constexpr int kMaxDevices = 64;
 
 int num_sms_current()
 {
-    static int cache[kMaxDevices] = {0};
+    // per device, 0 until first asked; threads that race all store the same value
+    static std::atomic<int> cache[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-    if (cache[dev] == 0) {
-        int n = 0;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             n = 148;
-        cache[dev] = n;
+        cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
 }
 
 bool chunks_ok(int64_t K, int wbits)
