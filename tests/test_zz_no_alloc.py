@@ -25,7 +25,7 @@ pytestmark = pytest.mark.gpu
 def dev():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    qbuild.build()
+    qbuild.build(check=qrx.lib_path() == qbuild.CHECK_LIB)    # the library the binding loads
     torch.cuda.set_device(0)
     return torch.device("cuda:0")
 
