@@ -29,6 +29,10 @@
  *   - Kernels that detect a bad value at run time (an expert index out of
  *     range, an exhausted bounded wait) set a sticky device flag;
  *     qrx_last_error() synchronises the device and reports it.
+ *   - libqrx_check.so, the same library built with -DQRX_CHECK, has this
+ *     ABI and these results; its kernels also test every index they take
+ *     from data (permutation positions, token rows, inv entries) against the
+ *     buffer it addresses, skip a miss and report it as QRX_EDEVICE.
  *   - Calls are not thread-safe with respect to the same workspace.
  *
  * Tensor layouts (row-major, C order):
