@@ -153,3 +153,21 @@ def test_parity_sample_against_the_baseline_reference():
     idx_bad[1, 0] = (idx_bad[1, 0] + 1) % wl.n_experts
     r = bench.parity_sample(ref, idx_bad, bad)
     assert r["ok"] and r["selection_differs"] == 1 and r["rows_compared"] == wl.T - 1
+
+
+def test_readme_bench_commands_parse(monkeypatch):
+    """Every `python bench.py ...` line of the README parses with the bench's own
+    argument parser, and every workload it names exists."""
+    import re
+    import shlex
+    sys.path.insert(0, ROOT)
+    import bench
+    from quantized_routed_expert_tc_b200 import workloads as W
+    with open(os.path.join(ROOT, "README.md"), encoding="utf-8") as f:
+        lines = [ln.split("#")[0].strip() for ln in f if ln.strip().startswith("python bench.py")]
+    assert len(lines) >= 5
+    for ln in lines:
+        argv = shlex.split(ln)[1:]
+        monkeypatch.setattr(sys, "argv", argv)
+        args = bench.parse()
+        assert args.workload in W.ALL, ln
