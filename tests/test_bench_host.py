@@ -158,7 +158,6 @@ def test_parity_sample_against_the_baseline_reference():
 def test_readme_bench_commands_parse(monkeypatch):
     """Every `python bench.py ...` line of the README parses with the bench's own
     argument parser, and every workload it names exists."""
-    import re
     import shlex
     sys.path.insert(0, ROOT)
     import bench
