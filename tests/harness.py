@@ -9,8 +9,7 @@ from __future__ import annotations
 import numpy as np
 
 import oracle
-from quantized_routed_expert_tc_b200 import synth, workloads as W
-from quantized_routed_expert_tc_b200.layer import activations, expert_f32, router_weights  # noqa: F401
+from quantized_routed_expert_tc_b200.layer import expert_f32, router_weights
 
 
 class OracleLayer:
