@@ -723,7 +723,7 @@ static cudaError_t tc_go(TcP &p, const void *w, const void *w_sh, int64_t w_stri
     p.mtiles = p.rows / TC_M;
     p.kstages = p.K / TC_BK;
     const int row_bytes = p.K / 2;
-    CUtensorMap mw, mwsh, mb;
+    CUtensorMap mw{}, mwsh{}, mb{};      // zeroed: a launch without one expert set leaves its map unused
     bool ok = true;
     if (p.routed) ok = ok && tc_map_weights(&mw, w, row_bytes, p.rows, p.E, w_stride);
     if (p.shared) ok = ok && tc_map_weights(&mwsh, w_sh, row_bytes, p.rows, 1, (int64_t)p.rows * row_bytes);
