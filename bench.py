@@ -92,6 +92,28 @@ def uses_tensor_cores(wl) -> bool:
     return wl.afmt == 2 and wl.wbits == 4 and wl.T >= TC_MIN_T
 
 
+DECODE_T_MAX = 4        # calls of up to this many tokens run the decode GEMV (k_gemv2)
+
+
+def uses_decode_gemv(wl) -> bool:
+    return not uses_tensor_cores(wl) and wl.T <= DECODE_T_MAX
+
+
+def dtype_label(wl) -> str:
+    """The arithmetic the expert FFN computes in.  GEMV engines: exact int32 sums
+    of int8 activation digits times the packed codes -- f32 / bf16 activations as
+    three int8 digit planes of a 22-bit fixed point (one power-of-two scale per
+    row in the decode GEMV, per 32-block in the multi-token GEMV), Q8_0 as its
+    int8 codes with f32 block scales; the tensor-core engine: bf16 x bf16 -> f32."""
+    if uses_tensor_cores(wl):
+        return "bf16"
+    w = f"int{wl.wbits}"
+    if wl.afmt == 1:
+        return f"int8 (Q8_0) x {w} -> int32"
+    src = "bf16" if wl.afmt == 2 else "f32"
+    return f"int8x3 digit planes (22-bit fixed point of {src}) x {w} -> int32"
+
+
 # How the dominant kernel's duration is taken: events placed between the layer's
 # kernels on the launching stream would stop the launches overlapping inside the
 # timed steps, so they go in a second loop over the same batches and weights.
@@ -136,10 +158,11 @@ def _code_only(text: str) -> str:
                      if ln.strip() and not re.search(r"qrx_check", ln, flags=re.I))
 
 
-def kernel_source_hash(kernel: str = "k_ffn_gemv_gateup") -> str:
+def kernel_source_hash(kernel: str = "k_gemv2_gateup") -> str:
     """Hash of a kernel's code (comments excluded): traffic figures apply only to it."""
     h = hashlib.sha256()
     files = ("k_ffn_tc.cuh", "qrx_dev.cuh") if kernel.startswith("k_ffn_tc") else \
+        ("k_gemv2.cuh", "qrx_dev.cuh") if kernel.startswith("k_gemv2") else \
         ("k_ffn_gemv.cuh", "qrx_dev.cuh")
     for f in files:
         with open(os.path.join(ROOT, "quantized_routed_expert_tc_b200", "csrc", f), encoding="utf-8") as fh:
@@ -517,7 +540,9 @@ def run_qrx(args, wl, rank, world, local_rank):
         tc_peak, tc_peak_kind = tensor_peak()
     nu_all = np.array([unions[i % npool] for i in range(args.steps)], dtype=np.float64)
     weight_gbs = float(((nu_all + 1) * exp_bytes).mean() / (ms_step / 1e3) / 1e9)
-    traffic = recorded_traffic("k_ffn_tc_gateup" if tc else "k_ffn_gemv_gateup", wl.name)
+    decode = uses_decode_gemv(wl)
+    gv_kernel = "k_gemv2" if decode else "k_ffn_gemv"
+    traffic = recorded_traffic("k_ffn_tc_gateup" if tc else f"{gv_kernel}_gateup", wl.name)
 
     e2e = None
     if not args.no_e2e:
@@ -557,16 +582,17 @@ def run_qrx(args, wl, rank, world, local_rank):
 
     if rank == 0:
         stages = ["act_records", "router", "permute", "gateup", "down", "combine"]
-        # library kernels per layer call: GEMV engine: activation records, router
-        # (dot + selection), permutation, gate/up, h records, down, combine = 8;
-        # tensor-core engine: router (2), permutation, token gather, gate/up, down,
-        # combine = 7 (top-p and usage add none)
-        launches_per_step = 7 if tc else 8
+        # library kernels per layer call: decode GEMV (T <= 4): router (dot +
+        # selection), permutation, gate/up, down, combine = 6; multi-token GEMV:
+        # activation records, router (2), permutation, gate/up, h records, down,
+        # combine = 8; tensor-core engine: router (2), permutation, token gather,
+        # gate/up, down, combine = 7 (top-p and usage add none)
+        launches_per_step = 7 if tc else (6 if decode else 8)
         line = {
             "metric": METRIC, "value": T * world / (ms_step / 1e3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if tc else "int32",
+            "dtype": dtype_label(wl),
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights quantised by the "
                     "library; no trained weights)",
             "config": workload_config(wl, args.topp),
@@ -587,7 +613,7 @@ def run_qrx(args, wl, rank, world, local_rank):
                           "weight_bytes_per_launch": float(gateup_bytes.mean()),
                           "weight_gbs": achieved}
                          if tc else
-                         {"kernel": "k_ffn_gemv (gate/up + SwiGLU)", "bound": "hbm",
+                         {"kernel": f"{gv_kernel} (gate/up + SwiGLU)", "bound": "hbm",
                           "achieved": achieved, "peak": peak, "unit": "GB/s",
                           "frac": achieved / peak, "peak_kind": peak_kind,
                           "traffic": traffic, "timing": ROOFLINE_TIMING,

@@ -40,13 +40,18 @@
  *   W_router [E][H]      f32;  bias [E] f32 (score-correction bias)
  *   topk_idx [T][k]      int32 (-1: a slot dropped by adaptive top-p);
  *   topk_w   [T][k]      f32 (0 for a dropped slot)
- *   Expert weights, `n` experts back to back (n = E routed, 1 shared):
- *     w13 [n][2I][H*b/8] uint8: row 2i is gate row i, row 2i+1 is up row i
- *     s13 [n][2I]        f32 row scales of w13
- *     w2  [n][H][I*b/8]  uint8: down projection rows
- *     s2  [n][H]         f32 row scales of w2
- *     (b = 8, 4 or 2 bits; packed fields as in the README: int4 low nibble
- *     first, int2 lowest bit pair first, two's-complement codes.)
+ *   Expert weights (qrx_experts): three packed matrices per expert in the
+ *   [out][in] orientation, each with per-row f32 scales, in the container the
+ *   README and the blog describe (int4 container with a per-row scale,
+ *   dequantised on use) and read in place, never repacked:
+ *     gate [I][H*b/8] uint8, scales [I]
+ *     up   [I][H*b/8] uint8, scales [I]
+ *     down [H][I*b/8] uint8, scales [H]
+ *   Expert e's matrix starts expert_stride_q bytes after expert e-1's, its
+ *   scales expert_stride_s floats after (n = E routed experts, or 1 shared);
+ *   rows are contiguous (K*b/8 bytes each).
+ *   (b = 8, 4 or 2 bits; packed fields as in the README: int4 low nibble
+ *   first, int2 lowest bit pair first, two's-complement codes.)
  *   Assignment a = t*k + j.  Sorted order groups assignments by expert,
  *   stable in a; position p indexes that order; h and y rows are positions.
  */
@@ -85,12 +90,24 @@ typedef struct {
     int32_t afmt;                  /* qrx_afmt of the activations */
 } qrx_cfg;
 
-/* Packed experts (see layout above).  All device pointers, 16-byte aligned. */
+/* One packed matrix of every expert (see layout above).  q and scale are
+ * device pointers, 16-byte aligned; expert_stride_q is a multiple of 16
+ * bytes and expert_stride_s a multiple of 4 floats (QRX_EINVAL otherwise).
+ * A set of one expert (the shared expert) ignores both strides. */
 typedef struct {
-    const uint8_t *w13;
-    const float *s13;
-    const uint8_t *w2;
-    const float *s2;
+    const uint8_t *q;          /* codes of expert 0: [rows][K*b/8] */
+    const float *scale;        /* row scales of expert 0: [rows] */
+    int64_t expert_stride_q;   /* bytes from one expert's codes to the next */
+    int64_t expert_stride_s;   /* floats from one expert's scales to the next */
+} qrx_mat;
+
+/* An expert set: the SwiGLU FFN's three matrices (README "已实现的功能":
+ * SwiGLU experts with per-row scales; blog "让它变得可以忍受的那些装置": int4
+ * container with per-row scale, dequant-on-use). */
+typedef struct {
+    qrx_mat gate;   /* [I][H*b/8], scales [I] */
+    qrx_mat up;     /* [I][H*b/8], scales [I] */
+    qrx_mat down;   /* [H][I*b/8], scales [H] */
 } qrx_experts;
 
 /* Batch-union permutation buffers (device, int32):
@@ -247,6 +264,27 @@ int qrx_expert_down(const qrx_cfg *cfg, const qrx_experts *routed, const qrx_per
                     const float *h_sorted, int32_t T, float *y_sorted, void *ws,
                     size_t ws_bytes, void *stream);
 
+/* The exact int32 accumulators of the Q8_0 path, for checking them bit for
+ * bit (README "已实现的功能": Q8_0-style int8-activation integer dot kernels;
+ * blocks of 32 codes with one f32 scale each).  These run the routed FFN's own
+ * decode kernels (calls of T <= 4 tokens, cfg->afmt == QRX_A_Q8_0; otherwise
+ * QRX_EUNSUPPORTED) with one more store: every 32-block's accumulator
+ * acc_b = sum of code(row, i) * q8(act)[i] over the block, exactly as the
+ * kernel forms it before scaling it by the block's d_b.
+ *   qrx_expert_gateup_q8_sums: the gate/up stage of qrx_expert_ffn on act;
+ *     h_sorted [T*k][I] f32 output; acc [T*k][2][I][H/32] int32 (gate rows,
+ *     then up rows) for every routed position.
+ *   qrx_expert_down_q8_sums: the down stage of qrx_expert_down on a given
+ *     h_sorted [T*k][I] f32, which the kernel re-quantises to Q8_0 as the
+ *     layer does; y_sorted [T*k][H] f32 output; acc [T*k][H][I/32] int32.
+ * ws: at least qrx_workspace_bytes(cfg, T) bytes. */
+int qrx_expert_gateup_q8_sums(const qrx_cfg *cfg, const qrx_experts *routed, const qrx_perm *perm,
+                              const qrx_act *act, int32_t T, float *h_sorted, int32_t *acc,
+                              void *ws, size_t ws_bytes, void *stream);
+int qrx_expert_down_q8_sums(const qrx_cfg *cfg, const qrx_experts *routed, const qrx_perm *perm,
+                            const float *h_sorted, int32_t T, float *y_sorted, int32_t *acc,
+                            void *ws, size_t ws_bytes, void *stream);
+
 /* Shared expert (README "已实现的功能"): the same FFN on every token, weight
  * 1, ungated.  h_sh [T][I] (may be NULL), y_sh [T][H] f32. */
 int qrx_shared_ffn(const qrx_cfg *cfg, const qrx_experts *shared, const qrx_act *act,
@@ -276,9 +314,12 @@ int qrx_combine(const qrx_cfg *cfg, const float *y_sorted, const float *y_sh,
  *     k = 8) that is T <= 58 with f32 or bf16 activations.  Larger T returns
  *     QRX_ENOSPACE before any launch.
  *   - The array is a file-scope device variable: every GPU that loads the
- *     library holds its 8 MiB until the process exits.  The first call on a
- *     device looks up the array's device address (cudaGetSymbolAddress) with
- *     that device current; make that first call before any stream capture.
+ *     library holds its 8 MiB until the process exits.  Every call looks up
+ *     the array's device address in the current device's context
+ *     (cudaGetSymbolAddress, which allocates nothing), so the address stays
+ *     right after cudaDeviceReset or in another context.  The first call on a
+ *     device may load the library's kernels into that device's context: make
+ *     it before any stream capture.
  *   - The array is shared by all calls on a device and keeps the last call's
  *     contents; nothing in it needs clearing, because every record and every
  *     row of h that a kernel reads is written by the same call first.  Calls

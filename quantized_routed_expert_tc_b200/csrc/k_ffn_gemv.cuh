@@ -28,8 +28,10 @@
 // only by the per-stage partial sums (64 tokens at the GLM shape), so each
 // expert's weights stream once per call at decode batch sizes.  Reductions
 // are fixed-order (warp butterflies, then warp partials in index order), so
-// results are deterministic.  For gate/up the matrix rows are interleaved
-// (gate row i, up row i) so the SwiGLU is applied where both sums meet.
+// results are deterministic.  For gate/up a block holds rows of the gate
+// matrix and the same rows of the up matrix (two copies into one stage), so
+// the SwiGLU is applied where both sums meet.  Calls of more than four tokens
+// use this engine; k_gemv2.cuh takes decode calls of up to four.
 #pragma once
 #include <atomic>
 #include <cuda/atomic>
@@ -261,15 +263,18 @@ __host__ __device__ inline GvSmem gv_smem(int stages, int ts, int rb, int tpc, i
 }
 
 struct GemvP {
-    int K, rows, row_bytes, cpr, tpc, rb, nblk, ts, wpt, stages, maxslots, nthreads;
+    int K, rows, row_bytes, cpr, tpc, rb, rbm, nblk, ts, wpt, stages, maxslots, nthreads;
     RecLayout rec;
     GvSmem sm;
-    const uint8_t *w;
-    int64_t w_stride;        // bytes between experts' matrices
-    const float *s;
-    int64_t s_stride;        // floats between experts' scale vectors
-    const uint8_t *w_sh;
-    const float *s_sh;
+    // matrix m of expert e: codes w[m] + e*w_stride[m] bytes, scales s[m] +
+    // e*s_stride[m] floats; gate/up: m = 0 gate, 1 up (rbm rows of each per
+    // block, gate rows first); down: m = 0 only (rbm = rb)
+    const uint8_t *w[2];
+    int64_t w_stride[2];
+    const float *s[2];
+    int64_t s_stride[2];
+    const uint8_t *w_sh[2];
+    const float *s_sh[2];
     int routed, shared;
     const int32_t *offsets, *sorted, *union_ids, *n_union;
     int E, k, T;
@@ -434,8 +439,8 @@ struct Units {
     int s, j, ntok, nt;
     int64_t b, bend;
     bool valid;
-    const uint8_t *W;        // the slot's weights and row scales, looked up once per slot
-    const float *S;
+    const uint8_t *W[2];     // the slot's weights and row scales, looked up once per slot
+    const float *S[2];
 };
 
 __device__ __forceinline__ int slot_ntok(const GemvP &p, int s, int nu)
@@ -447,8 +452,8 @@ __device__ __forceinline__ int slot_ntok(const GemvP &p, int s, int nu)
     return p.T;
 }
 
-__device__ __forceinline__ const uint8_t *slot_weights(const GemvP &p, int s, int nu);
-__device__ __forceinline__ const float *slot_scales(const GemvP &p, int s, int nu);
+__device__ __forceinline__ const uint8_t *slot_weights(const GemvP &p, int s, int nu, int m);
+__device__ __forceinline__ const float *slot_scales(const GemvP &p, int s, int nu, int m);
 
 // Enter slot s: token count and the slot's weight / scale base pointers.
 __device__ __forceinline__ void units_enter_slot(Units &u, const GemvP &p, int s)
@@ -457,8 +462,10 @@ __device__ __forceinline__ void units_enter_slot(Units &u, const GemvP &p, int s
     u.j = -1;
     if (s < u.nslots) {
         u.ntok = slot_ntok(p, s, u.nu);
-        u.W = slot_weights(p, s, u.nu);
-        u.S = slot_scales(p, s, u.nu);
+        u.W[0] = slot_weights(p, s, u.nu, 0);
+        u.S[0] = slot_scales(p, s, u.nu, 0);
+        u.W[1] = slot_weights(p, s, u.nu, 1);
+        u.S[1] = slot_scales(p, s, u.nu, 1);
     }
 }
 
@@ -489,24 +496,24 @@ __device__ void units_advance(Units &u, const GemvP &p)
     }
 }
 
-__device__ __forceinline__ const float *slot_scales(const GemvP &p, int s, int nu)
+__device__ __forceinline__ const float *slot_scales(const GemvP &p, int s, int nu, int m)
 {
     if (s < nu) {
         int e = p.union_ids[s];
         e = (e >= 0 && e < p.E) ? e : 0;
-        return p.s + (int64_t)e * p.s_stride;
+        return (m ? p.s[1] : p.s[0]) + (int64_t)e * (m ? p.s_stride[1] : p.s_stride[0]);
     }
-    return p.s_sh;
+    return m ? p.s_sh[1] : p.s_sh[0];
 }
 
-__device__ __forceinline__ const uint8_t *slot_weights(const GemvP &p, int s, int nu)
+__device__ __forceinline__ const uint8_t *slot_weights(const GemvP &p, int s, int nu, int m)
 {
     if (s < nu) {
         int e = p.union_ids[s];
         e = (e >= 0 && e < p.E) ? e : 0;     // a bad index was flagged when the slot was costed
-        return p.w + (int64_t)e * p.w_stride;
+        return (m ? p.w[1] : p.w[0]) + (int64_t)e * (m ? p.w_stride[1] : p.w_stride[0]);
     }
-    return p.w_sh;
+    return m ? p.w_sh[1] : p.w_sh[0];
 }
 
 template <int WB, int NDIG, int TP, bool GATEUP>
@@ -596,8 +603,8 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
         cu.s = lo;
     }
     cu.ntok = 0;
-    cu.W = nullptr;
-    cu.S = nullptr;
+    cu.W[0] = cu.W[1] = nullptr;
+    cu.S[0] = cu.S[1] = nullptr;
     units_enter_slot(cu, p, cu.s);
     cu.nt = 0;
     cu.b = cu.bend = 0;
@@ -607,20 +614,23 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
     // Every thread keeps a producer iterator `stages` units ahead of its own
     // consumer iterator; the last warp to finish unit n refills its stage with
     // unit n + stages.  Thread 0 issues the first `stages` units.
+    // A block holds rbm rows of each matrix: gate rows, then the same up rows.
     auto issue = [&](const Units &u, int stage) {
-        const int64_t row0 = u.b * (int64_t)p.rb;
-        const int64_t nrows = min((int64_t)p.rb, (int64_t)p.rows - row0);
-        const uint8_t *src = u.W + row0 * p.row_bytes;
-        const float *ssrc = u.S + row0;
+        constexpr int NMAT = GATEUP ? 2 : 1;
+        const int64_t row0 = u.b * (int64_t)p.rbm;
+        const int64_t nrows = min((int64_t)p.rbm, (int64_t)p.rows - row0);
         unsigned char *dst = ring + (size_t)stage * M.stage_bytes;
         const uint32_t mb = smem_u32(&mbar[stage]);
         const uint32_t wbytes = (uint32_t)(nrows * p.row_bytes), sbytes = (uint32_t)(nrows * 4);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb),
-                     "r"(wbytes + sbytes)
+                     "r"(NMAT * (wbytes + sbytes))
                      : "memory");
-        bulk_copy(smem_u32(dst), src, wbytes, mb);
-        bulk_copy(smem_u32(dst + M.scales_off), ssrc, sbytes, mb);
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+            bulk_copy(smem_u32(dst + (size_t)m * p.rbm * p.row_bytes), u.W[m] + row0 * p.row_bytes, wbytes, mb);
+            bulk_copy(smem_u32(dst + M.scales_off + m * p.rbm * 4), u.S[m] + row0, sbytes, mb);
+        }
     };
     Units pu = cu;
     for (int st = 0; st < p.stages && pu.valid; ++st) {
@@ -753,23 +763,23 @@ __global__ void __launch_bounds__(GvShape<WB, NDIG>::NT, 1) k_ffn_gemv(const Gem
             const float *scl = reinterpret_cast<const float *>(sbase + M.scales_off);
             const int rblk = (int)cu.b;
             if constexpr (GATEUP) {
-                const int per = p.tpc * (R / 2);
-                for (int f = lane; f < nt * per; f += 32) {
-                    const int t = f / per, rem = f % per;
-                    const int tf = rem / (R / 2), q = rem % (R / 2);
-                    const int lrow = tf * R + 2 * q;
-                    const int row_g = rblk * p.rb + lrow;
-                    if (row_g >= p.rows) continue;
-                    const float *src = rst + ((t * p.tpc + tf) * p.wpt) * R;
+                // gate row q of the block is local row q, its up row is local row rbm + q
+                const int rbm = p.rbm;
+                for (int f = lane; f < nt * rbm; f += 32) {
+                    const int t = f / rbm, q = f % rbm;
+                    const int row = rblk * rbm + q;
+                    if (row >= p.rows) continue;
+                    const int gl = q, ul = q + rbm;
+                    const float *gsrc = rst + ((t * p.tpc + gl / R) * p.wpt) * R + gl % R;
+                    const float *usrc = rst + ((t * p.tpc + ul / R) * p.wpt) * R + ul % R;
                     float G = 0.f, U = 0.f;
                     for (int w2 = 0; w2 < p.wpt; ++w2) {
-                        G += src[w2 * R + 2 * q];
-                        U += src[w2 * R + 2 * q + 1];
+                        G += gsrc[w2 * R];
+                        U += usrc[w2 * R];
                     }
                     const int orow = TP == 1 ? tout1 : row_out_of(tg + t);
                     QRX_CHECK_OR(orow >= 0 && orow < n_out, continue);
-                    p.out[(int64_t)orow * p.out_ld + (row_g >> 1)] =
-                        silu_mul(scl[lrow] * G, scl[lrow + 1] * U);
+                    p.out[(int64_t)orow * p.out_ld + row] = silu_mul(scl[gl] * G, scl[ul] * U);
                 }
             } else {
                 const int per = p.tpc * R;
@@ -813,7 +823,7 @@ struct GemvPlan {
 // Geometry for a matrix of `rows` x `K` codes at `wbits`, slots of at most
 // `maxtok` tokens, NDIG digit planes.  Picks the deepest weight ring and the
 // largest token group that fit in shared memory.
-static inline bool gemv_plan(GemvPlan &pl, int wbits, int ndig, int K, int rows, int maxtok,
+static inline bool gemv_plan(GemvPlan &pl, int wbits, int ndig, int K, int rows, int nm, int maxtok,
                              int maxslots)
 {
     GemvP &p = pl.p;
@@ -829,7 +839,8 @@ static inline bool gemv_plan(GemvPlan &pl, int wbits, int ndig, int K, int rows,
     if (p.cpr > 32 && (p.cpr % 32) != 0) return false;
     p.tpc = NT / p.cpr;
     p.rb = p.tpc * R;
-    p.nblk = (rows + p.rb - 1) / p.rb;
+    p.rbm = nm == 2 ? p.rb / 2 : p.rb;        // rows of each matrix per block
+    p.nblk = (rows + p.rbm - 1) / p.rbm;
     p.wpt = p.cpr >= 32 ? p.cpr / 32 : 1;
     if (p.rb * 4 % 16 != 0) return false;
     pl.tp = maxtok <= 1 ? 1 : (ndig == 1 ? 4 : 2);
@@ -922,21 +933,28 @@ cudaError_t launch_act_digits(const FfnArgs &a, cudaStream_t st)
 cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
 {
     if (ffn_use_tc(a)) return launch_ffn_tc_gateup(a, num_sms, st);
+    if (g2_use(a)) return launch_g2_gateup(a, num_sms, st);
     const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
     GemvPlan pl;
-    if (!gemv_plan(pl, a.wbits, ndig, a.H, 2 * a.I, a.T, a.E + 1)) return cudaErrorInvalidValue;
+    if (!gemv_plan(pl, a.wbits, ndig, a.H, a.I, 2, a.T, a.E + 1)) return cudaErrorInvalidValue;
     if (a.prep_records) {
         const cudaError_t err = launch_act_digits(a, st);
         if (err != cudaSuccess) return err;
     }
     GemvP &p = pl.p;
     gemv_common(p, a);
-    p.w = a.w13;
-    p.w_stride = (int64_t)2 * a.I * p.row_bytes;
-    p.s = a.s13;
-    p.s_stride = (int64_t)2 * a.I;
-    p.w_sh = a.w13_sh;
-    p.s_sh = a.s13_sh;
+    p.w[0] = a.gate.q;
+    p.w[1] = a.up.q;
+    p.w_stride[0] = a.gate.sq;
+    p.w_stride[1] = a.up.sq;
+    p.s[0] = a.gate.s;
+    p.s[1] = a.up.s;
+    p.s_stride[0] = a.gate.ss;
+    p.s_stride[1] = a.up.ss;
+    p.w_sh[0] = a.gate_sh.q;
+    p.w_sh[1] = a.up_sh.q;
+    p.s_sh[0] = a.gate_sh.s;
+    p.s_sh[1] = a.up_sh.s;
     p.xrec = a.xrec;
     p.sh_in_row0 = 0;
     p.out = a.h;
@@ -948,17 +966,18 @@ cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
 cudaError_t launch_ffn_down(const FfnArgs &a, int num_sms, cudaStream_t st)
 {
     if (ffn_use_tc(a)) return launch_ffn_tc_down(a, num_sms, st);
+    if (g2_use(a)) return launch_g2_down(a, num_sms, st);
     const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
     GemvPlan pl;
-    if (!gemv_plan(pl, a.wbits, ndig, a.I, a.H, a.T, a.E + 1)) return cudaErrorInvalidValue;
+    if (!gemv_plan(pl, a.wbits, ndig, a.I, a.H, 1, a.T, a.E + 1)) return cudaErrorInvalidValue;
     GemvP &p = pl.p;
     gemv_common(p, a);
-    p.w = a.w2;
-    p.w_stride = (int64_t)a.H * p.row_bytes;
-    p.s = a.s2;
-    p.s_stride = a.H;
-    p.w_sh = a.w2_sh;
-    p.s_sh = a.s2_sh;
+    p.w[0] = p.w[1] = a.down.q;
+    p.w_stride[0] = p.w_stride[1] = a.down.sq;
+    p.s[0] = p.s[1] = a.down.s;
+    p.s_stride[0] = p.s_stride[1] = a.down.ss;
+    p.w_sh[0] = p.w_sh[1] = a.down_sh.q;
+    p.s_sh[0] = p.s_sh[1] = a.down_sh.s;
     // h rows -> digit records (all rows the down projection reads)
     const int hrows = max(a.routed ? a.T * a.k : 0, a.shared ? (int)a.sh_h_row0 + a.T : 0);
     {

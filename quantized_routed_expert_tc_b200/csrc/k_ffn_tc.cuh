@@ -10,8 +10,9 @@
 // the per-row scale multiplies the accumulator in the epilogue.
 //
 // Tiles.  A work item is (slot, 256 weight rows, up to 128 tokens): the
-// weights are the MMA's M side (two M=128 halves sharing one B tile) and the
-// tokens its N side; K advances in stages of 64 (one 128-byte swizzle atom of
+// weights are the MMA's M side (two M=128 halves sharing one B tile: for
+// gate/up 128 rows of the gate matrix and the same 128 rows of the up matrix,
+// for down 256 consecutive rows) and the tokens its N side; K advances in stages of 64 (one 128-byte swizzle atom of
 // bf16).  B is always a run of consecutive rows of one bf16 matrix: for
 // gate/up the tokens gathered into expert order by k_gather_x, for down the
 // rows of h that gate/up wrote in the same order.  Roles per CTA (one CTA per
@@ -94,10 +95,11 @@ __host__ __device__ constexpr int tc_perm(int p) { return (p & 1) ? 4 + (p >> 1)
 __host__ __device__ constexpr int tc_inv_perm(int e) { return e < 4 ? 2 * e : 2 * (e - 4) + 1; }
 
 struct TcP {
-    int rows, K, mtiles, kstages;
-    const float *s;         // routed row scales, expert stride s_stride
-    int64_t s_stride;
-    const float *s_sh;
+    int rows, K, mtiles, kstages;     // rows per matrix (gate/up: I, down: H)
+    int half_rows;                    // row offset of half 1 within an item (gate/up: 0, down: 128)
+    const float *s[2];                // routed row scales of half 0 / 1's matrix, expert stride s_stride
+    int64_t s_stride[2];
+    const float *s_sh[2];
     int routed, shared, E, k, T;
     const int32_t *offsets, *union_ids, *n_union;
     int64_t b_sh_row0;           // B row of the shared expert's first token
@@ -287,8 +289,16 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t *bar, uint32_t parity, vol
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// First weight row of half `hf` of row tile mt (gate/up: both halves start at
+// mt*128 of their own matrix; down: mt*256 and mt*256 + 128 of one matrix).
+__device__ __forceinline__ int tc_row0(const TcP &p, int mt, int hf)
+{
+    return p.half_rows ? mt * TC_M + hf * TC_HALF : mt * TC_HALF;
+}
+
 __global__ void __launch_bounds__(TC_THREADS, 1)
-    k_ffn_tc(const __grid_constant__ CUtensorMap mw, const __grid_constant__ CUtensorMap mwsh,
+    k_ffn_tc(const __grid_constant__ CUtensorMap mw0, const __grid_constant__ CUtensorMap mw1,
+             const __grid_constant__ CUtensorMap msh0, const __grid_constant__ CUtensorMap msh1,
              const __grid_constant__ CUtensorMap mb, const TcP p)
 {
     extern __shared__ __align__(1024) unsigned char tsm_raw[];
@@ -379,10 +389,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             if (pf_it < nitems) pf_d = tc_decode(p, pre, nslots, nu, pf_it);
             auto pf_step = [&]() {
                 if (pf_it >= nitems) return;
-                const CUtensorMap *m = pf_d.routed ? &mw : &mwsh;
                 const int zz = pf_d.routed ? pf_d.e : 0;
-                tma_prefetch_3d(m, pf_kr * 128, pf_d.mt * TC_M, zz);
-                tma_prefetch_3d(m, pf_kr * 128, pf_d.mt * TC_M + TC_HALF, zz);
+                tma_prefetch_3d(pf_d.routed ? &mw0 : &msh0, pf_kr * 128, tc_row0(p, pf_d.mt, 0), zz);
+                tma_prefetch_3d(pf_d.routed ? &mw1 : &msh1, pf_kr * 128, tc_row0(p, pf_d.mt, 1), zz);
                 if (++pf_kr == kraw) {
                     pf_kr = 0;
                     pf_it += gridDim.x;
@@ -392,7 +401,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int i = 0; i < TC_PF; ++i) pf_step();
             for (int64_t it = blockIdx.x; ok && it < nitems && !*abort_flag; it += gridDim.x) {
                 const TcItem d = tc_decode(p, pre, nslots, nu, it);
-                const CUtensorMap *wm = d.routed ? &mw : &mwsh;
+                const CUtensorMap *wm0 = d.routed ? &mw0 : &msh0;
+                const CUtensorMap *wm1 = d.routed ? &mw1 : &msh1;
                 const int z = d.routed ? d.e : 0;
                 const int nbox = (d.nn + TC_BOX_ROWS - 1) / TC_BOX_ROWS;
                 for (int kb = 0; kb < p.kstages; ++kb) {
@@ -406,8 +416,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         const uint32_t dst = smem_u32(sR + rs * TC_RAW_BYTES);
                         const uint32_t bar = smem_u32(&raw_full[(rs) * TC_BS]);
                         mbar_expect(bar, TC_RAW_BYTES);
-                        tma_load_3d(dst, wm, (kb / TC_RK) * 128, d.mt * TC_M, z, bar);
-                        tma_load_3d(dst + TC_RAW_BYTES / 2, wm, (kb / TC_RK) * 128, d.mt * TC_M + TC_HALF, z,
+                        tma_load_3d(dst, wm0, (kb / TC_RK) * 128, tc_row0(p, d.mt, 0), z, bar);
+                        tma_load_3d(dst + TC_RAW_BYTES / 2, wm1, (kb / TC_RK) * 128, tc_row0(p, d.mt, 1), z,
                                     bar);
                         ++rg;
                     }
@@ -498,53 +508,66 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         int local = 0;
         for (int64_t it = blockIdx.x; it < nitems && !*abort_flag; it += gridDim.x, ++local) {
             const TcItem d = tc_decode(p, pre, nslots, nu, it);
-            const float *sc_base = d.routed ? p.s + (int64_t)d.e * p.s_stride : p.s_sh;
-            const int row0 = d.mt * TC_M + q4 * 32 + lane;           // row of half 0
-            const float sc0 = sc_base[row0], sc1 = sc_base[row0 + TC_HALF];
+            // this thread's row of each half, and that row's scale
+            const int r0 = tc_row0(p, d.mt, 0) + q4 * 32 + lane, r1 = tc_row0(p, d.mt, 1) + q4 * 32 + lane;
+            const float *sb0 = d.routed ? p.s[0] + (int64_t)d.e * p.s_stride[0] : p.s_sh[0];
+            const float *sb1 = d.routed ? p.s[1] + (int64_t)d.e * p.s_stride[1] : p.s_sh[1];
+            const float sc0 = sb0[r0], sc1 = sb1[r1];
             const int64_t orow0 = d.routed ? d.b0 : p.sh_out_row0 + d.n0;
             const int a = local & 1;
             if (!tc_wait_warp(&acc_full[(a) * TC_BS], (local >> 1) & 1, abort_flag, 256)) break;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-#pragma unroll 1
-            for (int hf = 0; hf < 2; ++hf) {
-                const int rowg = row0 + hf * TC_HALF;
-                const float sc = hf ? sc1 : sc0;
+            // 32 accumulator columns (tokens c0..c0+31) of half hf for this thread's row
+            auto ld32 = [&](int hf, int c0, uint32_t (&v)[32]) {
+                const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) +
+                                       (uint32_t)(a * 2 * TC_NMAX + hf * TC_NMAX + c0);
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+                    "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                      "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+                      "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+                      "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+                      "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+                      "=r"(v[31])
+                    : "r"(taddr));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            };
+            if (p.gateup) {
+                // half 0 holds gate row r0, half 1 the up row of the same index
 #pragma unroll 1
                 for (int c0 = 0; c0 < d.nn; c0 += 32) {
-                    uint32_t v[32];
-                    const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) +
-                                           (uint32_t)(a * 2 * TC_NMAX + hf * TC_NMAX + c0);
-                    asm volatile(
-                        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-                        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-                        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-                          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
-                          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-                          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
-                          "=r"(v[31])
-                        : "r"(taddr));
-                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    uint32_t vg[32], vu[32];
+                    ld32(0, c0, vg);
+                    ld32(1, c0, vu);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int n = c0 + j;
-                        const float acc = sc * __uint_as_float(v[j]);
+                        if (n >= d.nv) continue;
                         const int64_t orow = orow0 + n;
-                        if (p.gateup) {
-                            // gate on even rows, up on the odd row after it
-                            const float other = __shfl_xor_sync(0xffffffffu, acc, 1);
-                            if ((lane & 1) || n >= d.nv) continue;
-                            QRX_CHECK_OR(orow >= 0 && orow < n_out, continue);
-                            const int pair = rowg >> 1;
-                            const float h = silu_mul(acc, other);
-                            if (p.out) p.out[orow * p.out_ld + pair] = h;
-                            if (p.hperm)
-                                p.hperm[orow * (p.rows / 2) + (pair & ~7) + tc_inv_perm(pair & 7)] =
-                                    __float2bfloat16_rn(h);
-                        } else {
+                        QRX_CHECK_OR(orow >= 0 && orow < n_out, continue);
+                        const float h = silu_mul(sc0 * __uint_as_float(vg[j]), sc1 * __uint_as_float(vu[j]));
+                        if (p.out) p.out[orow * p.out_ld + r0] = h;
+                        if (p.hperm)
+                            p.hperm[orow * p.rows + (r0 & ~7) + tc_inv_perm(r0 & 7)] = __float2bfloat16_rn(h);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int rowg = hf ? r1 : r0;
+                    const float sc = hf ? sc1 : sc0;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < d.nn; c0 += 32) {
+                        uint32_t v[32];
+                        ld32(hf, c0, v);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int n = c0 + j;
                             if (n >= d.nv) continue;
+                            const int64_t orow = orow0 + n;
                             QRX_CHECK_OR(orow >= 0 && orow < n_out, continue);
-                            p.out[orow * p.out_ld + rowg] = acc;
+                            p.out[orow * p.out_ld + rowg] = sc * __uint_as_float(v[j]);
                         }
                     }
                 }
@@ -709,7 +732,7 @@ static bool tc_map_rows(CUtensorMap *m, const void *b, int K, int64_t nrows)
 bool tc_shape_ok(int afmt, int wbits, int64_t T, int64_t H, int64_t I)
 {
     return afmt == QRX_A_BF16 && wbits == 4 && T >= TC_MIN_T && H % (TC_BK * TC_RK) == 0 &&
-           I % (TC_BK * TC_RK) == 0 && H % TC_M == 0 && (2 * I) % TC_M == 0 && tc_encode_fn() != nullptr;
+           I % (TC_BK * TC_RK) == 0 && H % TC_M == 0 && I % TC_HALF == 0 && tc_encode_fn() != nullptr;
 }
 
 bool ffn_use_tc(const FfnArgs &a)
@@ -717,18 +740,33 @@ bool ffn_use_tc(const FfnArgs &a)
     return tc_shape_ok(a.afmt, a.wbits, a.T, a.H, a.I) && a.xperm && a.hperm;
 }
 
-static cudaError_t tc_go(TcP &p, const void *w, const void *w_sh, int64_t w_stride, const void *b,
-                         int64_t brows, int num_sms, cudaStream_t st, int maxslots)
+// Weight maps: half 0 / 1 of every item read routed matrices m0 / m1 (gate and
+// up, or down twice) and the shared expert's sh0 / sh1.
+static cudaError_t tc_go(TcP &p, const MatRef &m0, const MatRef &m1, const MatRef &sh0, const MatRef &sh1,
+                         const void *b, int64_t brows, int num_sms, cudaStream_t st, int maxslots)
 {
-    p.mtiles = p.rows / TC_M;
+    p.mtiles = p.half_rows ? p.rows / TC_M : p.rows / TC_HALF;
     p.kstages = p.K / TC_BK;
     const int row_bytes = p.K / 2;
-    CUtensorMap mw{}, mwsh{}, mb{};      // zeroed: a launch without one expert set leaves its map unused
+    // zeroed: a launch without one expert set leaves its maps unused
+    CUtensorMap mw0{}, mw1{}, msh0{}, msh1{}, mb{};
     bool ok = true;
-    if (p.routed) ok = ok && tc_map_weights(&mw, w, row_bytes, p.rows, p.E, w_stride);
-    if (p.shared) ok = ok && tc_map_weights(&mwsh, w_sh, row_bytes, p.rows, 1, (int64_t)p.rows * row_bytes);
-    if (!p.routed) mw = mwsh;
-    if (!p.shared) mwsh = mw;
+    if (p.routed) {
+        ok = ok && tc_map_weights(&mw0, m0.q, row_bytes, p.rows, p.E, m0.sq);
+        ok = ok && tc_map_weights(&mw1, m1.q, row_bytes, p.rows, p.E, m1.sq);
+    }
+    if (p.shared) {
+        ok = ok && tc_map_weights(&msh0, sh0.q, row_bytes, p.rows, 1, (int64_t)p.rows * row_bytes);
+        ok = ok && tc_map_weights(&msh1, sh1.q, row_bytes, p.rows, 1, (int64_t)p.rows * row_bytes);
+    }
+    if (!p.routed) {
+        mw0 = msh0;
+        mw1 = msh1;
+    }
+    if (!p.shared) {
+        msh0 = mw0;
+        msh1 = mw1;
+    }
     ok = ok && tc_map_rows(&mb, b, p.K, brows);
     if (!ok) return cudaErrorInvalidValue;
     const int smem = tc_smem_bytes(maxslots);
@@ -742,7 +780,7 @@ static cudaError_t tc_go(TcP &p, const void *w, const void *w_sh, int64_t w_stri
         if (err != cudaSuccess) return err;
         if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_release);
     }
-    return launch_k(k_ffn_tc, dim3(num_sms), dim3(TC_THREADS), (size_t)smem, st, mw, mwsh, mb, p);
+    return launch_k(k_ffn_tc, dim3(num_sms), dim3(TC_THREADS), (size_t)smem, st, mw0, mw1, msh0, msh1, mb, p);
 }
 
 static void tc_common(TcP &p, const FfnArgs &a)
@@ -769,18 +807,22 @@ cudaError_t launch_ffn_tc_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
     if (err != cudaSuccess) return err;
     TcP p{};
     tc_common(p, a);
-    p.rows = 2 * a.I;
+    p.rows = a.I;
+    p.half_rows = 0;
     p.K = a.H;
-    p.s = a.s13;
-    p.s_stride = 2 * a.I;
-    p.s_sh = a.s13_sh;
+    p.s[0] = a.gate.s;
+    p.s[1] = a.up.s;
+    p.s_stride[0] = a.gate.ss;
+    p.s_stride[1] = a.up.ss;
+    p.s_sh[0] = a.gate_sh.s;
+    p.s_sh[1] = a.up_sh.s;
     p.b_sh_row0 = A;
     p.out = a.h;
     p.out_ld = a.h_ld;
     p.sh_out_row0 = a.sh_h_row0;
     p.hperm = static_cast<__nv_bfloat16 *>(a.hperm);
     p.gateup = 1;
-    return tc_go(p, a.w13, a.w13_sh, (int64_t)2 * a.I * (a.H / 2), xs, rows, num_sms, st, a.E + 1);
+    return tc_go(p, a.gate, a.up, a.gate_sh, a.up_sh, xs, rows, num_sms, st, a.E + 1);
 }
 
 cudaError_t launch_ffn_tc_down(const FfnArgs &a, int num_sms, cudaStream_t st)
@@ -798,17 +840,18 @@ cudaError_t launch_ffn_tc_down(const FfnArgs &a, int num_sms, cudaStream_t st)
     TcP p{};
     tc_common(p, a);
     p.rows = a.H;
+    p.half_rows = TC_HALF;
     p.K = a.I;
-    p.s = a.s2;
-    p.s_stride = a.H;
-    p.s_sh = a.s2_sh;
+    p.s[0] = p.s[1] = a.down.s;
+    p.s_stride[0] = p.s_stride[1] = a.down.ss;
+    p.s_sh[0] = p.s_sh[1] = a.down_sh.s;
     p.b_sh_row0 = a.sh_h_row0;
     p.out = a.y;
     p.out_ld = a.y_ld;
     p.sh_out_row0 = a.sh_y_row0;
     p.hperm = nullptr;
     p.gateup = 0;
-    return tc_go(p, a.w2, a.w2_sh, (int64_t)a.H * (a.I / 2), hperm, rows, num_sms, st, a.E + 1);
+    return tc_go(p, a.down, a.down, a.down_sh, a.down_sh, hperm, rows, num_sms, st, a.E + 1);
 }
 
 }  // namespace qrx

@@ -1,0 +1,1067 @@
+// k_gemv2.cuh -- decode-shaped expert FFN: at most four tokens per expert
+// (calls of T <= 4 tokens), streamed from HBM at close to its bandwidth.
+//
+// README "JustVugg/colibri", section "已实现的功能": the batch-union MoE (each
+// unique expert of a batch read once and applied to all positions routed to
+// it), int8 / packed int4 / packed int2 weights with per-row scales
+// dequantised on use, Q8_0-style int8-activation integer dots; blog "GLM-5.2
+// on slow computers", section "核心技巧": a token costs the expert bytes it
+// reads.  The expert is a SwiGLU FFN: h = silu(s_g Q_g x) * (s_u Q_u x), then
+// y = s_d Q_d h.
+//
+// Work.  A unit is (slot, block of RB rows): a slot is one expert of the
+// union (or the shared expert) with its tokens; for gate/up a unit holds RB
+// gate rows and the same RB up rows, so the SwiGLU is applied where both sums
+// meet.  Units are cut into contiguous ranges of equal estimated cost, one
+// range per CTA, one CTA per SM.  A unit streams through the CTA as K-slices
+// of G2_KS bytes per row: each slice is one stage of a shared-memory ring.
+//
+// Roles.  Warp 8 is the producer: for each slice one thread issues one tiled
+// TMA copy per matrix (the slice of all the unit's rows; and, on a unit's last
+// slice, a bulk copy of the row scales) onto the stage's "full" mbarrier,
+// after the stage's "empty" mbarrier says that all compute warps left it.  Warps 0..7 compute: warp w owns rows
+// [w*RW, (w+1)*RW) of every unit; LPR lanes cover one row's chunks of a slice
+// (lane c reads 16-byte chunk c), so the rows a lane owns accumulate across
+// the slices of the unit in registers, and a unit ends with one transposed
+// warp butterfly -- no partial sums cross warps, no finaliser.
+//
+// Activations.  Every input row (a token of x for gate/up, a row of h for
+// down) is turned into a "record" in shared memory by the compute warps: NDIG
+// digit planes of signed bytes in the order the unpacked weight words use, so
+// each dot of 4 codes by 4 digits is one dp4a with an exact int32 sum.
+//   NDIG = 3 (f32, bf16 inputs): one power-of-two scale per row, sigma =
+//     2^-s with max|x| * 2^s in [2^21, 2^22), and x*2^s rounded to an integer
+//     split into three balanced bytes (x ~= sigma (d0 + 2^8 d1 + 2^16 d2),
+//     error <= 2^-22 of the row's largest magnitude).  The int32 sums of a
+//     lane run over all of its chunks; the planes are combined once per unit.
+//   NDIG = 1 (Q8_0): the record holds the Q8_0 codes and per-block scales d_b
+//     (README: Q8_0-style int8 activations, blocks of 32 with an f32 absmax
+//     scale); every 32-block's int32 accumulator is exact and is scaled by d_b
+//     in f32.
+// Packed int4 / int2 fields are flipped to offset binary (code + 8, code + 2)
+// by the unpack; the offset is removed through the digit sums (per block for
+// Q8_0, per lane and row for NDIG = 3), so every integer sum is exact.
+#pragma once
+#include "qrx_dev.cuh"
+#include "qrx_check.cuh"
+
+namespace qrx {
+
+constexpr int G2_NW = 8;                          // compute warps
+constexpr int G2_THREADS = 32 * (G2_NW + 1);      // + the producer warp
+constexpr int G2_KS = 512;                        // bytes of a row per stage (at most)
+constexpr int G2_TMAX = 4;                        // tokens per call
+constexpr int G2_SMEM_MAX = 227 * 1024;
+constexpr long long G2_WAIT_CAP = 1ll << 22;      // polls before a wait gives up
+
+// ---------------------------------------------------------------- records
+// Record of one input row of K codes, in shared memory:
+//   digits: piece (pl, q, c) = 16 bytes at ((pl * NQ + q) * cpr + c) * 16: the
+//           q-th group of four digit words of chunk c in plane pl (NQ = DW/4);
+//           lanes reading consecutive chunks read consecutive 16-byte pieces
+//   NDIG = 3: then float sigma, int D[3] (unused slot) -- 16 bytes
+//   NDIG = 1: then float d[K/32] (block scales), int corr[K/32]
+//             (corr_b = -OFF * sum of the block's codes)
+struct G2Rec {
+    int hdr, bytes;
+};
+__host__ __device__ inline G2Rec g2_rec(int ndig, int K)
+{
+    G2Rec r;
+    r.hdr = ndig * K;
+    r.bytes = r.hdr + (ndig == 3 ? 16 : 2 * (((K / 32) * 4 + 15) & ~15));
+    return r;
+}
+
+// ---------------------------------------------------------------- parameters
+struct G2Mat {
+    const uint8_t *q;      // codes of expert 0, rows of row_bytes
+    const float *s;        // row scales of expert 0
+    int64_t sq, ss;        // expert strides: bytes, floats
+};
+
+struct G2P {
+    int K, rows, row_bytes, cpr;     // codes per input row, rows per matrix, bytes per row, chunks per row
+    int ks, cps, nslice;             // bytes per slice, chunks per slice, slices per row
+    int lpr, gpw, rw, rb, nrb;       // lanes per row, row groups per warp, rows per warp, rows per unit, units per slot
+    int box_rows;                    // rows per TMA box (rb is a whole number of boxes)
+    int stages, stage_bytes, scale_off;
+    int rec_bytes, rec_off, nrec;    // record size, smem offset, records held
+    int bar_off, pre_off, red_off, smem;
+    G2Mat m[2], msh[2];              // gate/up: m[0] gate, m[1] up; down: m[0] down
+    int routed, shared;
+    const int32_t *offsets, *sorted, *union_ids, *n_union;
+    int E, k, T;
+    int afmt;
+    const void *x;                   // gate/up: x [T][K] (f32 or bf16); down: h f32 rows
+    const int8_t *xq;                // gate/up Q8_0: precomputed codes [T][K] (null: quantise x)
+    const float *xd;                 //              and block scales [T][K/32]
+    int64_t in_ld;                   // row stride of x / h (elements)
+    int64_t sh_in_row0;              // down: h row of the shared expert's first token
+    float *out;
+    int64_t out_ld, sh_out_row0;
+    int32_t *probe;                  // Q8_0: int32 block sums [pos][nmat][rows][K/32] (may be null)
+};
+
+// ---------------------------------------------------------------- small helpers
+__device__ __forceinline__ uint32_t g2_smem(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ bool g2_try(uint32_t mbar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(mbar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait; false if it gave up or another role raised the abort flag.
+__device__ __forceinline__ bool g2_wait(uint32_t mbar, uint32_t parity, volatile int *abort_flag)
+{
+    for (long long it = 0; it < G2_WAIT_CAP; ++it) {
+        if (g2_try(mbar, parity)) return true;
+        if ((it & 63) == 63 && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    raise_status(DERR_TIMEOUT);
+    return false;
+}
+
+// Barrier of the compute warps (not the producer): lane 0 of each warp
+// arrives on an mbarrier of G2_NW arrivals and every lane waits, bounded, for
+// the phase.  `ph` is the caller's phase bit.  False if the wait gave up.
+__device__ __forceinline__ bool g2_cbar(uint64_t *bar, uint32_t &ph, volatile int *abort_flag)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(g2_smem(bar));
+    const bool ok = g2_wait(g2_smem(bar), ph, abort_flag);
+    ph ^= 1u;
+    return ok;
+}
+
+// a[i] for a run-time i < N without indexing a register array
+template <int N, typename T>
+__device__ __forceinline__ T g2_pick(const T (&a)[N], int i)
+{
+    T r = a[0];
+#pragma unroll
+    for (int q = 1; q < N; ++q)
+        if (i == q) r = a[q];
+    return r;
+}
+
+// Transposed butterfly over the LPR lanes of a row group.  In: V values per
+// lane.  Out: with V <= LPR, lane c of the group holds the group total of
+// value c / (LPR / V) in v[0]; with V > LPR, it holds those of values
+// c * (V / LPR) + q in v[q], q < V / LPR.
+template <int N>
+__device__ __forceinline__ void g2_tr_step(float *v, int lane, int off)
+{
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+        const float send = up ? v[i] : v[i + N / 2];
+        const float keep = up ? v[i + N / 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+}
+
+template <int N, int OFF>
+__device__ __forceinline__ void g2_tr_rec(float *v, int lane)
+{
+    if constexpr (OFF >= 1) {
+        if constexpr (N > 1) {
+            g2_tr_step<N>(v, lane, OFF);
+            g2_tr_rec<N / 2, OFF / 2>(v, lane);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], OFF);
+            g2_tr_rec<1, OFF / 2>(v, lane);
+        }
+    }
+}
+
+template <int V, int LPR>
+__device__ __forceinline__ void g2_tr_reduce(float (&v)[V], int lane)
+{
+    g2_tr_rec<V, LPR / 2>(v, lane);
+}
+
+// ---------------------------------------------------------------- record builder
+// Build the records of `n` input rows into shared memory with all compute
+// threads (tid < G2_NW * 32).  Row i is row_of(i) of the input (x for gate/up,
+// h for down).  For bf16 activations h is rounded to bf16 here (x is given as
+// bf16).  `scr` is 64 bytes of scratch; `cb`/`ph` the compute barrier.
+// Returns false if a barrier wait gave up.
+template <int WB, int NDIG, typename RowFn>
+__device__ bool g2_build(const G2P &p, unsigned char *recs, int n, RowFn row_of, bool gateup, float *scr,
+                         uint64_t *cb, uint32_t &ph, volatile int *abort_flag)
+{
+    using F = Fmt<WB>;
+    constexpr int DW = F::DW, NQ = DW / 4, EPC = F::EPC;
+    const int tid = threadIdx.x, nth = G2_NW * 32;
+    const int K = p.K, cpr = p.cpr;
+    const G2Rec RL = g2_rec(NDIG, K);
+    const bool bf = p.afmt == QRX_A_BF16;
+    for (int i = 0; i < n; ++i) {
+        const int64_t row = row_of(i);
+        unsigned char *rec = recs + (size_t)i * p.rec_bytes;
+        // element e of the row as the dot sees it
+        auto val = [&](int e) -> float {
+            if (gateup) {
+                if (bf) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.x)[row * p.in_ld + e]);
+                return reinterpret_cast<const float *>(p.x)[row * p.in_ld + e];
+            }
+            const float h = reinterpret_cast<const float *>(p.x)[row * p.in_ld + e];
+            return bf ? __bfloat162float(__float2bfloat16_rn(h)) : h;
+        };
+        if constexpr (NDIG == 3) {
+            // the row's largest magnitude -> shift s (sigma = 2^-s)
+            float am = 0.f;
+            for (int e = tid; e < K; e += nth) am = fmaxf(am, fabsf(val(e)));
+            am = warp_max(am);
+            if ((tid & 31) == 0) scr[tid >> 5] = am;
+            if (!g2_cbar(cb, ph, abort_flag)) return false;
+            am = 0.f;
+#pragma unroll
+            for (int w = 0; w < G2_NW; ++w) am = fmaxf(am, scr[w]);
+            const int sh = am != 0.f ? fixed_shift(am) : 0;
+            const bool fast = sh >= -126 && sh <= 127;
+            const float mul = fast ? __int_as_float((sh + 127) << 23) : 0.f;
+            for (int c = tid; c < cpr; c += nth) {
+                uint32_t wd[3][DW];
+#pragma unroll
+                for (int wi = 0; wi < 4; ++wi)
+#pragma unroll
+                    for (int j = 0; j < F::UPW; ++j) {
+                        uint32_t b0 = 0, b1 = 0, b2 = 0;
+#pragma unroll
+                        for (int by = 0; by < 4; ++by) {
+                            const float v = val(c * EPC + elem_in_chunk<WB>(wi, j, by));
+                            int8_t d0 = 0, d1 = 0, d2 = 0;
+                            if (am != 0.f) split3(__float2int_rn(fast ? __fmul_rn(v, mul) : ldexpf(v, sh)), d0, d1, d2);
+                            b0 |= (uint32_t)(uint8_t)d0 << (8 * by);
+                            b1 |= (uint32_t)(uint8_t)d1 << (8 * by);
+                            b2 |= (uint32_t)(uint8_t)d2 << (8 * by);
+                        }
+                        wd[0][wi * F::UPW + j] = b0;
+                        wd[1][wi * F::UPW + j] = b1;
+                        wd[2][wi * F::UPW + j] = b2;
+                    }
+#pragma unroll
+                for (int pl = 0; pl < 3; ++pl)
+#pragma unroll
+                    for (int q = 0; q < NQ; ++q)
+                        *reinterpret_cast<uint4 *>(rec + ((size_t)(pl * NQ + q) * cpr + c) * 16) =
+                            make_uint4(wd[pl][4 * q], wd[pl][4 * q + 1], wd[pl][4 * q + 2], wd[pl][4 * q + 3]);
+            }
+            if (tid == 0) {
+                float sig = 0.f;
+                if (am != 0.f) sig = (-sh >= -126 && -sh <= 127) ? __int_as_float((127 - sh) << 23) : ldexpf(1.f, -sh);
+                *reinterpret_cast<float *>(rec + RL.hdr) = sig;
+            }
+            if (!g2_cbar(cb, ph, abort_flag)) return false;     // scr is reused by the next row
+        } else {
+            // Q8_0: codes and d_b per 32-block; a thread builds whole blocks
+            // (int8: two chunks, int4: one chunk, int2: one chunk of two blocks)
+            float *dsc = reinterpret_cast<float *>(rec + RL.hdr);
+            int *cor = reinterpret_cast<int *>(rec + RL.hdr + (RL.bytes - RL.hdr) / 2);
+            constexpr int EPU = EPC > 32 ? EPC : 32;            // elements per build unit
+            for (int u0 = tid; u0 < K / EPU; u0 += nth) {
+                int8_t code[EPU];
+#pragma unroll
+                for (int bb = 0; bb < EPU / 32; ++bb) {
+                    const int b = u0 * (EPU / 32) + bb;
+                    float dq = 0.f;
+                    int csum = 0;
+                    if (gateup && p.xq) {         // codes and scales from qrx_quantize_act_q8
+#pragma unroll
+                        for (int l = 0; l < 32; ++l) code[bb * 32 + l] = p.xq[row * p.in_ld + b * 32 + l];
+                        dq = p.xd[row * (p.in_ld / 32) + b];
+                    } else {                      // the same Q8_0 formula on f32 values
+                        float v[32];
+                        float am = 0.f;
+#pragma unroll
+                        for (int l = 0; l < 32; ++l) {
+                            v[l] = val(b * 32 + l);
+                            am = fmaxf(am, fabsf(v[l]));
+                        }
+                        const float f = am != 0.f ? __fdiv_rn(127.f, am) : 0.f;
+#pragma unroll
+                        for (int l = 0; l < 32; ++l) code[bb * 32 + l] = (int8_t)(am != 0.f ? q8_code(v[l], f) : 0);
+                        dq = am != 0.f ? __fdiv_rn(am, 127.f) : 0.f;
+                    }
+#pragma unroll
+                    for (int l = 0; l < 32; ++l) csum += code[bb * 32 + l];
+                    dsc[b] = dq;
+                    cor[b] = -F::OFF * csum;
+                }
+#pragma unroll
+                for (int cc = 0; cc < EPU / EPC; ++cc) {
+                    const int c = u0 * (EPU / EPC) + cc;
+                    uint32_t wd[DW];
+#pragma unroll
+                    for (int wi = 0; wi < 4; ++wi)
+#pragma unroll
+                        for (int j = 0; j < F::UPW; ++j) {
+                            uint32_t bw = 0;
+#pragma unroll
+                            for (int by = 0; by < 4; ++by)
+                                bw |= (uint32_t)(uint8_t)code[cc * EPC + elem_in_chunk<WB>(wi, j, by)] << (8 * by);
+                            wd[wi * F::UPW + j] = bw;
+                        }
+#pragma unroll
+                    for (int q = 0; q < NQ; ++q)
+                        *reinterpret_cast<uint4 *>(rec + ((size_t)q * cpr + c) * 16) =
+                            make_uint4(wd[4 * q], wd[4 * q + 1], wd[4 * q + 2], wd[4 * q + 3]);
+                }
+            }
+        }
+    }
+    return NDIG == 3 ? true : g2_cbar(cb, ph, abort_flag);
+}
+
+// ---------------------------------------------------------------- unit iterator
+// The CTA's units in order: slot s, row blocks [u, uend) of it.
+struct G2Units {
+    const int64_t *pre;
+    int nslots, nu, nrb;
+    int64_t c0, c1;
+    int s;
+    int64_t u, uend;
+    bool valid;
+};
+
+__device__ __forceinline__ int g2_slot_ntok(const G2P &p, int s, int nu)
+{
+    if (s < nu) {
+        const int e = p.union_ids[s];
+        return (e >= 0 && e < p.E) ? p.offsets[e + 1] - p.offsets[e] : 0;
+    }
+    return p.T;
+}
+
+// Cost of a unit: G2_BW for streaming its rows plus one per token (dot work).
+constexpr int64_t G2_BW = 4;
+
+__device__ void g2_units_next(G2Units &u)
+{
+    if (u.valid && ++u.u < u.uend) return;
+    u.valid = false;
+    for (;;) {
+        u.s = u.s < 0 ? 0 : u.s + 1;
+        if (u.s >= u.nslots || u.pre[u.s] >= u.c1) return;
+        const int64_t cost = (u.pre[u.s + 1] - u.pre[u.s]) / u.nrb;
+        if (cost <= 0) continue;
+        const int64_t g0 = u.pre[u.s];
+        int64_t bf = u.c0 > g0 ? (u.c0 - g0 + cost - 1) / cost : 0;
+        int64_t be = u.c1 > g0 ? (u.c1 - g0 + cost - 1) / cost : 0;
+        if (be > u.nrb) be = u.nrb;
+        if (bf < be) {
+            u.u = bf;
+            u.uend = be;
+            u.valid = true;
+            return;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- kernel
+template <int WB, int NDIG, int TP, int R, bool GATEUP, bool PROBE>
+__global__ void __launch_bounds__(G2_THREADS, 1)
+    k_gemv2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+            const __grid_constant__ CUtensorMap tsh0, const __grid_constant__ CUtensorMap tsh1,
+            const __grid_constant__ G2P p)
+{
+    using F = Fmt<WB>;
+    constexpr int NM = GATEUP ? 2 : 1;
+    constexpr int DW = F::DW, NQ = DW / 4, UPW = F::UPW;
+    constexpr int NP = NDIG == 3 ? 3 : 1;                 // integer accumulators per (token, row)
+    constexpr int NBC = WB == 2 ? 2 : 1;                 // Q8_0 blocks a chunk touches
+    constexpr int V = TP * NM * R;                        // values a lane reduces per unit
+    // int2 or many tokens: every token's digits at once would not fit in registers
+    constexpr bool TOK_OUTER = TP * NDIG * DW > 48;
+    extern __shared__ __align__(128) unsigned char sm[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + p.bar_off);
+    uint64_t *empty = full + p.stages;
+    uint64_t *cbar = empty + p.stages;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(cbar + 1);
+    int64_t *pre = reinterpret_cast<int64_t *>(sm + p.pre_off);
+    float *scr = reinterpret_cast<float *>(sm + p.red_off);
+    unsigned char *recs = sm + p.rec_off;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if constexpr (GATEUP) {
+        pdl_wait();        // the permutation comes from the kernels before
+        pdl_trigger();
+    }
+    const int nu = p.routed ? *p.n_union : 0;
+    const int nslots = nu + (p.shared ? 1 : 0);
+    if (warp == 0) {       // cost prefix over slots
+        int64_t run = 0;
+        for (int s0 = 0; s0 < nslots; s0 += 32) {
+            const int s = s0 + lane;
+            int64_t cost = 0;
+            if (s < nslots) {
+                if (s < nu) {
+                    const int e = p.union_ids[s];
+                    if (e < 0 || e >= p.E) raise_status(DERR_BADIDX);
+                }
+                const int nt = g2_slot_ntok(p, s, nu);
+                cost = nt > 0 ? (int64_t)p.nrb * (G2_BW + min(nt, TP)) : 0;
+            }
+            int64_t inc = cost;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int64_t v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            if (s < nslots) pre[s] = run + inc - cost;
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) pre[nslots] = run;
+    }
+    if (tid == 0) {
+        for (int st = 0; st < p.stages; ++st) {
+            mbar_init(g2_smem(&full[st]), 1);
+            mbar_init(g2_smem(&empty[st]), G2_NW);
+        }
+        mbar_init(g2_smem(cbar), G2_NW);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int64_t Ctot = pre[nslots];
+    G2Units U0;
+    U0.pre = pre;
+    U0.nslots = nslots;
+    U0.nu = nu;
+    U0.nrb = p.nrb;
+    U0.c0 = Ctot * blockIdx.x / gridDim.x;
+    U0.c1 = Ctot * (blockIdx.x + 1) / gridDim.x;
+    U0.s = -1;
+    U0.u = U0.uend = 0;
+    U0.valid = false;
+    g2_units_next(U0);
+
+    if (warp == G2_NW) {
+        // ======================== producer (one thread) ========================
+        // Each stage is one tiled TMA box per matrix (the slice's ks bytes of the
+        // unit's rb rows; rows past the matrix are zero-filled), plus, on the
+        // unit's last slice, one bulk copy of each matrix's row scales.
+        if (lane != 0) return;
+        G2Units u = U0;
+        uint32_t g = 0;
+        bool ok = true;
+        const int nbox = p.rb / p.box_rows;
+        while (ok && u.valid) {
+            const bool routed = u.s < nu;
+            int e = 0;
+            if (routed) {
+                e = p.union_ids[u.s];
+                e = (e >= 0 && e < p.E) ? e : 0;
+            }
+            const CUtensorMap *map0 = routed ? &tm0 : &tsh0;
+            const CUtensorMap *map1 = routed ? &tm1 : &tsh1;
+            const int z = routed ? e : 0;
+            const float *S0 = routed ? p.m[0].s + (int64_t)e * p.m[0].ss : p.msh[0].s;
+            const float *S1 = routed ? p.m[NM - 1].s + (int64_t)e * p.m[NM - 1].ss : p.msh[NM - 1].s;
+            const int r0 = (int)(u.u * p.rb);
+            const int nr = min(p.rb, p.rows - r0);
+            for (int j = 0; j < p.nslice; ++j) {
+                const uint32_t st = g % p.stages;
+                if (g >= (uint32_t)p.stages && !g2_wait(g2_smem(&empty[st]), ((g / p.stages) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const bool last = j == p.nslice - 1;
+                const uint32_t bytes = (uint32_t)(NM * p.rb * p.ks + (last ? NM * nr * 4 : 0));
+                const uint32_t fb = g2_smem(&full[st]);
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb), "r"(bytes) : "memory");
+                unsigned char *dst = sm + (size_t)st * p.stage_bytes;
+                const int x = j * (p.ks / 8);          // 8-byte elements
+                for (int b = 0; b < nbox; ++b) {
+                    tma_load_3d(g2_smem(dst + (size_t)b * p.box_rows * p.ks), map0, x, r0 + b * p.box_rows, z, fb);
+                    if constexpr (NM == 2)
+                        tma_load_3d(g2_smem(dst + (size_t)(p.rb + b * p.box_rows) * p.ks), map1, x, r0 + b * p.box_rows,
+                                    z, fb);
+                }
+                if (last) {
+                    bulk_copy(g2_smem(dst + p.scale_off), S0 + r0, (uint32_t)(nr * 4), fb);
+                    if constexpr (NM == 2) bulk_copy(g2_smem(dst + p.scale_off + p.rb * 4), S1 + r0, (uint32_t)(nr * 4), fb);
+                }
+                ++g;
+            }
+            g2_units_next(u);
+        }
+        // the copies issued land before the CTA may leave
+        for (uint32_t i = 0; i < (uint32_t)p.stages && i < g; ++i) {
+            const uint32_t gl = g - 1 - i;
+            bool done = false;
+            for (long long it = 0; it < G2_WAIT_CAP && !done; ++it)
+                done = g2_try(g2_smem(&full[gl % p.stages]), (gl / p.stages) & 1);
+            if (!done) raise_status(DERR_TIMEOUT);
+        }
+        return;
+    }
+
+    // ======================== compute warps ========================
+    const int LPR = p.lpr;
+    const int c = lane % LPR, grp = lane / LPR;
+    uint32_t cph = 0;      // compute-barrier phase
+    QRX_CHECK_ONLY(const int64_t n_pos = p.routed ? (int64_t)p.T * p.k : 0;)
+    QRX_CHECK_ONLY(const int64_t n_out = max(n_pos, p.shared ? p.sh_out_row0 + p.T : (int64_t)0);)
+    if constexpr (GATEUP) {
+        // the records of every token, once (x is an input of the call)
+        if (!g2_build<WB, NDIG>(p, recs, p.T, [](int i) -> int64_t { return i; }, true, scr, cbar, cph, abort_flag))
+            return;
+    } else {
+        pdl_wait();        // h comes from the kernel before
+        pdl_trigger();
+    }
+    G2Units u = U0;
+    uint32_t g = 0;
+    int cur_s = -1, nt = 0;
+    const unsigned char *rec[TP];
+    int64_t orow[TP];
+    int corr[TP][NP];      // NDIG = 3: OFF * (this lane's digit sums over its chunks), per plane
+    float sig[TP];         // NDIG = 3: the records' scales
+#pragma unroll
+    for (int t = 0; t < TP; ++t) {
+        rec[t] = recs;
+        orow[t] = 0;
+        sig[t] = 0.f;
+#pragma unroll
+        for (int pl = 0; pl < NP; ++pl) corr[t][pl] = 0;
+    }
+    bool ok = true;
+    while (ok && u.valid) {
+        if (u.s != cur_s) {
+            // ---- enter a slot: its tokens, their records, this lane's corrections
+            const bool routed = u.s < nu;
+            int p0 = 0;
+            if (routed) {
+                int e = p.union_ids[u.s];
+                e = (e >= 0 && e < p.E) ? e : 0;
+                p0 = p.offsets[e];
+            }
+            nt = min(g2_slot_ntok(p, u.s, nu), TP);
+            int64_t inrow[TP];
+#pragma unroll
+            for (int i = 0; i < TP; ++i) {
+                const int ii = min(i, max(nt - 1, 0));
+                if (routed) {
+                    QRX_CHECK_OR((int64_t)p0 + ii < n_pos, ok = false);
+                    orow[i] = p0 + ii;
+                    if constexpr (GATEUP) {
+                        const int a = p.sorted[p0 + ii];
+                        QRX_CHECK_OR(a >= 0 && a / p.k < p.T, ok = false);
+                        inrow[i] = a / p.k;
+                    } else {
+                        inrow[i] = p0 + ii;
+                    }
+                } else {
+                    orow[i] = p.sh_out_row0 + ii;
+                    inrow[i] = GATEUP ? ii : p.sh_in_row0 + ii;
+                }
+            }
+            if (!ok) break;
+            if constexpr (GATEUP) {
+#pragma unroll
+                for (int i = 0; i < TP; ++i) rec[i] = recs + (size_t)inrow[i] * p.rec_bytes;
+            } else {
+                // every warp is done with the previous slot's records
+                if (!g2_cbar(cbar, cph, abort_flag)) break;
+                if (!g2_build<WB, NDIG>(p, recs, nt, [&](int i) -> int64_t { return g2_pick(inrow, i); }, false,
+                                        scr, cbar, cph, abort_flag))
+                    break;
+#pragma unroll
+                for (int i = 0; i < TP; ++i) rec[i] = recs + (size_t)min(i, max(nt - 1, 0)) * p.rec_bytes;
+            }
+            if constexpr (NDIG == 3) {
+#pragma unroll
+                for (int i = 0; i < TP; ++i) {
+                    sig[i] = *reinterpret_cast<const float *>(rec[i] + g2_rec(3, p.K).hdr);
+#pragma unroll
+                    for (int pl = 0; pl < 3; ++pl) {
+                        int sum = 0;
+                        for (int j = 0; j < p.nslice; ++j) {
+                            const int cg = j * p.cps + c;
+#pragma unroll
+                            for (int q = 0; q < NQ; ++q) {
+                                const uint4 d4 = *reinterpret_cast<const uint4 *>(
+                                    rec[i] + ((size_t)(pl * NQ + q) * p.cpr + cg) * 16);
+                                sum = dp4a(0x01010101u, d4.x, sum);
+                                sum = dp4a(0x01010101u, d4.y, sum);
+                                sum = dp4a(0x01010101u, d4.z, sum);
+                                sum = dp4a(0x01010101u, d4.w, sum);
+                            }
+                        }
+                        corr[i][pl] = F::OFF * sum;
+                    }
+                }
+            }
+            cur_s = u.s;
+        }
+        // ---- one unit: nslice stages
+        int iacc[TP][NM][R][NP];
+        float facc[TP][NM][R];
+#pragma unroll
+        for (int t = 0; t < TP; ++t)
+#pragma unroll
+            for (int m = 0; m < NM; ++m)
+#pragma unroll
+                for (int i = 0; i < R; ++i) {
+                    facc[t][m][i] = 0.f;
+#pragma unroll
+                    for (int pl = 0; pl < NP; ++pl) iacc[t][m][i][pl] = 0;
+                }
+        const int lrow0 = warp * p.rw + grp;             // this lane's first row in the unit (then + gpw)
+        for (int j = 0; j < p.nslice; ++j, ++g) {
+            const uint32_t st = g % p.stages;
+            if (!g2_wait(g2_smem(&full[st]), (g / p.stages) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const unsigned char *stg = sm + (size_t)st * p.stage_bytes;
+            const int cg = j * p.cps + c;                // this lane's chunk of the row
+            auto load_dig = [&](int t, uint32_t (&d)[NDIG][DW]) {
+#pragma unroll
+                for (int pl = 0; pl < NDIG; ++pl)
+#pragma unroll
+                    for (int q = 0; q < NQ; ++q) {
+                        const uint4 d4 =
+                            *reinterpret_cast<const uint4 *>(rec[t] + ((size_t)(pl * NQ + q) * p.cpr + cg) * 16);
+                        d[pl][4 * q] = d4.x;
+                        d[pl][4 * q + 1] = d4.y;
+                        d[pl][4 * q + 2] = d4.z;
+                        d[pl][4 * q + 3] = d4.w;
+                    }
+            };
+            auto load_blk = [&](int t, float (&dq)[NBC], int (&cb)[NBC]) {
+                const G2Rec RL = g2_rec(1, p.K);
+                const float *dsc = reinterpret_cast<const float *>(rec[t] + RL.hdr);
+                const int *cor = reinterpret_cast<const int *>(rec[t] + RL.hdr + (RL.bytes - RL.hdr) / 2);
+#pragma unroll
+                for (int bc = 0; bc < NBC; ++bc) {
+                    const int b = WB == 8 ? (cg >> 1) : (WB == 4 ? cg : 2 * cg + bc);
+                    dq[bc] = dsc[b];
+                    cb[bc] = cor[b];
+                }
+            };
+            auto unpack = [&](int m, int i, uint32_t (&uw)[4][UPW]) {
+                const uint4 wv = *reinterpret_cast<const uint4 *>(
+                    stg + ((size_t)(m * p.rb + lrow0 + p.gpw * i)) * p.ks + (size_t)c * 16);
+                unpack_word<WB>(wv.x, uw[0]);
+                unpack_word<WB>(wv.y, uw[1]);
+                unpack_word<WB>(wv.z, uw[2]);
+                unpack_word<WB>(wv.w, uw[3]);
+            };
+            // one unpacked weight chunk against one token's digits
+            auto dot = [&](int t, int m, int i, const uint32_t (&uw)[4][UPW], const uint32_t (&d)[NDIG][DW],
+                           const float (&dq)[NBC], const int (&cb)[NBC]) {
+                if constexpr (NDIG == 3) {
+                    int a0 = iacc[t][m][i][0], a1 = iacc[t][m][i][1], a2 = iacc[t][m][i][2];
+#pragma unroll
+                    for (int wi = 0; wi < 4; ++wi)
+#pragma unroll
+                        for (int jj = 0; jj < UPW; ++jj) {
+                            a0 = dp4a(uw[wi][jj], d[0][wi * UPW + jj], a0);
+                            a1 = dp4a(uw[wi][jj], d[1][wi * UPW + jj], a1);
+                            a2 = dp4a(uw[wi][jj], d[2][wi * UPW + jj], a2);
+                        }
+                    iacc[t][m][i][0] = a0;
+                    iacc[t][m][i][1] = a1;
+                    iacc[t][m][i][2] = a2;
+                } else {
+                    int ib[NBC];
+#pragma unroll
+                    for (int bc = 0; bc < NBC; ++bc) ib[bc] = cb[bc];
+#pragma unroll
+                    for (int wi = 0; wi < 4; ++wi)
+#pragma unroll
+                        for (int jj = 0; jj < UPW; ++jj) {
+                            const int bc = WB == 2 ? (wi >> 1) : 0;
+                            ib[bc] = dp4a(uw[wi][jj], d[0][wi * UPW + jj], ib[bc]);
+                        }
+                    // int8: a block is two chunks on lanes 2b, 2b+1
+                    if constexpr (WB == 8) ib[0] += __shfl_xor_sync(0xffffffffu, ib[0], 1);
+                    const bool mine = WB != 8 || (c & 1) == 0;
+#pragma unroll
+                    for (int bc = 0; bc < NBC; ++bc) {
+                        if (mine) facc[t][m][i] = fmaf(dq[bc], (float)ib[bc], facc[t][m][i]);
+                        if constexpr (PROBE) {
+                            const int64_t row = u.u * p.rb + lrow0 + p.gpw * i;
+                            if (mine && row < p.rows) {
+                                const int b = WB == 8 ? (cg >> 1) : (WB == 4 ? cg : 2 * cg + bc);
+                                p.probe[((orow[t] * NM + m) * p.rows + row) * (int64_t)(p.K / 32) + b] = ib[bc];
+                            }
+                        }
+                    }
+                }
+            };
+            if constexpr (TOK_OUTER) {
+#pragma unroll
+                for (int t = 0; t < TP; ++t) {
+                    if (t < nt) {
+                        uint32_t d[NDIG][DW];
+                        float dq[NBC] = {};
+                        int cb[NBC] = {};
+                        load_dig(t, d);
+                        if constexpr (NDIG == 1) load_blk(t, dq, cb);
+#pragma unroll
+                        for (int m = 0; m < NM; ++m)
+#pragma unroll
+                            for (int i = 0; i < R; ++i) {
+                                uint32_t uw[4][UPW];
+                                unpack(m, i, uw);
+                                dot(t, m, i, uw, d, dq, cb);
+                            }
+                    }
+                }
+            } else {
+                uint32_t d[TP][NDIG][DW];
+                float dq[TP][NBC] = {};
+                int cb[TP][NBC] = {};
+#pragma unroll
+                for (int t = 0; t < TP; ++t)
+                    if (t < nt) {
+                        load_dig(t, d[t]);
+                        if constexpr (NDIG == 1) load_blk(t, dq[t], cb[t]);
+                    }
+#pragma unroll
+                for (int m = 0; m < NM; ++m)
+#pragma unroll
+                    for (int i = 0; i < R; ++i) {
+                        uint32_t uw[4][UPW];
+                        unpack(m, i, uw);
+#pragma unroll
+                        for (int t = 0; t < TP; ++t)
+                            if (t < nt) dot(t, m, i, uw, d[t], dq[t], cb[t]);
+                    }
+            }
+            if (j == p.nslice - 1) {
+                // ---- epilogue: lane partials -> row totals -> scales -> outputs
+                float v[V];
+#pragma unroll
+                for (int t = 0; t < TP; ++t)
+#pragma unroll
+                    for (int i = 0; i < R; ++i)
+#pragma unroll
+                        for (int m = 0; m < NM; ++m) {
+                            float x;
+                            if constexpr (NDIG == 3)
+                                x = fmaf(65536.f, (float)(iacc[t][m][i][2] - corr[t][2]),
+                                         fmaf(256.f, (float)(iacc[t][m][i][1] - corr[t][1]),
+                                              (float)(iacc[t][m][i][0] - corr[t][0])));
+                            else
+                                x = facc[t][m][i];
+                            v[(t * R + i) * NM + m] = t < nt ? x : 0.f;
+                        }
+                if (LPR == 32) g2_tr_reduce<V, 32>(v, lane);
+                else if (LPR == 16) g2_tr_reduce<V, 16>(v, lane);
+                else if (LPR == 8) g2_tr_reduce<V, 8>(v, lane);
+                else if (LPR == 4) g2_tr_reduce<V, 4>(v, lane);
+                else if (LPR == 2) g2_tr_reduce<V, 2>(v, lane);
+                const float *scl = reinterpret_cast<const float *>(stg + p.scale_off);
+                // total `tot` (and for gate/up the matching up total `upv`) of value idx
+                auto emit = [&](int idx, float tot, float upv) {
+                    const int t = idx / (NM * R), i = (idx / NM) % R;
+                    const int lrow = lrow0 + p.gpw * i;
+                    const int64_t row = u.u * p.rb + lrow;
+                    if (t >= nt || row >= p.rows) return;
+                    const int64_t o = g2_pick(orow, t);
+                    QRX_CHECK_OR(o >= 0 && o < n_out, return);
+                    const float sg = NDIG == 3 ? g2_pick(sig, t) : 1.f;
+                    if constexpr (GATEUP)
+                        p.out[o * p.out_ld + row] = silu_mul(scl[lrow] * (sg * tot), scl[p.rb + lrow] * (sg * upv));
+                    else
+                        p.out[o * p.out_ld + row] = scl[lrow] * (sg * tot);
+                };
+                if (V <= LPR) {
+                    const int rep = LPR / V;
+                    const int idx = c / rep;
+                    const float upv = GATEUP ? __shfl_xor_sync(0xffffffffu, v[0], rep) : 0.f;
+                    if (c % rep == 0 && (!GATEUP || (idx & 1) == 0)) emit(idx, v[0], upv);
+                } else {
+                    const int nv = V / LPR;
+#pragma unroll
+                    for (int q = 0; q < V; q += NM)
+                        if (q < nv) emit(c * nv + q, v[q], GATEUP ? v[q + NM - 1] : 0.f);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(g2_smem(&empty[st]));
+        }
+        g2_units_next(u);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+struct G2Plan {
+    G2P p;
+    int tp, r;
+};
+
+// Geometry for one projection: `nm` matrices of `rows` rows x K codes at wbits,
+// activations with ndig digit planes, calls of T <= G2_TMAX tokens.
+static inline bool g2_plan(G2Plan &pl, int wbits, int ndig, int K, int rows, int nm, int T, int maxslots)
+{
+    G2P &p = pl.p;
+    p = G2P{};
+    if (T < 1 || T > G2_TMAX) return false;
+    pl.tp = T == 1 ? 1 : (T == 2 ? 2 : 4);
+    // rows per lane: accumulators are NDIG (or 1) x nm x R x TP
+    const int perrow = (ndig == 3 ? 3 : 1) * nm * pl.tp;
+    pl.r = 48 / perrow >= 8 ? 8 : (48 / perrow >= 4 ? 4 : 2);
+    if (nm == 2 && pl.r > 4) pl.r = 4;
+    p.K = K;
+    p.rows = rows;
+    p.row_bytes = K * wbits / 8;
+    if (p.row_bytes % 16) return false;
+    p.cpr = p.row_bytes / 16;
+    p.ks = p.row_bytes < G2_KS ? p.row_bytes : G2_KS;
+    if (p.row_bytes % p.ks) return false;
+    p.cps = p.ks / 16;
+    if (32 % p.cps != 0 && p.cps != 32) return false;
+    p.nslice = p.row_bytes / p.ks;
+    p.lpr = p.cps;
+    p.gpw = 32 / p.lpr;
+    p.rw = pl.r * p.gpw;
+    p.rb = G2_NW * p.rw;
+    p.nrb = (rows + p.rb - 1) / p.rb;
+    p.box_rows = p.rb < 256 ? p.rb : 256;    // a TMA box spans at most 256 rows
+    p.scale_off = nm * p.rb * p.ks;
+    p.stage_bytes = (p.scale_off + nm * p.rb * 4 + 127) & ~127;
+    p.rec_bytes = (g2_rec(ndig, K).bytes + 127) & ~127;
+    p.nrec = nm == 2 ? T : pl.tp;        // gate/up: every token; down: one slot's rows
+    const int fixed_tail = 128 /*barriers*/ + 256 /*scratch*/ + (maxslots + 2) * 8;
+    const int avail = G2_SMEM_MAX - p.nrec * p.rec_bytes - fixed_tail;
+    int stages = avail / p.stage_bytes;
+    if (stages > 8) stages = 8;
+    if (stages < 2) return false;
+    p.stages = stages;
+    int o = stages * p.stage_bytes;
+    p.rec_off = o;
+    o += p.nrec * p.rec_bytes;
+    p.bar_off = o;
+    o += 2 * stages * 8 + 16;
+    o = (o + 15) & ~15;
+    p.red_off = o;
+    o += 256;
+    p.pre_off = o;
+    o += (maxslots + 2) * 8;
+    p.smem = o;
+    return o <= G2_SMEM_MAX;
+}
+
+// Tiled TMA map of one packed matrix of nexp experts: 8-byte elements, dims
+// (row_bytes/8, rows, nexp), box (ks/8, box_rows, 1), no swizzle (a box lands as
+// box_rows rows of ks bytes).  Encoded maps are kept in a small cache keyed by
+// every argument, so a call with the same experts encodes nothing.
+struct G2MapKey {
+    const void *q;
+    int64_t row_bytes, rows, nexp, stride, ks, box_rows;
+    bool operator==(const G2MapKey &o) const
+    {
+        return q == o.q && row_bytes == o.row_bytes && rows == o.rows && nexp == o.nexp && stride == o.stride &&
+               ks == o.ks && box_rows == o.box_rows;
+    }
+};
+
+static bool g2_map(CUtensorMap *m, const G2MapKey &k)
+{
+    constexpr int NC = 64;
+    static std::mutex mu;
+    static G2MapKey keys[NC];
+    static CUtensorMap maps[NC];
+    static int used = 0, next = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (keys[i] == k) {
+                *m = maps[i];
+                return true;
+            }
+    }
+    const auto fn = tc_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)(k.row_bytes / 8), (cuuint64_t)k.rows, (cuuint64_t)k.nexp};
+    const cuuint64_t strides[2] = {(cuuint64_t)k.row_bytes, (cuuint64_t)k.stride};
+    const cuuint32_t box[3] = {(cuuint32_t)(k.ks / 8), (cuuint32_t)k.box_rows, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    CUtensorMap t{};
+    if (fn(&t, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void *>(k.q), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    std::lock_guard<std::mutex> lock(mu);
+    keys[next] = k;
+    maps[next] = t;
+    next = (next + 1) % NC;
+    if (used < NC) ++used;
+    *m = t;
+    return true;
+}
+
+// The four maps of a launch: routed matrices 0/1 and the shared expert's 0/1
+// (down: one matrix each; unused maps are copies, never read).
+struct G2Maps {
+    CUtensorMap m0, m1, s0, s1;
+};
+
+static bool g2_maps(G2Maps &M, const G2P &p, int nm, const MatRef &r0, const MatRef &r1, const MatRef &sh0,
+                    const MatRef &sh1)
+{
+    M = G2Maps{};
+    const int64_t one = (int64_t)p.rows * p.row_bytes;
+    bool ok = true;
+    if (p.routed) {
+        ok = ok && g2_map(&M.m0, G2MapKey{r0.q, p.row_bytes, p.rows, p.E, p.E > 1 ? r0.sq : one, p.ks, p.box_rows});
+        if (nm == 2)
+            ok = ok && g2_map(&M.m1, G2MapKey{r1.q, p.row_bytes, p.rows, p.E, p.E > 1 ? r1.sq : one, p.ks, p.box_rows});
+    }
+    if (p.shared) {
+        ok = ok && g2_map(&M.s0, G2MapKey{sh0.q, p.row_bytes, p.rows, 1, one, p.ks, p.box_rows});
+        if (nm == 2) ok = ok && g2_map(&M.s1, G2MapKey{sh1.q, p.row_bytes, p.rows, 1, one, p.ks, p.box_rows});
+    }
+    if (nm == 1) {
+        M.m1 = M.m0;
+        M.s1 = M.s0;
+    }
+    if (!p.routed) {
+        M.m0 = M.s0;
+        M.m1 = M.s1;
+    }
+    if (!p.shared) {
+        M.s0 = M.m0;
+        M.s1 = M.m1;
+    }
+    return ok;
+}
+
+template <int WB, int ND, int TP, int R, bool GU, bool PR>
+static cudaError_t g2_go(const G2Maps &M, const G2P &p, int grid, cudaStream_t st)
+{
+    auto kern = k_gemv2<WB, ND, TP, R, GU, PR>;
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= 64 || !(configured.load(std::memory_order_acquire) >> dev & 1ull)) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G2_SMEM_MAX);
+        if (err != cudaSuccess) return err;
+        if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_release);
+    }
+    return launch_k(kern, dim3(grid), dim3(G2_THREADS), (size_t)p.smem, st, M.m0, M.m1, M.s0, M.s1, p);
+}
+
+template <bool GU, bool PR>
+static cudaError_t g2_dispatch(const G2Maps &M, const G2Plan &pl, int wbits, int ndig, int grid, cudaStream_t st)
+{
+#define QRX_G2(WB, ND, TP, R) \
+    if (wbits == WB && ndig == ND && pl.tp == TP && pl.r == R) return g2_go<WB, ND, TP, R, GU, PR>(M, pl.p, grid, st);
+    // rows per lane R: the accumulators (NDIG or 1) x matrices x R x TP stay within 48
+    if constexpr (PR) {        // Q8_0 with the block-sum side output
+        if constexpr (GU) {
+            QRX_G2(4, 1, 1, 4) QRX_G2(4, 1, 2, 4) QRX_G2(4, 1, 4, 4)
+            QRX_G2(8, 1, 1, 4) QRX_G2(8, 1, 2, 4) QRX_G2(8, 1, 4, 4)
+            QRX_G2(2, 1, 1, 4) QRX_G2(2, 1, 2, 4) QRX_G2(2, 1, 4, 4)
+        } else {
+            QRX_G2(4, 1, 1, 8) QRX_G2(4, 1, 2, 8) QRX_G2(4, 1, 4, 8)
+            QRX_G2(8, 1, 1, 8) QRX_G2(8, 1, 2, 8) QRX_G2(8, 1, 4, 8)
+            QRX_G2(2, 1, 1, 8) QRX_G2(2, 1, 2, 8) QRX_G2(2, 1, 4, 8)
+        }
+    } else if constexpr (GU) {
+        QRX_G2(4, 3, 1, 4) QRX_G2(4, 3, 2, 4) QRX_G2(4, 3, 4, 2) QRX_G2(4, 1, 1, 4) QRX_G2(4, 1, 2, 4) QRX_G2(4, 1, 4, 4)
+        QRX_G2(8, 3, 1, 4) QRX_G2(8, 3, 2, 4) QRX_G2(8, 3, 4, 2) QRX_G2(8, 1, 1, 4) QRX_G2(8, 1, 2, 4) QRX_G2(8, 1, 4, 4)
+        QRX_G2(2, 3, 1, 4) QRX_G2(2, 3, 2, 4) QRX_G2(2, 3, 4, 2) QRX_G2(2, 1, 1, 4) QRX_G2(2, 1, 2, 4) QRX_G2(2, 1, 4, 4)
+    } else {
+        QRX_G2(4, 3, 1, 8) QRX_G2(4, 3, 2, 8) QRX_G2(4, 3, 4, 4) QRX_G2(4, 1, 1, 8) QRX_G2(4, 1, 2, 8) QRX_G2(4, 1, 4, 8)
+        QRX_G2(8, 3, 1, 8) QRX_G2(8, 3, 2, 8) QRX_G2(8, 3, 4, 4) QRX_G2(8, 1, 1, 8) QRX_G2(8, 1, 2, 8) QRX_G2(8, 1, 4, 8)
+        QRX_G2(2, 3, 1, 8) QRX_G2(2, 3, 2, 8) QRX_G2(2, 3, 4, 4) QRX_G2(2, 1, 1, 8) QRX_G2(2, 1, 2, 8) QRX_G2(2, 1, 4, 8)
+    }
+#undef QRX_G2
+    return cudaErrorInvalidValue;
+}
+
+static inline void g2_common(G2P &p, const FfnArgs &a)
+{
+    p.routed = a.routed;
+    p.shared = a.shared;
+    p.offsets = a.offsets;
+    p.sorted = a.sorted;
+    p.union_ids = a.union_ids;
+    p.n_union = a.n_union;
+    p.E = a.E;
+    p.k = a.k;
+    p.T = a.T;
+    p.afmt = a.afmt;
+}
+
+static inline G2Mat g2_mat(const MatRef &m) { return G2Mat{m.q, m.s, m.sq, m.ss}; }
+
+bool g2_use(const FfnArgs &a)
+{
+    if (a.T < 1 || a.T > G2_TMAX || !tc_encode_fn()) return false;
+    const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
+    G2Plan pg, pd;
+    return g2_plan(pg, a.wbits, ndig, a.H, a.I, 2, a.T, a.E + 1) && g2_plan(pd, a.wbits, ndig, a.I, a.H, 1, a.T, a.E + 1);
+}
+
+cudaError_t launch_g2_gateup(const FfnArgs &a, int num_sms, cudaStream_t st, int32_t *probe)
+{
+    if (!a.routed && !a.shared) return cudaSuccess;
+    const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
+    G2Plan pl;
+    if (!g2_plan(pl, a.wbits, ndig, a.H, a.I, 2, a.T, a.E + 1)) return cudaErrorInvalidValue;
+    G2P &p = pl.p;
+    g2_common(p, a);
+    p.m[0] = g2_mat(a.gate);
+    p.m[1] = g2_mat(a.up);
+    p.msh[0] = g2_mat(a.gate_sh);
+    p.msh[1] = g2_mat(a.up_sh);
+    p.x = a.x;
+    p.xq = a.xq;
+    p.xd = a.xd;
+    p.in_ld = a.H;
+    p.sh_in_row0 = 0;
+    p.out = a.h;
+    p.out_ld = a.h_ld;
+    p.sh_out_row0 = a.sh_h_row0;
+    p.probe = probe;
+    G2Maps M;
+    if (!g2_maps(M, p, 2, a.gate, a.up, a.gate_sh, a.up_sh)) return cudaErrorInvalidValue;
+    if (probe) return ndig == 1 ? g2_dispatch<true, true>(M, pl, a.wbits, ndig, num_sms, st) : cudaErrorInvalidValue;
+    return g2_dispatch<true, false>(M, pl, a.wbits, ndig, num_sms, st);
+}
+
+cudaError_t launch_g2_down(const FfnArgs &a, int num_sms, cudaStream_t st, int32_t *probe)
+{
+    if (!a.routed && !a.shared) return cudaSuccess;
+    const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
+    G2Plan pl;
+    if (!g2_plan(pl, a.wbits, ndig, a.I, a.H, 1, a.T, a.E + 1)) return cudaErrorInvalidValue;
+    G2P &p = pl.p;
+    g2_common(p, a);
+    p.m[0] = p.m[1] = g2_mat(a.down);
+    p.msh[0] = p.msh[1] = g2_mat(a.down_sh);
+    p.x = a.h;
+    p.xq = nullptr;
+    p.xd = nullptr;
+    p.in_ld = a.h_ld;
+    p.sh_in_row0 = a.sh_h_row0;
+    p.out = a.y;
+    p.out_ld = a.y_ld;
+    p.sh_out_row0 = a.sh_y_row0;
+    p.probe = probe;
+    G2Maps M;
+    if (!g2_maps(M, p, 1, a.down, a.down, a.down_sh, a.down_sh)) return cudaErrorInvalidValue;
+    if (probe) return ndig == 1 ? g2_dispatch<false, true>(M, pl, a.wbits, ndig, num_sms, st) : cudaErrorInvalidValue;
+    return g2_dispatch<false, false>(M, pl, a.wbits, ndig, num_sms, st);
+}
+
+}  // namespace qrx

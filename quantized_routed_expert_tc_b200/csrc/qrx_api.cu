@@ -10,7 +10,6 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
-#include <mutex>
 
 #include "qrx_internal.h"
 #include "qrx_dev.cuh"
@@ -19,6 +18,7 @@
 #include "k_permute.cuh"
 #include "k_ffn_gemv.cuh"
 #include "k_ffn_tc.cuh"
+#include "k_gemv2.cuh"
 #include "k_combine.cuh"
 
 using namespace qrx;
@@ -128,13 +128,27 @@ int check_ws(const qrx_cfg *c, int T, void *ws, size_t ws_bytes)
     return QRX_OK;
 }
 
-int check_experts(const qrx_experts *x)
+// One packed matrix: pointers 16-byte aligned; for a set of several experts
+// the strides keep every expert's codes and scales 16-byte aligned.
+int check_mat(const qrx_mat &m, bool several)
 {
-    if (!x || !x->w13 || !x->s13 || !x->w2 || !x->s2) return QRX_EINVAL;
-    if (!aligned(x->w13, 16) || !aligned(x->w2, 16) || !aligned(x->s13, 16) || !aligned(x->s2, 16))
+    if (!m.q || !m.scale || !aligned(m.q, 16) || !aligned(m.scale, 16)) return QRX_EINVAL;
+    if (several && (m.expert_stride_q < 0 || m.expert_stride_q % 16 != 0 || m.expert_stride_q >= ((int64_t)1 << 40) ||
+                    m.expert_stride_s < 0 || m.expert_stride_s % 4 != 0))
         return QRX_EINVAL;
     return QRX_OK;
 }
+
+int check_experts(const qrx_experts *x, bool several = true)
+{
+    if (!x) return QRX_EINVAL;
+    int v;
+    if ((v = check_mat(x->gate, several)) || (v = check_mat(x->up, several)) || (v = check_mat(x->down, several)))
+        return v;
+    return QRX_OK;
+}
+
+MatRef mat_ref(const qrx_mat &m) { return MatRef{m.q, m.scale, m.expert_stride_q, m.expert_stride_s}; }
 
 int check_act(const qrx_cfg *c, const qrx_act *a)
 {
@@ -174,10 +188,9 @@ void set_act(FfnArgs &a, const qrx_act *act)
 void set_routed(FfnArgs &a, const qrx_experts *r, const qrx_perm *p)
 {
     a.routed = 1;
-    a.w13 = r->w13;
-    a.s13 = r->s13;
-    a.w2 = r->w2;
-    a.s2 = r->s2;
+    a.gate = mat_ref(r->gate);
+    a.up = mat_ref(r->up);
+    a.down = mat_ref(r->down);
     a.offsets = p->offsets;
     a.sorted = p->sorted;
     a.union_ids = p->union_ids;
@@ -187,10 +200,9 @@ void set_routed(FfnArgs &a, const qrx_experts *r, const qrx_perm *p)
 void set_shared(FfnArgs &a, const qrx_experts *s)
 {
     a.shared = 1;
-    a.w13_sh = s->w13;
-    a.s13_sh = s->s13;
-    a.w2_sh = s->w2;
-    a.s2_sh = s->s2;
+    a.gate_sh = mat_ref(s->gate);
+    a.up_sh = mat_ref(s->up);
+    a.down_sh = mat_ref(s->down);
 }
 
 }  // namespace
@@ -415,12 +427,49 @@ int qrx_expert_down(const qrx_cfg *c, const qrx_experts *routed, const qrx_perm 
     return cuda_code(launch_ffn_down(a, num_sms_current(), (cudaStream_t)stream));
 }
 
+int qrx_expert_gateup_q8_sums(const qrx_cfg *c, const qrx_experts *routed, const qrx_perm *perm,
+                              const qrx_act *act, int32_t T, float *h_sorted, int32_t *acc, void *ws,
+                              size_t ws_bytes, void *stream)
+{
+    int v = check_common(c, T);
+    if (v) return v;
+    if ((v = check_experts(routed)) || (v = check_perm(perm)) || (v = check_act(c, act))) return v;
+    if (!h_sorted || !acc) return QRX_EINVAL;
+    if ((v = check_ws(c, T, ws, ws_bytes))) return v;
+    FfnArgs a = ffn_args(c, T);
+    set_act(a, act);
+    set_routed(a, routed, perm);
+    if (c->afmt != QRX_A_Q8_0 || !g2_use(a)) return QRX_EUNSUPPORTED;
+    a.h = h_sorted;
+    a.h_ld = c->inter;
+    return cuda_code(launch_g2_gateup(a, num_sms_current(), (cudaStream_t)stream, acc));
+}
+
+int qrx_expert_down_q8_sums(const qrx_cfg *c, const qrx_experts *routed, const qrx_perm *perm,
+                            const float *h_sorted, int32_t T, float *y_sorted, int32_t *acc, void *ws,
+                            size_t ws_bytes, void *stream)
+{
+    int v = check_common(c, T);
+    if (v) return v;
+    if ((v = check_experts(routed)) || (v = check_perm(perm))) return v;
+    if (!h_sorted || !y_sorted || !acc) return QRX_EINVAL;
+    if ((v = check_ws(c, T, ws, ws_bytes))) return v;
+    FfnArgs a = ffn_args(c, T);
+    set_routed(a, routed, perm);
+    if (c->afmt != QRX_A_Q8_0 || !g2_use(a)) return QRX_EUNSUPPORTED;
+    a.h = const_cast<float *>(h_sorted);
+    a.h_ld = c->inter;
+    a.y = y_sorted;
+    a.y_ld = c->hidden;
+    return cuda_code(launch_g2_down(a, num_sms_current(), (cudaStream_t)stream, acc));
+}
+
 int qrx_shared_ffn(const qrx_cfg *c, const qrx_experts *shared, const qrx_act *act, int32_t T,
                    float *h_sh, float *y_sh, void *ws, size_t ws_bytes, void *stream)
 {
     int v = check_common(c, T);
     if (v) return v;
-    if ((v = check_experts(shared)) || (v = check_act(c, act))) return v;
+    if ((v = check_experts(shared, false)) || (v = check_act(c, act))) return v;
     if (!y_sh) return QRX_EINVAL;
     if ((v = check_ws(c, T, ws, ws_bytes))) return v;
     const Ws L = ws_layout(c, T);
@@ -474,7 +523,7 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     if (!x || !Wr || !bias || !topk_idx || !topk_w || !out) return QRX_EINVAL;
     if (!aligned(x, 16)) return QRX_EINVAL;
     if ((v = check_experts(routed))) return v;
-    if (shared && (v = check_experts(shared))) return v;
+    if (shared && (v = check_experts(shared, false))) return v;
     if ((v = check_ws(c, T, ws, ws_bytes))) return v;
     if (!aligned(out, 16)) return QRX_EINVAL;
     if (opts && (!(opts->expert_top_p == opts->expert_top_p) || (opts->usage && !aligned(opts->usage, 8))))
@@ -495,12 +544,13 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     a.hperm = at<unsigned char>(ws, L.hperm);
     a.hperm_ready = 1;
     if (!mark(0)) return QRX_ECUDA;
-    const bool tc = ffn_use_tc(a);     // the tensor-core path needs no digit records
-    cudaError_t e = tc ? cudaSuccess : launch_act_digits(a, st);
+    // the tensor-core path needs no digit records; the decode GEMV builds its own
+    const bool tc = ffn_use_tc(a), own_records = tc || g2_use(a);
+    cudaError_t e = own_records ? cudaSuccess : launch_act_digits(a, st);
     if (e != cudaSuccess || !mark(1)) return QRX_ECUDA;
     // 2.. the rest chained with programmatic dependent launch (the first kernel
     // of the call never is: it must follow whatever the stream held before)
-    PdlScope pdl(!tc);
+    PdlScope pdl(!own_records);
     if ((v = route_impl(c, x, T, Wr, bias, topk_idx, topk_w, ws, ws_bytes, stream, topp_thr))) return v;
     g_pdl = true;
     if (!mark(2)) return QRX_ECUDA;
@@ -604,21 +654,14 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 
-std::mutex g_noalloc_mu;
-void *g_noalloc_addr[kMaxDevices] = {nullptr};
-
+// The array's device address in the current device's context.  Looked up on
+// every call: the lookup allocates nothing, and a cached address could be
+// stale after cudaDeviceReset or in another context on the same device.
 int noalloc_scratch(void **out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return QRX_ECUDA;
-    if (dev < 0 || dev >= kMaxDevices) return QRX_EUNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QRX_ECUDA;
-        g_noalloc_addr[dev] = p;
-    }
-    *out = g_noalloc_addr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QRX_ECUDA;
+    *out = p;
     return QRX_OK;
 }
 

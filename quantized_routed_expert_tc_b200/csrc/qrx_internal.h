@@ -63,15 +63,21 @@ cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const qrx_pe
                            cudaStream_t st, uint64_t *usage = nullptr);
 cudaError_t launch_usage_add(const int32_t *counts, int E, uint64_t *usage, cudaStream_t st);
 
-// expert FFN over the union (GEMV-shaped kernels)
+// One packed matrix of every expert: expert e's codes at q + e*sq bytes,
+// its row scales at s + e*ss floats (qrx_mat).
+struct MatRef {
+    const uint8_t *q;
+    const float *s;
+    int64_t sq, ss;
+};
+
+// expert FFN over the union
 struct FfnArgs {
     int wbits, afmt;
     int H, I, E, k, T;
-    // routed experts (may be null if !routed), shared expert (may be null)
-    const uint8_t *w13, *w2;
-    const float *s13, *s2;
-    const uint8_t *w13_sh, *w2_sh;
-    const float *s13_sh, *s2_sh;
+    // routed experts (unused if !routed), shared expert (unused if !shared)
+    MatRef gate, up, down;
+    MatRef gate_sh, up_sh, down_sh;
     int routed, shared;
     const int32_t *offsets, *sorted, *union_ids, *n_union;
     // activations
@@ -98,6 +104,10 @@ cudaError_t launch_ffn_tc_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
 cudaError_t launch_ffn_tc_down(const FfnArgs &a, int num_sms, cudaStream_t st);
 cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st);
 cudaError_t launch_ffn_down(const FfnArgs &a, int num_sms, cudaStream_t st);
+// decode GEMV (T <= 4): whether it takes this call, and its launches
+bool g2_use(const FfnArgs &a);
+cudaError_t launch_g2_gateup(const FfnArgs &a, int num_sms, cudaStream_t st, int32_t *probe = nullptr);
+cudaError_t launch_g2_down(const FfnArgs &a, int num_sms, cudaStream_t st, int32_t *probe = nullptr);
 
 cudaError_t launch_combine(const float *y_sorted, const float *y_sh, const float *w,
                            const int32_t *inv, int T, int k, int H, float *out,

@@ -39,9 +39,15 @@ class Cfg(ctypes.Structure):
                 ("afmt", ctypes.c_int32)]
 
 
+class CMat(ctypes.Structure):
+    """qrx_mat: one packed matrix of every expert."""
+    _fields_ = [("q", ctypes.c_void_p), ("scale", ctypes.c_void_p),
+                ("expert_stride_q", ctypes.c_int64), ("expert_stride_s", ctypes.c_int64)]
+
+
 class CExperts(ctypes.Structure):
-    _fields_ = [("w13", ctypes.c_void_p), ("s13", ctypes.c_void_p), ("w2", ctypes.c_void_p),
-                ("s2", ctypes.c_void_p)]
+    """qrx_experts: the gate, up and down matrices of an expert set."""
+    _fields_ = [("gate", CMat), ("up", CMat), ("down", CMat)]
 
 
 class COpts(ctypes.Structure):
@@ -81,6 +87,10 @@ _SIGS = {
     "qrx_expert_ffn_noalloc": ([P(Cfg), P(CExperts), P(CPerm), P(CAct), i32, vp, vp],
                                ctypes.c_int),
     "qrx_expert_down": ([P(Cfg), P(CExperts), P(CPerm), vp, i32, vp, vp, sz, vp], ctypes.c_int),
+    "qrx_expert_gateup_q8_sums": ([P(Cfg), P(CExperts), P(CPerm), P(CAct), i32, vp, vp, vp, sz, vp],
+                                  ctypes.c_int),
+    "qrx_expert_down_q8_sums": ([P(Cfg), P(CExperts), P(CPerm), vp, i32, vp, vp, vp, sz, vp],
+                                ctypes.c_int),
     "qrx_shared_ffn": ([P(Cfg), P(CExperts), P(CAct), i32, vp, vp, vp, sz, vp], ctypes.c_int),
     "qrx_combine": ([P(Cfg), vp, vp, vp, vp, i32, vp, vp], ctypes.c_int),
     "qrx_moe_forward": ([P(Cfg), vp, i32, vp, vp, P(CExperts), P(CExperts), vp, vp, vp, vp, sz,
@@ -155,18 +165,28 @@ def cfg_of(w) -> Cfg:
 
 @dataclass
 class Experts:
-    """Packed experts on the device (layout of include/qrx.h)."""
-    w13: torch.Tensor    # [n, 2I, H*b/8] uint8
-    s13: torch.Tensor    # [n, 2I] f32
-    w2: torch.Tensor     # [n, H, I*b/8] uint8
-    s2: torch.Tensor     # [n, H] f32
+    """Packed experts on the device (layout of include/qrx.h): three matrices,
+    each [n][rows][K*b/8] uint8 with row scales [n][rows] f32."""
+    gate: torch.Tensor     # [n, I, H*b/8] uint8
+    gate_s: torch.Tensor   # [n, I] f32
+    up: torch.Tensor       # [n, I, H*b/8] uint8
+    up_s: torch.Tensor     # [n, I] f32
+    down: torch.Tensor     # [n, H, I*b/8] uint8
+    down_s: torch.Tensor   # [n, H] f32
+
+    @staticmethod
+    def _cmat(q, s) -> CMat:
+        if q.dim() != 3 or s.dim() != 2 or q.stride(2) != 1 or q.stride(1) != q.shape[2] or s.stride(1) != 1:
+            raise ValueError("expert matrices must have contiguous rows and scales")
+        return CMat(q.data_ptr(), s.data_ptr(), q.stride(0) * q.element_size(), s.stride(0))
 
     def c(self) -> CExperts:
         """The qrx_experts struct of these tensors, built once: a call passes it
-        without rebuilding it, and assigning any of the four tensors drops it."""
+        without rebuilding it, and assigning any of the six tensors drops it."""
         cs = self.__dict__.get("_cstruct")
         if cs is None:
-            cs = CExperts(_p(self.w13), _p(self.s13), _p(self.w2), _p(self.s2))
+            cs = CExperts(self._cmat(self.gate, self.gate_s), self._cmat(self.up, self.up_s),
+                          self._cmat(self.down, self.down_s))
             self.__dict__["_cstruct"] = cs
         return cs
 
@@ -176,13 +196,19 @@ class Experts:
 
     @staticmethod
     def empty(n: int, H: int, I: int, wbits: int, device="cuda") -> "Experts":
-        return Experts(torch.empty((n, 2 * I, H * wbits // 8), dtype=torch.uint8, device=device),
-                       torch.empty((n, 2 * I), dtype=torch.float32, device=device),
-                       torch.empty((n, H, I * wbits // 8), dtype=torch.uint8, device=device),
-                       torch.empty((n, H), dtype=torch.float32, device=device))
+        u8, f32 = torch.uint8, torch.float32
+        return Experts(torch.empty((n, I, H * wbits // 8), dtype=u8, device=device),
+                       torch.empty((n, I), dtype=f32, device=device),
+                       torch.empty((n, I, H * wbits // 8), dtype=u8, device=device),
+                       torch.empty((n, I), dtype=f32, device=device),
+                       torch.empty((n, H, I * wbits // 8), dtype=u8, device=device),
+                       torch.empty((n, H), dtype=f32, device=device))
+
+    def tensors(self):
+        return (self.gate, self.gate_s, self.up, self.up_s, self.down, self.down_s)
 
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in (self.w13, self.s13, self.w2, self.s2))
+        return sum(t.numel() * t.element_size() for t in self.tensors())
 
 
 @dataclass
@@ -279,7 +305,7 @@ def qrx_expert_ffn(cfg, routed: Experts, perm: Perm, T, y_sorted, ws, x=None, xq
 
 def qrx_expert_ffn_noalloc(cfg, routed: Experts, perm: Perm, T, y_sorted, x=None, xq=None,
                            xd=None, stream=None):
-    """qrx_expert_ffn with no caller workspace (the library's fixed 4 MiB array)."""
+    """qrx_expert_ffn with no caller workspace (the library's fixed 8 MiB array)."""
     _check("qrx_expert_ffn_noalloc", lib().qrx_expert_ffn_noalloc(
         ctypes.byref(cfg), ctypes.byref(routed.c()), ctypes.byref(perm.c()),
         ctypes.byref(_act(cfg, x, xq, xd)), T, _p(y_sorted), _st(stream)))
@@ -289,6 +315,25 @@ def qrx_expert_down(cfg, routed: Experts, perm: Perm, h_sorted, T, y_sorted, ws,
     _check("qrx_expert_down", lib().qrx_expert_down(
         ctypes.byref(cfg), ctypes.byref(routed.c()), ctypes.byref(perm.c()), _p(h_sorted), T,
         _p(y_sorted), _p(ws), ws.numel(), _st(stream)))
+
+
+def qrx_expert_gateup_q8_sums(cfg, routed: Experts, perm: Perm, T, h_sorted, acc, ws, xq, xd,
+                              stream=None):
+    """Gate/up of the routed FFN (Q8_0, T <= 4) with its int32 block accumulators
+    acc [T*k, 2, I, H/32]."""
+    _check("qrx_expert_gateup_q8_sums", lib().qrx_expert_gateup_q8_sums(
+        ctypes.byref(cfg), ctypes.byref(routed.c()), ctypes.byref(perm.c()),
+        ctypes.byref(_act(cfg, None, xq, xd)), T, _p(h_sorted), _p(acc), _p(ws), ws.numel(),
+        _st(stream)))
+
+
+def qrx_expert_down_q8_sums(cfg, routed: Experts, perm: Perm, h_sorted, T, y_sorted, acc, ws,
+                            stream=None):
+    """Down of the routed FFN from a given h (Q8_0, T <= 4) with its int32 block
+    accumulators acc [T*k, H, I/32]."""
+    _check("qrx_expert_down_q8_sums", lib().qrx_expert_down_q8_sums(
+        ctypes.byref(cfg), ctypes.byref(routed.c()), ctypes.byref(perm.c()), _p(h_sorted), T,
+        _p(y_sorted), _p(acc), _p(ws), ws.numel(), _st(stream)))
 
 
 def qrx_shared_ffn(cfg, shared: Experts, T, y_sh, ws, x=None, xq=None, xd=None, h_sh=None,
@@ -369,12 +414,6 @@ def qrx_moe_forward_hostio(cfg, x_host, Wr, bias, routed: Experts, shared: Exper
 def quantize_expert_into(ex: Experts, e: int, gate: torch.Tensor, up: torch.Tensor,
                          down: torch.Tensor, wbits: int, stream=None) -> None:
     """Quantise one expert's f32 gate [I,H], up [I,H], down [H,I] (device tensors)
-    into slot e of `ex`: gate rows to the even rows of w13, up rows to the odd rows."""
-    I, H = gate.shape
-    rb13 = ex.w13.shape[2]
-    w13 = ex.w13[e]
-    s13 = ex.s13[e]
-    qrx_quantize_weights(gate, wbits, w13.data_ptr(), 2 * rb13, s13.data_ptr(), 2, stream)
-    qrx_quantize_weights(up, wbits, w13.data_ptr() + rb13, 2 * rb13, s13.data_ptr() + 4, 2, stream)
-    qrx_quantize_weights(down, wbits, ex.w2[e].data_ptr(), ex.w2.shape[2], ex.s2[e].data_ptr(), 1,
-                         stream)
+    into slot e of `ex` with the library's per-row quantiser."""
+    for w, q, sc in ((gate, ex.gate, ex.gate_s), (up, ex.up, ex.up_s), (down, ex.down, ex.down_s)):
+        qrx_quantize_weights(w, wbits, q[e].data_ptr(), q.shape[2], sc[e].data_ptr(), 1, stream)

@@ -174,6 +174,64 @@ def test_block_dots_bitexact(dev, bits):
         assert np.array_equal(np_(acc), acc_ref)
 
 
+# ------------------------------------------------------------------ exact Q8_0 accumulators
+def _q8_block_sums_case(glay, olay, wl, batch):
+    """The decode engine's int32 block accumulators of gate/up (from the
+    library's Q8_0 codes of x, which equal the oracle's) and of down (from the
+    oracle's h, re-quantised by the kernel) against the oracle's exact sums."""
+    T, k, H, I, bits = wl.T, wl.top_k, wl.hidden, wl.inter, wl.wbits
+    x = activations(wl, T, batch=batch)
+    _, bias = router_weights(wl)
+    r = oracle.router(wl, x, olay.Wr, bias)
+    p = oracle.permute(r["idx"], wl.n_experts)
+    xq_o, xd_o = oracle.quantize_q8(x)
+    ex = olay.experts(r["idx"].ravel(), bits)
+    h_o, _ = oracle.expert_ffn(wl, ex, p, x)
+    c = qrx.cfg_of(wl)
+    ws = qrx.workspace(c, T)
+    perm = qrx.Perm.empty(T, k, wl.n_experts)
+    qrx.qrx_permute(c, cu(r["idx"]), perm)
+    xq = torch.empty((T, H), dtype=torch.int8, device="cuda")
+    xd = torch.empty((T, H // 32), dtype=torch.float32, device="cuda")
+    qrx.qrx_quantize_act_q8(cu(x), xq, xd)
+    A = T * k
+    hs = torch.empty((A, I), dtype=torch.float32, device="cuda")
+    acc_gu = torch.full((A, 2, I, H // 32), -7, dtype=torch.int32, device="cuda")
+    qrx.qrx_expert_gateup_q8_sums(c, glay.routed[bits], perm, T, hs, acc_gu, ws, xq, xd)
+    ys = torch.empty((A, H), dtype=torch.float32, device="cuda")
+    acc_d = torch.full((A, H, I // 32), -7, dtype=torch.int32, device="cuda")
+    qrx.qrx_expert_down_q8_sums(c, glay.routed[bits], perm, cu(h_o), T, ys, acc_d, ws)
+    torch.cuda.synchronize()
+    assert qrx.qrx_last_error() == qrx.QRX_OK
+    assert np.array_equal(np_(xq), xq_o) and np.array_equal(np_(xd), xd_o)
+    acc_gu, acc_d = np_(acc_gu), np_(acc_d)
+    flat = r["idx"].ravel()
+    for pos in range(A):
+        a = int(p["sorted"][pos])
+        e, t = int(flat[a]), a // k
+        o = ex[e]
+        assert np.array_equal(acc_gu[pos, 0], oracle.block_dots_q8(o.gate_q, H, bits, xq_o[t])), (pos, "gate")
+        assert np.array_equal(acc_gu[pos, 1], oracle.block_dots_q8(o.up_q, H, bits, xq_o[t])), (pos, "up")
+        hq, _ = oracle.quantize_q8(h_o[pos:pos + 1])
+        assert np.array_equal(acc_d[pos], oracle.block_dots_q8(o.down_q, I, bits, hq[0])), (pos, "down")
+    assert rel_err(np_(hs), h_o) <= TOL
+
+
+@pytest.mark.parametrize("bits", [8, 4, 2])
+@pytest.mark.parametrize("T", [1, 4])
+def test_q8_block_sums_bitexact_tiny(tiny, bits, T):
+    glay, olay = tiny
+    _q8_block_sums_case(glay, olay, W.TINY.with_(wbits=bits, afmt=W.A_Q8, T=T), 40 + T)
+
+
+@pytest.mark.parametrize("bits", [8, 4, 2])
+@pytest.mark.parametrize("T", [1, 4])
+def test_q8_block_sums_bitexact_glm(glm, bits, T):
+    """At the GLM shape: 2I x 192 gate/up and H x 64 down block sums per position."""
+    glay, olay = glm
+    _q8_block_sums_case(glay, olay, W.GLM_DECODE_T1.with_(wbits=bits, afmt=W.A_Q8, T=T), 50 + T)
+
+
 # ------------------------------------------------------------------ router and permutation
 def _route_gpu(glay, wl, x_np, bias_np):
     c = qrx.cfg_of(wl)
@@ -504,9 +562,10 @@ def test_glm_decode_t1(glm):
 
 
 def test_glm_decode_t32_q8(glm):
+    """Every token of the skewed 32-token Q8_0 batch."""
     glay, olay = glm
     wl = W.GLM_DECODE_T32_Q8
-    res = check_layer(glay, olay, wl, activations(wl), [0, 13, 31])
+    res = check_layer(glay, olay, wl, activations(wl), range(32))
     n_union = len(np.unique(res["idx"]))
     assert n_union < 256                       # skewed bias: the union is below E
 
@@ -516,7 +575,7 @@ def test_glm_decode_t32_q8_topp(glm):
     glay, olay = glm
     wl = W.GLM_DECODE_T32_Q8
     x = activations(wl)
-    res = check_layer(glay, olay, wl, x, [0, 13, 31], topp=0.7)
+    res = check_layer(glay, olay, wl, x, range(32), topp=0.7)
     idx0, _, _ = gpu_layer(glay, wl, x)
     nu_p = len(np.unique(res["idx"][res["idx"] >= 0]))
     assert nu_p < len(np.unique(idx0))
@@ -529,16 +588,20 @@ def test_glm_verify_t4_bf16(glm):
 
 
 def test_glm_prefill_t2048_bf16(glm):
+    """128 tokens spread over the 2048-token batch (every 16th, and the last): on
+    the tensor-core engine each expert's token tiles are hit, on the ~1,100 work
+    items that 148 persistent CTAs take about seven at a time, so every CTA's
+    later items (second accumulator buffer, later ring phases) are compared."""
     glay, olay = glm
     wl = W.GLM_PREFILL_T2048_BF16
-    check_layer(glay, olay, wl, activations(wl), [0, 1031, 2047])
+    check_layer(glay, olay, wl, activations(wl), list(range(0, 2048, 16)) + [2047])
 
 
 @pytest.mark.parametrize("wl", W.sweep(), ids=lambda w: w.name)
 def test_glm_sweep(glm, wl):
+    """Every token of each format-sweep batch (1 or 64 tokens)."""
     glay, olay = glm
-    toks = [0] if wl.T == 1 else [0, wl.T - 1]
-    check_layer(glay, olay, wl, activations(wl), toks, bits=wl.wbits)
+    check_layer(glay, olay, wl, activations(wl), range(wl.T), bits=wl.wbits)
 
 
 def test_glm_all_tokens_one_expert_set(glm):
