@@ -371,8 +371,11 @@ int qrx_moe_forward_opts(const qrx_cfg *cfg, const void *x, int32_t T, const flo
 
 /* qrx_moe_forward with stage timing: events[0..6] are cudaEvent_t handles
  * (passed as void*) recorded on `stream` before the activation-record
- * kernel, after it, after the router, after the permutation, after the
- * gate/up kernel, after the down kernel and after the combine.  n_events must
+ * kernel, after it (the two coincide when the expert engine builds its own
+ * records), after the router, after the permutation, after the gate/up
+ * kernel, after the down kernel and after the combine.  For batches of up to
+ * 32 tokens the expert selection runs in the permutation's kernel, so
+ * "router" is the logits kernel and "permutation" the selection with it.  n_events must
  * be 7.  The events separate the kernels, so the launch overlap that
  * qrx_moe_forward gets from programmatic dependent launch is lost here: the
  * stage times add up to more than a plain call takes.  opts as in

@@ -225,28 +225,37 @@ __device__ __forceinline__ TcItem tc_decode(const TcP &p, const int64_t *pre, in
 
 // Bounded wait that also gives up (false, no new status) once another role
 // has raised the abort flag; on its own timeout it raises both.  Roles off
-// the MMA's critical path poll with a sleep in between (sleep_ns > 0), which
-// leaves the issue slots of their SM sub-partition to the warps that work.
+// the MMA's critical path (park = true) are parked by the barrier itself: each
+// try_wait carries a suspend-time hint, so the warp sleeps until the phase
+// completes (or the hint runs out) and leaves the issue slots of its SM
+// sub-partition to the warps that work.  The MMA thread polls (park = false).
+constexpr uint32_t TC_PARK_NS = 1000;          // suspend hint of a parked poll
+constexpr long long TC_PARK_CAP = 1ll << 21;   // parked polls before a wait gives up
+
 __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                        unsigned sleep_ns = 0)
+                                        bool park = false)
 {
     const uint32_t a = smem_u32(bar);
-    for (long long it = 0; it < GV_WAIT_CAP; ++it) {
+    for (long long it = 0; it < (park ? TC_PARK_CAP : GV_WAIT_CAP); ++it) {
         uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(a), "r"(parity)
-            : "memory");
+        if (park)
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(done)
+                : "r"(a), "r"(parity), "r"(TC_PARK_NS)
+                : "memory");
+        else
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(done)
+                : "r"(a), "r"(parity)
+                : "memory");
         if (done) return true;
-        if (sleep_ns) {
-            __nanosleep(sleep_ns);
-            if (*abort_flag) return false;
-        } else if ((it & 255) == 255 && *abort_flag) {
-            return false;
-        }
+        if ((park || (it & 255) == 255) && *abort_flag) return false;
     }
     *abort_flag = 1;
     raise_status(DERR_TIMEOUT);
@@ -282,10 +291,10 @@ __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t da, uint64_t db, uin
 // tc_wait for a whole warp: lane 0 polls (one shared-memory request per poll
 // instead of 32) and broadcasts the outcome.
 __device__ __forceinline__ bool tc_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             unsigned sleep_ns = 0)
+                                             bool park = false)
 {
     int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = tc_wait(bar, parity, abort_flag, sleep_ns) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = tc_wait(bar, parity, abort_flag, park) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -408,7 +417,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int kb = 0; kb < p.kstages; ++kb) {
                     if (kb % TC_RK == 0) {
                         const uint32_t rs = rg % TC_RS;
-                        if (rg >= TC_RS && !tc_wait(&raw_empty[(rs) * TC_BS], ((rg / TC_RS) - 1) & 1, abort_flag, 64)) {
+                        if (rg >= TC_RS && !tc_wait(&raw_empty[(rs) * TC_BS], ((rg / TC_RS) - 1) & 1, abort_flag, true)) {
                             ok = false;
                             break;
                         }
@@ -422,7 +431,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         ++rg;
                     }
                     const uint32_t sb = g % TC_S;
-                    if (g >= TC_S && !tc_wait(&empty[(sb) * TC_BS], ((g / TC_S) - 1) & 1, abort_flag, 64)) {
+                    if (g >= TC_S && !tc_wait(&empty[(sb) * TC_BS], ((g / TC_S) - 1) & 1, abort_flag, true)) {
                         ok = false;
                         break;
                     }
@@ -515,7 +524,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const float sc0 = sb0[r0], sc1 = sb1[r1];
             const int64_t orow0 = d.routed ? d.b0 : p.sh_out_row0 + d.n0;
             const int a = local & 1;
-            if (!tc_wait_warp(&acc_full[(a) * TC_BS], (local >> 1) & 1, abort_flag, 256)) break;
+            if (!tc_wait_warp(&acc_full[(a) * TC_BS], (local >> 1) & 1, abort_flag, true)) break;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             // 32 accumulator columns (tokens c0..c0+31) of half hf for this thread's row
             auto ld32 = [&](int hf, int c0, uint32_t (&v)[32]) {
@@ -586,12 +595,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         for (int64_t it = blockIdx.x; ok && it < nitems && !*abort_flag; it += gridDim.x) {
             for (int kb = 0; kb < p.kstages; ++kb) {
                 const uint32_t rs = rg % TC_RS;
-                if (kb % TC_RK == 0 && !tc_wait_warp(&raw_full[(rs) * TC_BS], (rg / TC_RS) & 1, abort_flag, 32)) {
+                if (kb % TC_RK == 0 && !tc_wait_warp(&raw_full[(rs) * TC_BS], (rg / TC_RS) & 1, abort_flag, true)) {
                     ok = false;
                     break;
                 }
                 const uint32_t st = g % TC_S;
-                if (g >= TC_S && !tc_wait_warp(&empty[(st) * TC_BS], ((g / TC_S) - 1) & 1, abort_flag, 32)) {
+                if (g >= TC_S && !tc_wait_warp(&empty[(st) * TC_BS], ((g / TC_S) - 1) & 1, abort_flag, true)) {
                     ok = false;
                     break;
                 }

@@ -47,12 +47,13 @@
 
 namespace qrx {
 
-constexpr int G2_NW = 8;                          // compute warps
+constexpr int G2_NW = 11;                         // compute warps (3 warps per SM sub-partition in all)
 constexpr int G2_THREADS = 32 * (G2_NW + 1);      // + the producer warp
 constexpr int G2_KS = 512;                        // bytes of a row per stage (at most)
 constexpr int G2_TMAX = 4;                        // tokens per call
 constexpr int G2_SMEM_MAX = 227 * 1024;
-constexpr long long G2_WAIT_CAP = 1ll << 22;      // polls before a wait gives up
+constexpr long long G2_WAIT_CAP = 1ll << 21;      // polls before a wait gives up
+constexpr uint32_t G2_SUSPEND_NS = 1000;          // a waiting thread sleeps up to this long per poll
 
 // ---------------------------------------------------------------- records
 // Record of one input row of K codes, in shared memory:
@@ -85,7 +86,7 @@ struct G2P {
     int ks, cps, nslice;             // bytes per slice, chunks per slice, slices per row
     int lpr, gpw, rw, rb, nrb;       // lanes per row, row groups per warp, rows per warp, rows per unit, units per slot
     int box_rows;                    // rows per TMA box (rb is a whole number of boxes)
-    int stages, stage_bytes, scale_off;
+    int stages, stage_bytes, scale_off, sc_stride;   // sc_stride: floats from matrix 0's scales to matrix 1's
     int rec_bytes, rec_off, nrec;    // record size, smem offset, records held
     int bar_off, pre_off, red_off, smem;
     G2Mat m[2], msh[2];              // gate/up: m[0] gate, m[1] up; down: m[0] down
@@ -119,12 +120,31 @@ __device__ __forceinline__ bool g2_try(uint32_t mbar, uint32_t parity)
     return done != 0;
 }
 
+// dp4a of unsigned weight bytes by signed digit bytes (the int4 high halves
+// are kept in place, as 16 x the code, so they need the unsigned form).
+__device__ __forceinline__ int g2_dp4a_us(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
 // Bounded wait; false if it gave up or another role raised the abort flag.
+// Each poll may suspend the thread (up to G2_SUSPEND_NS) until the phase
+// completes, so a waiting warp takes no issue slots from the working ones.
 __device__ __forceinline__ bool g2_wait(uint32_t mbar, uint32_t parity, volatile int *abort_flag)
 {
     for (long long it = 0; it < G2_WAIT_CAP; ++it) {
-        if (g2_try(mbar, parity)) return true;
-        if ((it & 63) == 63 && *abort_flag) return false;
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(mbar), "r"(parity), "r"(G2_SUSPEND_NS)
+            : "memory");
+        if (done) return true;
+        if (*abort_flag) return false;
     }
     *abort_flag = 1;
     raise_status(DERR_TIMEOUT);
@@ -191,11 +211,51 @@ __device__ __forceinline__ void g2_tr_reduce(float (&v)[V], int lane)
 }
 
 // ---------------------------------------------------------------- record builder
+// Element values of one input row as the dot sees them, loaded 16 bytes at a
+// time: f32 rows (x, or h -- rounded to bf16 first for bf16 activations) or
+// bf16 rows (x).
+struct G2Row {
+    const void *base;     // the row
+    bool bf16_in;         // the row is bf16 (gate/up input with bf16 activations)
+    bool round_bf16;      // f32 values rounded to bf16 (down input with bf16 activations)
+
+    // values e0 .. e0 + 4*N - 1 (e0 a multiple of 4; of 8 for bf16 rows)
+    template <int N>
+    __device__ __forceinline__ void load(int e0, float (&v)[4 * N]) const
+    {
+        if (bf16_in) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(base) + e0);
+#pragma unroll
+            for (int i = 0; i < N / 2; ++i) {
+                const uint4 r = src[i];
+                const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    v[8 * i + 2 * q] = __uint_as_float(w[q] << 16);
+                    v[8 * i + 2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+                }
+            }
+        } else {
+            const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(base) + e0);
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const float4 r = src[i];
+                v[4 * i] = r.x;
+                v[4 * i + 1] = r.y;
+                v[4 * i + 2] = r.z;
+                v[4 * i + 3] = r.w;
+            }
+            if (round_bf16)
+#pragma unroll
+                for (int i = 0; i < 4 * N; ++i) v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+        }
+    }
+};
+
 // Build the records of `n` input rows into shared memory with all compute
-// threads (tid < G2_NW * 32).  Row i is row_of(i) of the input (x for gate/up,
-// h for down).  For bf16 activations h is rounded to bf16 here (x is given as
-// bf16).  `scr` is 64 bytes of scratch; `cb`/`ph` the compute barrier.
-// Returns false if a barrier wait gave up.
+// threads (tid < G2_NW * 32).  row_of(i) is row i's index in the input (x for
+// gate/up, h for down).  `scr` holds G2_NW floats of scratch; `cb`/`ph` the
+// compute barrier.  Returns false if a barrier wait gave up.
 template <int WB, int NDIG, typename RowFn>
 __device__ bool g2_build(const G2P &p, unsigned char *recs, int n, RowFn row_of, bool gateup, float *scr,
                          uint64_t *cb, uint32_t &ph, volatile int *abort_flag)
@@ -209,19 +269,21 @@ __device__ bool g2_build(const G2P &p, unsigned char *recs, int n, RowFn row_of,
     for (int i = 0; i < n; ++i) {
         const int64_t row = row_of(i);
         unsigned char *rec = recs + (size_t)i * p.rec_bytes;
-        // element e of the row as the dot sees it
-        auto val = [&](int e) -> float {
-            if (gateup) {
-                if (bf) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.x)[row * p.in_ld + e]);
-                return reinterpret_cast<const float *>(p.x)[row * p.in_ld + e];
-            }
-            const float h = reinterpret_cast<const float *>(p.x)[row * p.in_ld + e];
-            return bf ? __bfloat162float(__float2bfloat16_rn(h)) : h;
-        };
+        G2Row src;
+        src.bf16_in = gateup && bf;
+        src.round_bf16 = !gateup && bf;
+        src.base = src.bf16_in ? static_cast<const void *>(static_cast<const __nv_bfloat16 *>(p.x) + row * p.in_ld)
+                               : static_cast<const void *>(static_cast<const float *>(p.x) + row * p.in_ld);
         if constexpr (NDIG == 3) {
-            // the row's largest magnitude -> shift s (sigma = 2^-s)
+            // the row's largest magnitude -> shift s (sigma = 2^-s); 8 values per load step
             float am = 0.f;
-            for (int e = tid; e < K; e += nth) am = fmaxf(am, fabsf(val(e)));
+#pragma unroll 4
+            for (int e = tid * 8; e < K; e += nth * 8) {
+                float v[8];
+                src.load<2>(e, v);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) am = fmaxf(am, fabsf(v[q]));
+            }
             am = warp_max(am);
             if ((tid & 31) == 0) scr[tid >> 5] = am;
             if (!g2_cbar(cb, ph, abort_flag)) return false;
@@ -232,6 +294,8 @@ __device__ bool g2_build(const G2P &p, unsigned char *recs, int n, RowFn row_of,
             const bool fast = sh >= -126 && sh <= 127;
             const float mul = fast ? __int_as_float((sh + 127) << 23) : 0.f;
             for (int c = tid; c < cpr; c += nth) {
+                float v[EPC];
+                src.load<EPC / 4>(c * EPC, v);
                 uint32_t wd[3][DW];
 #pragma unroll
                 for (int wi = 0; wi < 4; ++wi)
@@ -240,9 +304,9 @@ __device__ bool g2_build(const G2P &p, unsigned char *recs, int n, RowFn row_of,
                         uint32_t b0 = 0, b1 = 0, b2 = 0;
 #pragma unroll
                         for (int by = 0; by < 4; ++by) {
-                            const float v = val(c * EPC + elem_in_chunk<WB>(wi, j, by));
+                            const float x = v[elem_in_chunk<WB>(wi, j, by)];
                             int8_t d0 = 0, d1 = 0, d2 = 0;
-                            if (am != 0.f) split3(__float2int_rn(fast ? __fmul_rn(v, mul) : ldexpf(v, sh)), d0, d1, d2);
+                            if (am != 0.f) split3(__float2int_rn(fast ? __fmul_rn(x, mul) : ldexpf(x, sh)), d0, d1, d2);
                             b0 |= (uint32_t)(uint8_t)d0 << (8 * by);
                             b1 |= (uint32_t)(uint8_t)d1 << (8 * by);
                             b2 |= (uint32_t)(uint8_t)d2 << (8 * by);
@@ -278,17 +342,18 @@ __device__ bool g2_build(const G2P &p, unsigned char *recs, int n, RowFn row_of,
                     float dq = 0.f;
                     int csum = 0;
                     if (gateup && p.xq) {         // codes and scales from qrx_quantize_act_q8
+                        const uint4 *qs = reinterpret_cast<const uint4 *>(p.xq + row * p.in_ld + b * 32);
+                        const uint4 q0 = qs[0], q1 = qs[1];
+                        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-                        for (int l = 0; l < 32; ++l) code[bb * 32 + l] = p.xq[row * p.in_ld + b * 32 + l];
+                        for (int l = 0; l < 32; ++l) code[bb * 32 + l] = (int8_t)(w[l >> 2] >> (8 * (l & 3)));
                         dq = p.xd[row * (p.in_ld / 32) + b];
-                    } else {                      // the same Q8_0 formula on f32 values
+                    } else {                      // the same Q8_0 formula on the values
                         float v[32];
+                        src.load<8>(b * 32, v);
                         float am = 0.f;
 #pragma unroll
-                        for (int l = 0; l < 32; ++l) {
-                            v[l] = val(b * 32 + l);
-                            am = fmaxf(am, fabsf(v[l]));
-                        }
+                        for (int l = 0; l < 32; ++l) am = fmaxf(am, fabsf(v[l]));
                         const float f = am != 0.f ? __fdiv_rn(127.f, am) : 0.f;
 #pragma unroll
                         for (int l = 0; l < 32; ++l) code[bb * 32 + l] = (int8_t)(am != 0.f ? q8_code(v[l], f) : 0);
@@ -379,7 +444,12 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
     using F = Fmt<WB>;
     constexpr int NM = GATEUP ? 2 : 1;
     constexpr int DW = F::DW, NQ = DW / 4, UPW = F::UPW;
-    constexpr int NP = NDIG == 3 ? 3 : 1;                 // integer accumulators per (token, row)
+    constexpr int NP = NDIG == 3 ? 3 : 1;                 // planes accumulated per (token, row)
+    // int4: each packed word is split by one LOP3 per half -- low nibbles as
+    // they are, high nibbles left in place (16 x the code) -- and the two halves
+    // sum into separate exact accumulators, the second divided by 16 at the end
+    constexpr bool HI16 = WB == 4;
+    constexpr int NA = HI16 ? 2 : 1;
     constexpr int NBC = WB == 2 ? 2 : 1;                 // Q8_0 blocks a chunk touches
     constexpr int V = TP * NM * R;                        // values a lane reduces per unit
     // int2 or many tokens: every token's digits at once would not fit in registers
@@ -394,7 +464,24 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
     unsigned char *recs = sm + p.rec_off;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        for (int st = 0; st < p.stages; ++st) {
+            mbar_init(g2_smem(&full[st]), 1);
+            mbar_init(g2_smem(&empty[st]), G2_NW);
+        }
+        mbar_init(g2_smem(cbar), G2_NW);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    uint32_t cph = 0;      // compute-barrier phase (compute warps)
+    bool built = true;
     if constexpr (GATEUP) {
+        // the records of every token, before the dependency wait: x is an input
+        // of the call, so this overlaps the kernels that route
+        if (warp < G2_NW)
+            built = g2_build<WB, NDIG>(p, recs, p.T, [](int i) -> int64_t { return i; }, true, scr, cbar, cph,
+                                       abort_flag);
         pdl_wait();        // the permutation comes from the kernels before
         pdl_trigger();
     }
@@ -423,15 +510,6 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
             run += __shfl_sync(0xffffffffu, inc, 31);
         }
         if (lane == 0) pre[nslots] = run;
-    }
-    if (tid == 0) {
-        for (int st = 0; st < p.stages; ++st) {
-            mbar_init(g2_smem(&full[st]), 1);
-            mbar_init(g2_smem(&empty[st]), G2_NW);
-        }
-        mbar_init(g2_smem(cbar), G2_NW);
-        *abort_flag = 0;
-        fence_mbar_init();
     }
     __syncthreads();
     const int64_t Ctot = pre[nslots];
@@ -471,6 +549,9 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
             const float *S1 = routed ? p.m[NM - 1].s + (int64_t)e * p.m[NM - 1].ss : p.msh[NM - 1].s;
             const int r0 = (int)(u.u * p.rb);
             const int nr = min(p.rb, p.rows - r0);
+            // the unit's row scales, copied from the 16-byte boundary at or below
+            // row r0 (rows is a multiple of 64, so the rounded-up end stays inside)
+            const int s0 = r0 & ~3, sn = ((r0 + nr + 3) & ~3) - s0;
             for (int j = 0; j < p.nslice; ++j) {
                 const uint32_t st = g % p.stages;
                 if (g >= (uint32_t)p.stages && !g2_wait(g2_smem(&empty[st]), ((g / p.stages) - 1) & 1, abort_flag)) {
@@ -478,7 +559,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                     break;
                 }
                 const bool last = j == p.nslice - 1;
-                const uint32_t bytes = (uint32_t)(NM * p.rb * p.ks + (last ? NM * nr * 4 : 0));
+                const uint32_t bytes = (uint32_t)(NM * p.rb * p.ks + (last ? NM * sn * 4 : 0));
                 const uint32_t fb = g2_smem(&full[st]);
                 asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb), "r"(bytes) : "memory");
                 unsigned char *dst = sm + (size_t)st * p.stage_bytes;
@@ -490,8 +571,9 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                                     z, fb);
                 }
                 if (last) {
-                    bulk_copy(g2_smem(dst + p.scale_off), S0 + r0, (uint32_t)(nr * 4), fb);
-                    if constexpr (NM == 2) bulk_copy(g2_smem(dst + p.scale_off + p.rb * 4), S1 + r0, (uint32_t)(nr * 4), fb);
+                    bulk_copy(g2_smem(dst + p.scale_off), S0 + s0, (uint32_t)(sn * 4), fb);
+                    if constexpr (NM == 2)
+                        bulk_copy(g2_smem(dst + p.scale_off + p.sc_stride * 4), S1 + s0, (uint32_t)(sn * 4), fb);
                 }
                 ++g;
             }
@@ -511,14 +593,10 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
     // ======================== compute warps ========================
     const int LPR = p.lpr;
     const int c = lane % LPR, grp = lane / LPR;
-    uint32_t cph = 0;      // compute-barrier phase
     QRX_CHECK_ONLY(const int64_t n_pos = p.routed ? (int64_t)p.T * p.k : 0;)
     QRX_CHECK_ONLY(const int64_t n_out = max(n_pos, p.shared ? p.sh_out_row0 + p.T : (int64_t)0);)
-    if constexpr (GATEUP) {
-        // the records of every token, once (x is an input of the call)
-        if (!g2_build<WB, NDIG>(p, recs, p.T, [](int i) -> int64_t { return i; }, true, scr, cbar, cph, abort_flag))
-            return;
-    } else {
+    if (!built) return;
+    if constexpr (!GATEUP) {
         pdl_wait();        // h comes from the kernel before
         pdl_trigger();
     }
@@ -607,7 +685,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
             cur_s = u.s;
         }
         // ---- one unit: nslice stages
-        int iacc[TP][NM][R][NP];
+        int iacc[TP][NM][R][NP][NA];
         float facc[TP][NM][R];
 #pragma unroll
         for (int t = 0; t < TP; ++t)
@@ -617,7 +695,9 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                 for (int i = 0; i < R; ++i) {
                     facc[t][m][i] = 0.f;
 #pragma unroll
-                    for (int pl = 0; pl < NP; ++pl) iacc[t][m][i][pl] = 0;
+                    for (int pl = 0; pl < NP; ++pl)
+#pragma unroll
+                        for (int h = 0; h < NA; ++h) iacc[t][m][i][pl][h] = 0;
                 }
         const int lrow0 = warp * p.rw + grp;             // this lane's first row in the unit (then + gpw)
         for (int j = 0; j < p.nslice; ++j, ++g) {
@@ -655,29 +735,33 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
             auto unpack = [&](int m, int i, uint32_t (&uw)[4][UPW]) {
                 const uint4 wv = *reinterpret_cast<const uint4 *>(
                     stg + ((size_t)(m * p.rb + lrow0 + p.gpw * i)) * p.ks + (size_t)c * 16);
-                unpack_word<WB>(wv.x, uw[0]);
-                unpack_word<WB>(wv.y, uw[1]);
-                unpack_word<WB>(wv.z, uw[2]);
-                unpack_word<WB>(wv.w, uw[3]);
+                const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                for (int wi = 0; wi < 4; ++wi) {
+                    if constexpr (HI16) {
+                        uw[wi][0] = (ww[wi] ^ 0x88888888u) & 0x0F0F0F0Fu;   // elements 0, 2, 4, 6 (code + 8)
+                        uw[wi][1] = (ww[wi] ^ 0x88888888u) & 0xF0F0F0F0u;   // elements 1, 3, 5, 7, x16
+                    } else {
+                        unpack_word<WB>(ww[wi], uw[wi]);
+                    }
+                }
             };
             // one unpacked weight chunk against one token's digits
             auto dot = [&](int t, int m, int i, const uint32_t (&uw)[4][UPW], const uint32_t (&d)[NDIG][DW],
                            const float (&dq)[NBC], const int (&cb)[NBC]) {
                 if constexpr (NDIG == 3) {
-                    int a0 = iacc[t][m][i][0], a1 = iacc[t][m][i][1], a2 = iacc[t][m][i][2];
 #pragma unroll
                     for (int wi = 0; wi < 4; ++wi)
 #pragma unroll
-                        for (int jj = 0; jj < UPW; ++jj) {
-                            a0 = dp4a(uw[wi][jj], d[0][wi * UPW + jj], a0);
-                            a1 = dp4a(uw[wi][jj], d[1][wi * UPW + jj], a1);
-                            a2 = dp4a(uw[wi][jj], d[2][wi * UPW + jj], a2);
-                        }
-                    iacc[t][m][i][0] = a0;
-                    iacc[t][m][i][1] = a1;
-                    iacc[t][m][i][2] = a2;
+                        for (int jj = 0; jj < UPW; ++jj)
+#pragma unroll
+                            for (int pl = 0; pl < 3; ++pl) {
+                                int &a = iacc[t][m][i][pl][HI16 ? jj : 0];
+                                a = HI16 ? g2_dp4a_us(uw[wi][jj], d[pl][wi * UPW + jj], a)
+                                         : dp4a(uw[wi][jj], d[pl][wi * UPW + jj], a);
+                            }
                 } else {
-                    int ib[NBC];
+                    int ib[NBC], ibh = 0;
 #pragma unroll
                     for (int bc = 0; bc < NBC; ++bc) ib[bc] = cb[bc];
 #pragma unroll
@@ -685,8 +769,10 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
 #pragma unroll
                         for (int jj = 0; jj < UPW; ++jj) {
                             const int bc = WB == 2 ? (wi >> 1) : 0;
-                            ib[bc] = dp4a(uw[wi][jj], d[0][wi * UPW + jj], ib[bc]);
+                            if (HI16 && jj == 1) ibh = g2_dp4a_us(uw[wi][jj], d[0][wi * UPW + jj], ibh);
+                            else ib[bc] = dp4a(uw[wi][jj], d[0][wi * UPW + jj], ib[bc]);
                         }
+                    if constexpr (HI16) ib[0] += ibh >> 4;
                     // int8: a block is two chunks on lanes 2b, 2b+1
                     if constexpr (WB == 8) ib[0] += __shfl_xor_sync(0xffffffffu, ib[0], 1);
                     const bool mine = WB != 8 || (c & 1) == 0;
@@ -753,10 +839,14 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
 #pragma unroll
                         for (int m = 0; m < NM; ++m) {
                             float x;
-                            if constexpr (NDIG == 3)
-                                x = fmaf(65536.f, (float)(iacc[t][m][i][2] - corr[t][2]),
-                                         fmaf(256.f, (float)(iacc[t][m][i][1] - corr[t][1]),
-                                              (float)(iacc[t][m][i][0] - corr[t][0])));
+                            if constexpr (NDIG == 3) {
+                                int P[3];
+#pragma unroll
+                                for (int pl = 0; pl < 3; ++pl)
+                                    P[pl] = (HI16 ? iacc[t][m][i][pl][0] + (iacc[t][m][i][pl][NA - 1] >> 4)
+                                                  : iacc[t][m][i][pl][0]) - corr[t][pl];
+                                x = fmaf(65536.f, (float)P[2], fmaf(256.f, (float)P[1], (float)P[0]));
+                            }
                             else
                                 x = facc[t][m][i];
                             v[(t * R + i) * NM + m] = t < nt ? x : 0.f;
@@ -766,7 +856,8 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                 else if (LPR == 8) g2_tr_reduce<V, 8>(v, lane);
                 else if (LPR == 4) g2_tr_reduce<V, 4>(v, lane);
                 else if (LPR == 2) g2_tr_reduce<V, 2>(v, lane);
-                const float *scl = reinterpret_cast<const float *>(stg + p.scale_off);
+                // row scales of the unit, from the 16-byte boundary at or below its first row
+                const float *scl = reinterpret_cast<const float *>(stg + p.scale_off) + ((u.u * p.rb) & 3);
                 // total `tot` (and for gate/up the matching up total `upv`) of value idx
                 auto emit = [&](int idx, float tot, float upv) {
                     const int t = idx / (NM * R), i = (idx / NM) % R;
@@ -777,7 +868,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                     QRX_CHECK_OR(o >= 0 && o < n_out, return);
                     const float sg = NDIG == 3 ? g2_pick(sig, t) : 1.f;
                     if constexpr (GATEUP)
-                        p.out[o * p.out_ld + row] = silu_mul(scl[lrow] * (sg * tot), scl[p.rb + lrow] * (sg * upv));
+                        p.out[o * p.out_ld + row] = silu_mul(scl[lrow] * (sg * tot), scl[p.sc_stride + lrow] * (sg * upv));
                     else
                         p.out[o * p.out_ld + row] = scl[lrow] * (sg * tot);
                 };
@@ -814,10 +905,12 @@ static inline bool g2_plan(G2Plan &pl, int wbits, int ndig, int K, int rows, int
     p = G2P{};
     if (T < 1 || T > G2_TMAX) return false;
     pl.tp = T == 1 ? 1 : (T == 2 ? 2 : 4);
-    // rows per lane: accumulators are NDIG (or 1) x nm x R x TP
-    const int perrow = (ndig == 3 ? 3 : 1) * nm * pl.tp;
-    pl.r = 48 / perrow >= 8 ? 8 : (48 / perrow >= 4 ? 4 : 2);
-    if (nm == 2 && pl.r > 4) pl.r = 4;
+    // rows per lane R: the integer accumulators (3 planes, x2 for int4's split
+    // halves; Q8_0: one f32) x matrices x R x TP stay within 48 registers
+    const int perrow = (ndig == 3 ? 3 * (wbits == 4 ? 2 : 1) : 1) * nm * pl.tp;
+    const int rmax = nm == 2 ? 4 : 8;
+    pl.r = 1;
+    while (pl.r * 2 <= rmax && pl.r * 2 * perrow <= 48) pl.r *= 2;
     p.K = K;
     p.rows = rows;
     p.row_bytes = K * wbits / 8;
@@ -833,9 +926,16 @@ static inline bool g2_plan(G2Plan &pl, int wbits, int ndig, int K, int rows, int
     p.rw = pl.r * p.gpw;
     p.rb = G2_NW * p.rw;
     p.nrb = (rows + p.rb - 1) / p.rb;
-    p.box_rows = p.rb < 256 ? p.rb : 256;    // a TMA box spans at most 256 rows
+    if (rows % 4) return false;
+    // a TMA box spans at most 256 rows: rb is cut into equal boxes, each landing
+    // on a 128-byte boundary of shared memory
+    int nbox = (p.rb + 255) / 256;
+    while (p.rb % nbox) ++nbox;
+    p.box_rows = p.rb / nbox;
+    if ((p.box_rows * p.ks) % 128) return false;
     p.scale_off = nm * p.rb * p.ks;
-    p.stage_bytes = (p.scale_off + nm * p.rb * 4 + 127) & ~127;
+    p.sc_stride = (p.rb + 7) & ~3;           // rb + up to 3 leading rows, rounded to 16 bytes
+    p.stage_bytes = (p.scale_off + nm * p.sc_stride * 4 + 127) & ~127;
     p.rec_bytes = (g2_rec(ndig, K).bytes + 127) & ~127;
     p.nrec = nm == 2 ? T : pl.tp;        // gate/up: every token; down: one slot's rows
     const int fixed_tail = 128 /*barriers*/ + 256 /*scratch*/ + (maxslots + 2) * 8;
@@ -976,11 +1076,11 @@ static cudaError_t g2_dispatch(const G2Maps &M, const G2Plan &pl, int wbits, int
             QRX_G2(2, 1, 1, 8) QRX_G2(2, 1, 2, 8) QRX_G2(2, 1, 4, 8)
         }
     } else if constexpr (GU) {
-        QRX_G2(4, 3, 1, 4) QRX_G2(4, 3, 2, 4) QRX_G2(4, 3, 4, 2) QRX_G2(4, 1, 1, 4) QRX_G2(4, 1, 2, 4) QRX_G2(4, 1, 4, 4)
+        QRX_G2(4, 3, 1, 4) QRX_G2(4, 3, 2, 2) QRX_G2(4, 3, 4, 1) QRX_G2(4, 1, 1, 4) QRX_G2(4, 1, 2, 4) QRX_G2(4, 1, 4, 4)
         QRX_G2(8, 3, 1, 4) QRX_G2(8, 3, 2, 4) QRX_G2(8, 3, 4, 2) QRX_G2(8, 1, 1, 4) QRX_G2(8, 1, 2, 4) QRX_G2(8, 1, 4, 4)
         QRX_G2(2, 3, 1, 4) QRX_G2(2, 3, 2, 4) QRX_G2(2, 3, 4, 2) QRX_G2(2, 1, 1, 4) QRX_G2(2, 1, 2, 4) QRX_G2(2, 1, 4, 4)
     } else {
-        QRX_G2(4, 3, 1, 8) QRX_G2(4, 3, 2, 8) QRX_G2(4, 3, 4, 4) QRX_G2(4, 1, 1, 8) QRX_G2(4, 1, 2, 8) QRX_G2(4, 1, 4, 8)
+        QRX_G2(4, 3, 1, 8) QRX_G2(4, 3, 2, 4) QRX_G2(4, 3, 4, 2) QRX_G2(4, 1, 1, 8) QRX_G2(4, 1, 2, 8) QRX_G2(4, 1, 4, 8)
         QRX_G2(8, 3, 1, 8) QRX_G2(8, 3, 2, 8) QRX_G2(8, 3, 4, 4) QRX_G2(8, 1, 1, 8) QRX_G2(8, 1, 2, 8) QRX_G2(8, 1, 4, 8)
         QRX_G2(2, 3, 1, 8) QRX_G2(2, 3, 2, 8) QRX_G2(2, 3, 4, 4) QRX_G2(2, 1, 1, 8) QRX_G2(2, 1, 2, 8) QRX_G2(2, 1, 4, 8)
     }

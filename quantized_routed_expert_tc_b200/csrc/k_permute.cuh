@@ -52,15 +52,14 @@ __device__ __forceinline__ int block_exclusive_scan_1024(int v, int *tmp, int &t
     return r;
 }
 
-__global__ void __launch_bounds__(1024, 1) k_permute(const int32_t *__restrict__ idx, int A, int E,
-                                                     qrx_perm p, uint64_t *__restrict__ usage)
+// The permutation by one CTA of 1024 threads; psm: (PERM_WARPS * E + 40) ints
+// of shared memory.  Every thread of the CTA calls it.
+__device__ __forceinline__ void permute_cta(const int32_t *__restrict__ idx, int A, int E, const qrx_perm &p,
+                                            uint64_t *__restrict__ usage, int *psm)
 {
-    extern __shared__ __align__(16) int psm[];
     int *whist = psm;                          // [PERM_WARPS][E]
     int *tmp = psm + PERM_WARPS * E;           // [33]
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    pdl_wait();
-    pdl_trigger();
     for (int i = tid; i < PERM_WARPS * E; i += 1024) whist[i] = 0;
     __syncthreads();
 
@@ -128,10 +127,21 @@ __global__ void __launch_bounds__(1024, 1) k_permute(const int32_t *__restrict__
     }
 }
 
+__global__ void __launch_bounds__(1024, 1) k_permute(const int32_t *__restrict__ idx, int A, int E,
+                                                     qrx_perm p, uint64_t *__restrict__ usage)
+{
+    extern __shared__ __align__(16) int psm[];
+    pdl_wait();
+    pdl_trigger();
+    permute_cta(idx, A, E, p, usage, psm);
+}
+
+__host__ __device__ inline size_t permute_smem_bytes(int E) { return ((size_t)PERM_WARPS * E + 40) * sizeof(int); }
+
 cudaError_t launch_permute(const int32_t *idx, int T, int k, int E, const qrx_perm &p,
                            cudaStream_t st, uint64_t *usage)
 {
-    const size_t smem = ((size_t)PERM_WARPS * E + 40) * sizeof(int);
+    const size_t smem = permute_smem_bytes(E);
     if (smem > 48 * 1024) {
         cudaError_t err = cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)smem);

@@ -16,7 +16,9 @@
 // adaptive expert top-p on the result (README, "快速开始": the --topp knob),
 // which k_topp_prune also applies on its own to a router output in memory.
 #pragma once
+#include <algorithm>
 #include "qrx_dev.cuh"
+#include "k_permute.cuh"
 
 namespace qrx {
 
@@ -162,20 +164,16 @@ __global__ void __launch_bounds__(256) k_router_tile(RouterArgs a)
 // gscore[G] (f32), kept[G] (int), sel[32] (int, the chosen experts in order).
 __host__ __device__ inline size_t select_smem_per_warp(int E, int G) { return (size_t)(2 * E + 2 * G + 32) * 4; }
 
-__global__ void __launch_bounds__(256) k_router_select(RouterArgs a)
+// The selection of token t by one warp; wsm: select_smem_per_warp(E, G) bytes
+// of shared memory of its own.
+__device__ __forceinline__ void select_token_warp(const RouterArgs &a, int t, int lane, unsigned char *wsm)
 {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int t = blockIdx.x * 8 + wid;
     const int E = a.E, G = a.G, gs = a.E / a.G;
-    float *s_s = reinterpret_cast<float *>(smem_raw + select_smem_per_warp(E, G) * wid);
+    float *s_s = reinterpret_cast<float *>(wsm);
     float *sc_s = s_s + E;
     float *gsc = sc_s + E;
     int *kept = reinterpret_cast<int *>(gsc + G);
     int *sel = kept + G;
-    pdl_wait();
-    pdl_trigger();
-    if (t >= a.T) return;
 
     for (int e = lane; e < E; e += 32) {
         const float lg = a.logits[(int64_t)t * E + e];
@@ -246,6 +244,47 @@ __global__ void __launch_bounds__(256) k_router_select(RouterArgs a)
     }
 }
 
+__global__ void __launch_bounds__(256) k_router_select(RouterArgs a)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int t = blockIdx.x * 8 + wid;
+    pdl_wait();
+    pdl_trigger();
+    if (t >= a.T) return;
+    select_token_warp(a, t, lane, smem_raw + select_smem_per_warp(a.E, a.G) * wid);
+}
+
+// Selection and batch-union permutation of a small batch in one CTA of 1024
+// threads: warp t selects token t's experts (written to a.idx / a.w), then the
+// whole CTA sorts the assignments.  Saves a launch on the decode path.
+__global__ void __launch_bounds__(1024, 1) k_select_permute(RouterArgs a, qrx_perm p, uint64_t *__restrict__ usage)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    pdl_wait();
+    pdl_trigger();
+    if (wid < a.T) select_token_warp(a, wid, lane, smem_raw + select_smem_per_warp(a.E, a.G) * wid);
+    __syncthreads();        // the selection (global a.idx) is visible to the whole CTA
+    permute_cta(a.idx, a.T * a.k, a.E, p, usage, reinterpret_cast<int *>(smem_raw));
+}
+
+bool select_permute_fused_ok(int T, int E, int G)
+{
+    return T <= 32 && T * select_smem_per_warp(E, G) <= 200 * 1024 && permute_smem_bytes(E) <= 200 * 1024;
+}
+
+cudaError_t launch_select_permute(const RouterArgs &a, const qrx_perm &p, uint64_t *usage, cudaStream_t st)
+{
+    const size_t smem = std::max((size_t)a.T * select_smem_per_warp(a.E, a.G), permute_smem_bytes(a.E));
+    if (smem > 48 * 1024) {
+        const cudaError_t err =
+            cudaFuncSetAttribute(k_select_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+    }
+    return launch_k(k_select_permute, dim3(1), dim3(1024), smem, st, a, p, usage);
+}
+
 // Adaptive expert top-p on a router output already in memory: warp per token.
 __global__ void __launch_bounds__(256) k_topp_prune(int32_t *__restrict__ idx, float *__restrict__ w, int T,
                                                     int k, double thr)
@@ -270,7 +309,7 @@ cudaError_t launch_topp_prune(int32_t *idx, float *w, int T, int k, double thr, 
     return launch_k(k_topp_prune, dim3((unsigned)((T + 7) / 8)), dim3(256), 0, st, idx, w, T, k, thr);
 }
 
-cudaError_t launch_router(const RouterArgs &a, cudaStream_t st)
+cudaError_t launch_router(const RouterArgs &a, cudaStream_t st, bool select)
 {
     cudaError_t err;
     if (a.T <= RG_TMAX && a.H <= 16 * 32 * RG_W4) {
@@ -281,7 +320,7 @@ cudaError_t launch_router(const RouterArgs &a, cudaStream_t st)
         dim3 grid((a.E + RT_E - 1) / RT_E, (a.T + RT_T - 1) / RT_T);
         err = launch_k(a.x_bf16 ? k_router_tile<true> : k_router_tile<false>, grid, dim3(256), 0, st, a);
     }
-    if (err != cudaSuccess) return err;
+    if (err != cudaSuccess || !select) return err;
     const size_t smem = (size_t)8 * select_smem_per_warp(a.E, a.G);
     if (smem > 48 * 1024) {
         err = cudaFuncSetAttribute(k_router_select, cudaFuncAttributeMaxDynamicSharedMemorySize,

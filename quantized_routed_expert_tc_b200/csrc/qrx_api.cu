@@ -14,8 +14,8 @@
 #include "qrx_internal.h"
 #include "qrx_dev.cuh"
 #include "k_quant.cuh"
-#include "k_router.cuh"
 #include "k_permute.cuh"
+#include "k_router.cuh"
 #include "k_ffn_gemv.cuh"
 #include "k_ffn_tc.cuh"
 #include "k_gemv2.cuh"
@@ -307,14 +307,9 @@ int qrx_block_dots_q8(int32_t wbits, const uint8_t *q, int64_t rows, int64_t K, 
 }
 
 // The router, with adaptive top-p applied in its select kernel when topp_thr > 0.
-static int route_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr, const float *bias,
-                      int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream,
-                      double topp_thr)
+static RouterArgs router_args(const qrx_cfg *c, const void *x, int32_t T, const float *Wr, const float *bias,
+                              int32_t *topk_idx, float *topk_w, void *ws, double topp_thr)
 {
-    int v = check_common(c, T);
-    if (v) return v;
-    if (!x || !Wr || !bias || !topk_idx || !topk_w) return QRX_EINVAL;
-    if ((v = check_ws(c, T, ws, ws_bytes))) return v;
     const Ws L = ws_layout(c, T);
     RouterArgs a{};
     a.x = x;
@@ -332,6 +327,18 @@ static int route_impl(const qrx_cfg *c, const void *x, int32_t T, const float *W
     a.idx = topk_idx;
     a.w = topk_w;
     a.topp_thr = topp_thr;
+    return a;
+}
+
+static int route_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr, const float *bias,
+                      int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream,
+                      double topp_thr)
+{
+    int v = check_common(c, T);
+    if (v) return v;
+    if (!x || !Wr || !bias || !topk_idx || !topk_w) return QRX_EINVAL;
+    if ((v = check_ws(c, T, ws, ws_bytes))) return v;
+    const RouterArgs a = router_args(c, x, T, Wr, bias, topk_idx, topk_w, ws, topp_thr);
     return cuda_code(launch_router(a, (cudaStream_t)stream));
 }
 
@@ -551,12 +558,16 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     // 2.. the rest chained with programmatic dependent launch (the first kernel
     // of the call never is: it must follow whatever the stream held before)
     PdlScope pdl(!own_records);
-    if ((v = route_impl(c, x, T, Wr, bias, topk_idx, topk_w, ws, ws_bytes, stream, topp_thr))) return v;
-    g_pdl = true;
-    if (!mark(2)) return QRX_ECUDA;
     qrx_perm perm{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.sorted),
                   at<int32_t>(ws, L.inv), at<int32_t>(ws, L.uids), at<int32_t>(ws, L.nu)};
-    e = launch_permute(topk_idx, T, c->top_k, c->n_experts, perm, st, usage);
+    const RouterArgs ra = router_args(c, x, T, Wr, bias, topk_idx, topk_w, ws, topp_thr);
+    // small batches: selection and permutation in one kernel after the logits
+    const bool fused = select_permute_fused_ok(T, c->n_experts, c->n_group);
+    e = launch_router(ra, st, !fused);
+    g_pdl = true;
+    if (e != cudaSuccess || !mark(2)) return QRX_ECUDA;
+    e = fused ? launch_select_permute(ra, perm, usage, st)
+              : launch_permute(topk_idx, T, c->top_k, c->n_experts, perm, st, usage);
     if (e != cudaSuccess || !mark(3)) return QRX_ECUDA;
     float *h = at<float>(ws, L.h), *y = at<float>(ws, L.y);
     set_routed(a, routed, &perm);

@@ -55,7 +55,11 @@ struct RouterArgs {
     float *w;               // [T][k]
     double topp_thr;        // adaptive top-p: p * rsf; 0 = off
 };
-cudaError_t launch_router(const RouterArgs &a, cudaStream_t st);
+// the logits kernel, then (select) the selection kernel
+cudaError_t launch_router(const RouterArgs &a, cudaStream_t st, bool select = true);
+// selection and permutation in one kernel, for small batches
+bool select_permute_fused_ok(int T, int E, int G);
+cudaError_t launch_select_permute(const RouterArgs &a, const qrx_perm &p, uint64_t *usage, cudaStream_t st);
 cudaError_t launch_topp_prune(int32_t *idx, float *w, int T, int k, double thr, cudaStream_t st);
 
 // usage (may be null): per-expert counters [E], += this call's counts
