@@ -1,5 +1,5 @@
-// k_gemv2.cuh -- decode-shaped expert FFN: at most four tokens per expert
-// (calls of T <= 4 tokens), streamed from HBM at close to its bandwidth.
+// k_gemv2.cuh -- decode-shaped expert FFN: calls of at most four tokens, so
+// at most four tokens per expert, streamed from HBM at close to its bandwidth.
 //
 // README "JustVugg/colibri", section "已实现的功能": the batch-union MoE (each
 // unique expert of a batch read once and applied to all positions routed to
@@ -13,43 +13,42 @@
 // union (or the shared expert) with its tokens; for gate/up a unit holds RB
 // gate rows and the same RB up rows, so the SwiGLU is applied where both sums
 // meet.  Units are cut into contiguous ranges of equal estimated cost, one
-// range per CTA, one CTA per SM.  A unit streams through the CTA as K-slices
-// of G2_KS bytes per row: each slice is one stage of a shared-memory ring.
+// range per CTA, one CTA of 16 warps per SM.
 //
-// Roles.  Warp 8 is the producer: for each slice one thread issues one tiled
-// TMA copy per matrix (the slice of all the unit's rows; and, on a unit's last
-// slice, a bulk copy of the row scales) onto the stage's "full" mbarrier,
-// after the stage's "empty" mbarrier says that all compute warps left it.  Warps 0..7 compute: warp w owns rows
-// [w*RW, (w+1)*RW) of every unit; LPR lanes cover one row's chunks of a slice
-// (lane c reads 16-byte chunk c), so the rows a lane owns accumulate across
-// the slices of the unit in registers, and a unit ends with one transposed
-// warp butterfly -- no partial sums cross warps, no finaliser.
+// A warp owns R rows of each matrix of a unit for the whole of K: lane l
+// reads 16-byte chunks l, l + 32, ... of its rows straight from HBM (128-bit
+// loads that skip L1, the next chunk's loads issued before the current chunk
+// is computed), unpacks the codes in registers and dots them with the
+// activation digits (dp4a); its integer sums run over all of K, and the unit
+// ends with one transposed warp butterfly and the epilogue (row scales,
+// SwiGLU).  Rows of fewer than 32 chunks are covered by LPR = chunks lanes
+// each, several rows per warp.  No weight staging, no barrier and no partial
+// sum crosses warps in the streaming loop.
 //
 // Activations.  Every input row (a token of x for gate/up, a row of h for
-// down) is turned into a "record" in shared memory by the compute warps: NDIG
-// digit planes of signed bytes in the order the unpacked weight words use, so
-// each dot of 4 codes by 4 digits is one dp4a with an exact int32 sum.
+// down) is turned into a "record" in shared memory by the CTA: NDIG digit
+// planes of signed bytes in the order the unpacked weight words use, so each
+// dot of 4 codes by 4 digits is one dp4a with an exact int32 sum.
 //   NDIG = 3 (f32, bf16 inputs): one power-of-two scale per row, sigma =
 //     2^-s with max|x| * 2^s in [2^21, 2^22), and x*2^s rounded to an integer
 //     split into three balanced bytes (x ~= sigma (d0 + 2^8 d1 + 2^16 d2),
-//     error <= 2^-22 of the row's largest magnitude).  The int32 sums of a
-//     lane run over all of its chunks; the planes are combined once per unit.
+//     error <= 2^-22 of the row's largest magnitude).  A lane's sums per plane
+//     over its chunks are exact int32; the planes are combined once per unit.
 //   NDIG = 1 (Q8_0): the record holds the Q8_0 codes and per-block scales d_b
 //     (README: Q8_0-style int8 activations, blocks of 32 with an f32 absmax
 //     scale); every 32-block's int32 accumulator is exact and is scaled by d_b
 //     in f32.
 // Packed int4 / int2 fields are flipped to offset binary (code + 8, code + 2)
-// by the unpack; the offset is removed through the digit sums (per block for
-// Q8_0, per lane and row for NDIG = 3), so every integer sum is exact.
+// by the unpack; the offset is removed through the digit sums kept in the
+// record (per block for Q8_0, per chunk and plane for NDIG = 3).
 #pragma once
 #include "qrx_dev.cuh"
 #include "qrx_check.cuh"
 
 namespace qrx {
 
-constexpr int G2_NW = 11;                         // compute warps (3 warps per SM sub-partition in all)
-constexpr int G2_THREADS = 32 * (G2_NW + 1);      // + the producer warp
-constexpr int G2_KS = 512;                        // bytes of a row per stage (at most)
+constexpr int G2_NW = 16;                         // warps per CTA
+constexpr int G2_THREADS = 32 * G2_NW;
 constexpr int G2_TMAX = 4;                        // tokens per call
 constexpr int G2_SMEM_MAX = 227 * 1024;
 constexpr long long G2_WAIT_CAP = 1ll << 21;      // polls before a wait gives up
@@ -58,19 +57,20 @@ constexpr uint32_t G2_SUSPEND_NS = 1000;          // a waiting thread sleeps up 
 // ---------------------------------------------------------------- records
 // Record of one input row of K codes, in shared memory:
 //   digits: piece (pl, q, c) = 16 bytes at ((pl * NQ + q) * cpr + c) * 16: the
-//           q-th group of four digit words of chunk c in plane pl (NQ = DW/4);
-//           lanes reading consecutive chunks read consecutive 16-byte pieces
-//   NDIG = 3: then float sigma, int D[3] (unused slot) -- 16 bytes
+//           q-th group of four digit words of chunk c in plane pl (NQ = DW/4)
+//   NDIG = 3: then float sigma (16 bytes), then int csum[cpr][4]: the sums of
+//             chunk c's digits in planes 0, 1, 2 (and a zero)
 //   NDIG = 1: then float d[K/32] (block scales), int corr[K/32]
 //             (corr_b = -OFF * sum of the block's codes)
 struct G2Rec {
-    int hdr, bytes;
+    int hdr, csum, bytes;
 };
-__host__ __device__ inline G2Rec g2_rec(int ndig, int K)
+__host__ __device__ inline G2Rec g2_rec(int ndig, int K, int cpr)
 {
     G2Rec r;
     r.hdr = ndig * K;
-    r.bytes = r.hdr + (ndig == 3 ? 16 : 2 * (((K / 32) * 4 + 15) & ~15));
+    r.csum = r.hdr + 16;
+    r.bytes = ndig == 3 ? r.csum + cpr * 16 : r.hdr + 2 * (((K / 32) * 4 + 15) & ~15);
     return r;
 }
 
@@ -83,10 +83,8 @@ struct G2Mat {
 
 struct G2P {
     int K, rows, row_bytes, cpr;     // codes per input row, rows per matrix, bytes per row, chunks per row
-    int ks, cps, nslice;             // bytes per slice, chunks per slice, slices per row
-    int lpr, gpw, rw, rb, nrb;       // lanes per row, row groups per warp, rows per warp, rows per unit, units per slot
-    int box_rows;                    // rows per TMA box (rb is a whole number of boxes)
-    int stages, stage_bytes, scale_off, sc_stride;   // sc_stride: floats from matrix 0's scales to matrix 1's
+    int lpr, gpw, nj;                // lanes per row, row groups per warp, chunks per lane per row
+    int rw, rb, nrb;                 // rows per warp, rows per unit (per matrix), units per slot
     int rec_bytes, rec_off, nrec;    // record size, smem offset, records held
     int bar_off, pre_off, red_off, smem;
     G2Mat m[2], msh[2];              // gate/up: m[0] gate, m[1] up; down: m[0] down
@@ -120,8 +118,8 @@ __device__ __forceinline__ bool g2_try(uint32_t mbar, uint32_t parity)
     return done != 0;
 }
 
-// dp4a of unsigned weight bytes by signed digit bytes (the int4 high halves
-// are kept in place, as 16 x the code, so they need the unsigned form).
+// dp4a of unsigned weight bytes by signed digit bytes: int4 high halves are
+// kept in place (16 x the code), which needs the unsigned form.
 __device__ __forceinline__ int g2_dp4a_us(uint32_t a, uint32_t b, int c)
 {
     int d;
@@ -151,9 +149,9 @@ __device__ __forceinline__ bool g2_wait(uint32_t mbar, uint32_t parity, volatile
     return false;
 }
 
-// Barrier of the compute warps (not the producer): lane 0 of each warp
-// arrives on an mbarrier of G2_NW arrivals and every lane waits, bounded, for
-// the phase.  `ph` is the caller's phase bit.  False if the wait gave up.
+// Barrier of the compute warps: lane 0 of each warp arrives on an mbarrier of
+// G2_NW arrivals and every lane waits, bounded, for the phase.  `ph` is the
+// caller's phase bit.  False if the wait gave up.
 __device__ __forceinline__ bool g2_cbar(uint64_t *bar, uint32_t &ph, volatile int *abort_flag)
 {
     __syncwarp();
@@ -264,7 +262,7 @@ __device__ bool g2_build(const G2P &p, unsigned char *recs, int n, RowFn row_of,
     constexpr int DW = F::DW, NQ = DW / 4, EPC = F::EPC;
     const int tid = threadIdx.x, nth = G2_NW * 32;
     const int K = p.K, cpr = p.cpr;
-    const G2Rec RL = g2_rec(NDIG, K);
+    const G2Rec RL = g2_rec(NDIG, K, cpr);
     const bool bf = p.afmt == QRX_A_BF16;
     for (int i = 0; i < n; ++i) {
         const int64_t row = row_of(i);
@@ -297,6 +295,7 @@ __device__ bool g2_build(const G2P &p, unsigned char *recs, int n, RowFn row_of,
                 float v[EPC];
                 src.load<EPC / 4>(c * EPC, v);
                 uint32_t wd[3][DW];
+                int cs0 = 0, cs1 = 0, cs2 = 0;       // the chunk's digit sums per plane
 #pragma unroll
                 for (int wi = 0; wi < 4; ++wi)
 #pragma unroll
@@ -310,6 +309,9 @@ __device__ bool g2_build(const G2P &p, unsigned char *recs, int n, RowFn row_of,
                             b0 |= (uint32_t)(uint8_t)d0 << (8 * by);
                             b1 |= (uint32_t)(uint8_t)d1 << (8 * by);
                             b2 |= (uint32_t)(uint8_t)d2 << (8 * by);
+                            cs0 += d0;
+                            cs1 += d1;
+                            cs2 += d2;
                         }
                         wd[0][wi * F::UPW + j] = b0;
                         wd[1][wi * F::UPW + j] = b1;
@@ -321,6 +323,7 @@ __device__ bool g2_build(const G2P &p, unsigned char *recs, int n, RowFn row_of,
                     for (int q = 0; q < NQ; ++q)
                         *reinterpret_cast<uint4 *>(rec + ((size_t)(pl * NQ + q) * cpr + c) * 16) =
                             make_uint4(wd[pl][4 * q], wd[pl][4 * q + 1], wd[pl][4 * q + 2], wd[pl][4 * q + 3]);
+                *reinterpret_cast<int4 *>(rec + RL.csum + (size_t)c * 16) = make_int4(cs0, cs1, cs2, 0);
             }
             if (tid == 0) {
                 float sig = 0.f;
@@ -435,29 +438,24 @@ __device__ void g2_units_next(G2Units &u)
 }
 
 // ---------------------------------------------------------------- kernel
+// Shared memory: the records, the compute barrier and flags, scratch, the
+// slot cost prefix.
 template <int WB, int NDIG, int TP, int R, bool GATEUP, bool PROBE>
-__global__ void __launch_bounds__(G2_THREADS, 1)
-    k_gemv2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
-            const __grid_constant__ CUtensorMap tsh0, const __grid_constant__ CUtensorMap tsh1,
-            const __grid_constant__ G2P p)
+__global__ void __launch_bounds__(G2_THREADS, 1) k_gemv2(const __grid_constant__ G2P p)
 {
     using F = Fmt<WB>;
     constexpr int NM = GATEUP ? 2 : 1;
     constexpr int DW = F::DW, NQ = DW / 4, UPW = F::UPW;
-    constexpr int NP = NDIG == 3 ? 3 : 1;                 // planes accumulated per (token, row)
-    // int4: each packed word is split by one LOP3 per half -- low nibbles as
-    // they are, high nibbles left in place (16 x the code) -- and the two halves
-    // sum into separate exact accumulators, the second divided by 16 at the end
+    constexpr int NP = NDIG == 3 ? 3 : 1;                 // integer planes per (token, row)
+    // int4: a packed word splits by one LOP3 per half -- the low nibbles as
+    // they are, the high nibbles left in place (16 x the code) -- and the two
+    // halves sum into separate exact accumulators, the second divided by 16
     constexpr bool HI16 = WB == 4;
     constexpr int NA = HI16 ? 2 : 1;
     constexpr int NBC = WB == 2 ? 2 : 1;                 // Q8_0 blocks a chunk touches
     constexpr int V = TP * NM * R;                        // values a lane reduces per unit
-    // int2 or many tokens: every token's digits at once would not fit in registers
-    constexpr bool TOK_OUTER = TP * NDIG * DW > 48;
     extern __shared__ __align__(128) unsigned char sm[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm + p.bar_off);
-    uint64_t *empty = full + p.stages;
-    uint64_t *cbar = empty + p.stages;
+    uint64_t *cbar = reinterpret_cast<uint64_t *>(sm + p.bar_off);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(cbar + 1);
     int64_t *pre = reinterpret_cast<int64_t *>(sm + p.pre_off);
     float *scr = reinterpret_cast<float *>(sm + p.red_off);
@@ -465,26 +463,20 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) {
-        for (int st = 0; st < p.stages; ++st) {
-            mbar_init(g2_smem(&full[st]), 1);
-            mbar_init(g2_smem(&empty[st]), G2_NW);
-        }
         mbar_init(g2_smem(cbar), G2_NW);
         *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
-    uint32_t cph = 0;      // compute-barrier phase (compute warps)
-    bool built = true;
+    uint32_t cph = 0;      // barrier phase
     if constexpr (GATEUP) {
         // the records of every token, before the dependency wait: x is an input
         // of the call, so this overlaps the kernels that route
-        if (warp < G2_NW)
-            built = g2_build<WB, NDIG>(p, recs, p.T, [](int i) -> int64_t { return i; }, true, scr, cbar, cph,
-                                       abort_flag);
-        pdl_wait();        // the permutation comes from the kernels before
-        pdl_trigger();
+        if (!g2_build<WB, NDIG>(p, recs, p.T, [](int i) -> int64_t { return i; }, true, scr, cbar, cph, abort_flag))
+            return;
     }
+    pdl_wait();            // gate/up: the permutation; down: h, from the kernels before
+    pdl_trigger();
     const int nu = p.routed ? *p.n_union : 0;
     const int nslots = nu + (p.shared ? 1 : 0);
     if (warp == 0) {       // cost prefix over slots
@@ -513,121 +505,57 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
     }
     __syncthreads();
     const int64_t Ctot = pre[nslots];
-    G2Units U0;
-    U0.pre = pre;
-    U0.nslots = nslots;
-    U0.nu = nu;
-    U0.nrb = p.nrb;
-    U0.c0 = Ctot * blockIdx.x / gridDim.x;
-    U0.c1 = Ctot * (blockIdx.x + 1) / gridDim.x;
-    U0.s = -1;
-    U0.u = U0.uend = 0;
-    U0.valid = false;
-    g2_units_next(U0);
-
-    if (warp == G2_NW) {
-        // ======================== producer (one thread) ========================
-        // Each stage is one tiled TMA box per matrix (the slice's ks bytes of the
-        // unit's rb rows; rows past the matrix are zero-filled), plus, on the
-        // unit's last slice, one bulk copy of each matrix's row scales.
-        if (lane != 0) return;
-        G2Units u = U0;
-        uint32_t g = 0;
-        bool ok = true;
-        const int nbox = p.rb / p.box_rows;
-        while (ok && u.valid) {
-            const bool routed = u.s < nu;
-            int e = 0;
-            if (routed) {
-                e = p.union_ids[u.s];
-                e = (e >= 0 && e < p.E) ? e : 0;
-            }
-            const CUtensorMap *map0 = routed ? &tm0 : &tsh0;
-            const CUtensorMap *map1 = routed ? &tm1 : &tsh1;
-            const int z = routed ? e : 0;
-            const float *S0 = routed ? p.m[0].s + (int64_t)e * p.m[0].ss : p.msh[0].s;
-            const float *S1 = routed ? p.m[NM - 1].s + (int64_t)e * p.m[NM - 1].ss : p.msh[NM - 1].s;
-            const int r0 = (int)(u.u * p.rb);
-            const int nr = min(p.rb, p.rows - r0);
-            // the unit's row scales, copied from the 16-byte boundary at or below
-            // row r0 (rows is a multiple of 64, so the rounded-up end stays inside)
-            const int s0 = r0 & ~3, sn = ((r0 + nr + 3) & ~3) - s0;
-            for (int j = 0; j < p.nslice; ++j) {
-                const uint32_t st = g % p.stages;
-                if (g >= (uint32_t)p.stages && !g2_wait(g2_smem(&empty[st]), ((g / p.stages) - 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const bool last = j == p.nslice - 1;
-                const uint32_t bytes = (uint32_t)(NM * p.rb * p.ks + (last ? NM * sn * 4 : 0));
-                const uint32_t fb = g2_smem(&full[st]);
-                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb), "r"(bytes) : "memory");
-                unsigned char *dst = sm + (size_t)st * p.stage_bytes;
-                const int x = j * (p.ks / 8);          // 8-byte elements
-                for (int b = 0; b < nbox; ++b) {
-                    tma_load_3d(g2_smem(dst + (size_t)b * p.box_rows * p.ks), map0, x, r0 + b * p.box_rows, z, fb);
-                    if constexpr (NM == 2)
-                        tma_load_3d(g2_smem(dst + (size_t)(p.rb + b * p.box_rows) * p.ks), map1, x, r0 + b * p.box_rows,
-                                    z, fb);
-                }
-                if (last) {
-                    bulk_copy(g2_smem(dst + p.scale_off), S0 + s0, (uint32_t)(sn * 4), fb);
-                    if constexpr (NM == 2)
-                        bulk_copy(g2_smem(dst + p.scale_off + p.sc_stride * 4), S1 + s0, (uint32_t)(sn * 4), fb);
-                }
-                ++g;
-            }
-            g2_units_next(u);
-        }
-        // the copies issued land before the CTA may leave
-        for (uint32_t i = 0; i < (uint32_t)p.stages && i < g; ++i) {
-            const uint32_t gl = g - 1 - i;
-            bool done = false;
-            for (long long it = 0; it < G2_WAIT_CAP && !done; ++it)
-                done = g2_try(g2_smem(&full[gl % p.stages]), (gl / p.stages) & 1);
-            if (!done) raise_status(DERR_TIMEOUT);
-        }
-        return;
-    }
-
-    // ======================== compute warps ========================
-    const int LPR = p.lpr;
-    const int c = lane % LPR, grp = lane / LPR;
+    G2Units u;
+    u.pre = pre;
+    u.nslots = nslots;
+    u.nu = nu;
+    u.nrb = p.nrb;
+    u.c0 = Ctot * blockIdx.x / gridDim.x;
+    u.c1 = Ctot * (blockIdx.x + 1) / gridDim.x;
+    u.s = -1;
+    u.u = u.uend = 0;
+    u.valid = false;
+    g2_units_next(u);
     QRX_CHECK_ONLY(const int64_t n_pos = p.routed ? (int64_t)p.T * p.k : 0;)
     QRX_CHECK_ONLY(const int64_t n_out = max(n_pos, p.shared ? p.sh_out_row0 + p.T : (int64_t)0);)
-    if (!built) return;
-    if constexpr (!GATEUP) {
-        pdl_wait();        // h comes from the kernel before
-        pdl_trigger();
-    }
-    G2Units u = U0;
-    uint32_t g = 0;
+
+    const int LPR = p.lpr, nj = p.nj;
+    const int cl = lane % LPR, grp = lane / LPR;
+    const int lrow0 = warp * p.rw + grp;              // this lane's row i is lrow0 + gpw * i (in the unit)
+    const G2Rec RL = g2_rec(NDIG, p.K, p.cpr);
+    // after the butterfly (V <= LPR) lane cl holds value cl / rep: that value's
+    // token, row and (for gate/up: gate, with the up value on lane cl + rep)
+    const int rep = V <= LPR ? LPR / V : 1;
+    const int my_idx = cl / rep;
+    const int my_t = my_idx / (NM * R), my_i = (my_idx / NM) % R;
+    const bool writer = V <= LPR && cl % rep == 0 && (!GATEUP || (my_idx & 1) == 0);
+
     int cur_s = -1, nt = 0;
-    const unsigned char *rec[TP];
+    int rec[TP];           // shared-memory offsets of the slot's token records
     int64_t orow[TP];
     int corr[TP][NP];      // NDIG = 3: OFF * (this lane's digit sums over its chunks), per plane
-    float sig[TP];         // NDIG = 3: the records' scales
+    float sig[TP];
 #pragma unroll
     for (int t = 0; t < TP; ++t) {
-        rec[t] = recs;
+        rec[t] = p.rec_off;
         orow[t] = 0;
-        sig[t] = 0.f;
+        sig[t] = 1.f;
 #pragma unroll
         for (int pl = 0; pl < NP; ++pl) corr[t][pl] = 0;
     }
-    bool ok = true;
-    while (ok && u.valid) {
+    while (u.valid) {
+        const bool routed = u.s < nu;
+        int e = 0;
+        if (routed) {
+            e = p.union_ids[u.s];
+            e = (e >= 0 && e < p.E) ? e : 0;
+        }
         if (u.s != cur_s) {
             // ---- enter a slot: its tokens, their records, this lane's corrections
-            const bool routed = u.s < nu;
-            int p0 = 0;
-            if (routed) {
-                int e = p.union_ids[u.s];
-                e = (e >= 0 && e < p.E) ? e : 0;
-                p0 = p.offsets[e];
-            }
+            const int p0 = routed ? p.offsets[e] : 0;
             nt = min(g2_slot_ntok(p, u.s, nu), TP);
             int64_t inrow[TP];
+            bool ok = true;
 #pragma unroll
             for (int i = 0; i < TP; ++i) {
                 const int ii = min(i, max(nt - 1, 0));
@@ -646,45 +574,55 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                     inrow[i] = GATEUP ? ii : p.sh_in_row0 + ii;
                 }
             }
-            if (!ok) break;
+            if (!ok) return;
             if constexpr (GATEUP) {
 #pragma unroll
-                for (int i = 0; i < TP; ++i) rec[i] = recs + (size_t)inrow[i] * p.rec_bytes;
+                for (int i = 0; i < TP; ++i) rec[i] = p.rec_off + (int)inrow[i] * p.rec_bytes;
             } else {
                 // every warp is done with the previous slot's records
-                if (!g2_cbar(cbar, cph, abort_flag)) break;
-                if (!g2_build<WB, NDIG>(p, recs, nt, [&](int i) -> int64_t { return g2_pick(inrow, i); }, false,
-                                        scr, cbar, cph, abort_flag))
-                    break;
+                if (!g2_cbar(cbar, cph, abort_flag)) return;
+                if (!g2_build<WB, NDIG>(p, recs, nt, [&](int i) -> int64_t { return g2_pick(inrow, i); }, false, scr,
+                                        cbar, cph, abort_flag))
+                    return;
 #pragma unroll
-                for (int i = 0; i < TP; ++i) rec[i] = recs + (size_t)min(i, max(nt - 1, 0)) * p.rec_bytes;
+                for (int i = 0; i < TP; ++i) rec[i] = p.rec_off + min(i, max(nt - 1, 0)) * p.rec_bytes;
             }
             if constexpr (NDIG == 3) {
 #pragma unroll
-                for (int i = 0; i < TP; ++i) {
-                    sig[i] = *reinterpret_cast<const float *>(rec[i] + g2_rec(3, p.K).hdr);
-#pragma unroll
-                    for (int pl = 0; pl < 3; ++pl) {
-                        int sum = 0;
-                        for (int j = 0; j < p.nslice; ++j) {
-                            const int cg = j * p.cps + c;
-#pragma unroll
-                            for (int q = 0; q < NQ; ++q) {
-                                const uint4 d4 = *reinterpret_cast<const uint4 *>(
-                                    rec[i] + ((size_t)(pl * NQ + q) * p.cpr + cg) * 16);
-                                sum = dp4a(0x01010101u, d4.x, sum);
-                                sum = dp4a(0x01010101u, d4.y, sum);
-                                sum = dp4a(0x01010101u, d4.z, sum);
-                                sum = dp4a(0x01010101u, d4.w, sum);
-                            }
-                        }
-                        corr[i][pl] = F::OFF * sum;
+                for (int t = 0; t < TP; ++t) {
+                    sig[t] = *reinterpret_cast<const float *>(sm + rec[t] + RL.hdr);
+                    int s0 = 0, s1 = 0, s2 = 0;
+                    for (int j = 0; j < nj; ++j) {
+                        const int4 c4 = *reinterpret_cast<const int4 *>(sm + rec[t] + RL.csum + (cl + LPR * j) * 16);
+                        s0 += c4.x;
+                        s1 += c4.y;
+                        s2 += c4.z;
                     }
+                    corr[t][0] = F::OFF * s0;
+                    corr[t][1] = F::OFF * s1;
+                    corr[t][2] = F::OFF * s2;
                 }
             }
             cur_s = u.s;
         }
-        // ---- one unit: nslice stages
+        // ---- one unit: this lane's rows, their row pointers and (writers) scales
+        const int r0 = (int)(u.u * p.rb);
+        const uint8_t *wrow[NM][R];
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+            const uint8_t *base = routed ? p.m[m].q + (int64_t)e * p.m[m].sq : p.msh[m].q;
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                const int row = min(r0 + lrow0 + p.gpw * i, p.rows - 1);     // a row past the end is read, unused
+                wrow[m][i] = base + (int64_t)row * p.row_bytes;
+            }
+        }
+        float sc0 = 0.f, sc1 = 0.f;
+        const int wr_row = r0 + lrow0 + p.gpw * my_i;
+        if (writer && wr_row < p.rows) {
+            sc0 = routed ? p.m[0].s[(int64_t)e * p.m[0].ss + wr_row] : p.msh[0].s[wr_row];
+            if constexpr (GATEUP) sc1 = routed ? p.m[1].s[(int64_t)e * p.m[1].ss + wr_row] : p.msh[1].s[wr_row];
+        }
         int iacc[TP][NM][R][NP][NA];
         float facc[TP][NM][R];
 #pragma unroll
@@ -699,193 +637,165 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
 #pragma unroll
                         for (int h = 0; h < NA; ++h) iacc[t][m][i][pl][h] = 0;
                 }
-        const int lrow0 = warp * p.rw + grp;             // this lane's first row in the unit (then + gpw)
-        for (int j = 0; j < p.nslice; ++j, ++g) {
-            const uint32_t st = g % p.stages;
-            if (!g2_wait(g2_smem(&full[st]), (g / p.stages) & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            const unsigned char *stg = sm + (size_t)st * p.stage_bytes;
-            const int cg = j * p.cps + c;                // this lane's chunk of the row
-            auto load_dig = [&](int t, uint32_t (&d)[NDIG][DW]) {
+        auto load = [&](int j, uint4 (&b)[NM][R]) {
+#pragma unroll
+            for (int m = 0; m < NM; ++m)
+#pragma unroll
+                for (int i = 0; i < R; ++i) b[m][i] = ld_stream16(wrow[m][i] + (size_t)(cl + LPR * j) * 16);
+        };
+        // chunk j of every row of this lane, against every token of the slot
+        auto compute = [&](int j, const uint4 (&b)[NM][R]) {
+            const int c = cl + LPR * j;
+#pragma unroll
+            for (int t = 0; t < TP; ++t) {
+                if (t >= nt) break;
+                const unsigned char *rt = sm + rec[t];
+                const int cpr16 = p.cpr * 16;
+                uint32_t d[NDIG][DW];
 #pragma unroll
                 for (int pl = 0; pl < NDIG; ++pl)
 #pragma unroll
                     for (int q = 0; q < NQ; ++q) {
-                        const uint4 d4 =
-                            *reinterpret_cast<const uint4 *>(rec[t] + ((size_t)(pl * NQ + q) * p.cpr + cg) * 16);
+                        const uint4 d4 = *reinterpret_cast<const uint4 *>(rt + (pl * NQ + q) * cpr16 + c * 16);
                         d[pl][4 * q] = d4.x;
                         d[pl][4 * q + 1] = d4.y;
                         d[pl][4 * q + 2] = d4.z;
                         d[pl][4 * q + 3] = d4.w;
                     }
-            };
-            auto load_blk = [&](int t, float (&dq)[NBC], int (&cb)[NBC]) {
-                const G2Rec RL = g2_rec(1, p.K);
-                const float *dsc = reinterpret_cast<const float *>(rec[t] + RL.hdr);
-                const int *cor = reinterpret_cast<const int *>(rec[t] + RL.hdr + (RL.bytes - RL.hdr) / 2);
-#pragma unroll
-                for (int bc = 0; bc < NBC; ++bc) {
-                    const int b = WB == 8 ? (cg >> 1) : (WB == 4 ? cg : 2 * cg + bc);
-                    dq[bc] = dsc[b];
-                    cb[bc] = cor[b];
-                }
-            };
-            auto unpack = [&](int m, int i, uint32_t (&uw)[4][UPW]) {
-                const uint4 wv = *reinterpret_cast<const uint4 *>(
-                    stg + ((size_t)(m * p.rb + lrow0 + p.gpw * i)) * p.ks + (size_t)c * 16);
-                const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                for (int wi = 0; wi < 4; ++wi) {
-                    if constexpr (HI16) {
-                        uw[wi][0] = (ww[wi] ^ 0x88888888u) & 0x0F0F0F0Fu;   // elements 0, 2, 4, 6 (code + 8)
-                        uw[wi][1] = (ww[wi] ^ 0x88888888u) & 0xF0F0F0F0u;   // elements 1, 3, 5, 7, x16
-                    } else {
-                        unpack_word<WB>(ww[wi], uw[wi]);
-                    }
-                }
-            };
-            // one unpacked weight chunk against one token's digits
-            auto dot = [&](int t, int m, int i, const uint32_t (&uw)[4][UPW], const uint32_t (&d)[NDIG][DW],
-                           const float (&dq)[NBC], const int (&cb)[NBC]) {
-                if constexpr (NDIG == 3) {
-#pragma unroll
-                    for (int wi = 0; wi < 4; ++wi)
-#pragma unroll
-                        for (int jj = 0; jj < UPW; ++jj)
-#pragma unroll
-                            for (int pl = 0; pl < 3; ++pl) {
-                                int &a = iacc[t][m][i][pl][HI16 ? jj : 0];
-                                a = HI16 ? g2_dp4a_us(uw[wi][jj], d[pl][wi * UPW + jj], a)
-                                         : dp4a(uw[wi][jj], d[pl][wi * UPW + jj], a);
-                            }
-                } else {
-                    int ib[NBC], ibh = 0;
-#pragma unroll
-                    for (int bc = 0; bc < NBC; ++bc) ib[bc] = cb[bc];
-#pragma unroll
-                    for (int wi = 0; wi < 4; ++wi)
-#pragma unroll
-                        for (int jj = 0; jj < UPW; ++jj) {
-                            const int bc = WB == 2 ? (wi >> 1) : 0;
-                            if (HI16 && jj == 1) ibh = g2_dp4a_us(uw[wi][jj], d[0][wi * UPW + jj], ibh);
-                            else ib[bc] = dp4a(uw[wi][jj], d[0][wi * UPW + jj], ib[bc]);
-                        }
-                    if constexpr (HI16) ib[0] += ibh >> 4;
-                    // int8: a block is two chunks on lanes 2b, 2b+1
-                    if constexpr (WB == 8) ib[0] += __shfl_xor_sync(0xffffffffu, ib[0], 1);
-                    const bool mine = WB != 8 || (c & 1) == 0;
+                float dq[NBC];
+                int cb[NBC];
+                if constexpr (NDIG == 1) {
+                    const float *dsc = reinterpret_cast<const float *>(rt + RL.hdr);
+                    const int *cor = reinterpret_cast<const int *>(rt + RL.hdr + (RL.bytes - RL.hdr) / 2);
 #pragma unroll
                     for (int bc = 0; bc < NBC; ++bc) {
-                        if (mine) facc[t][m][i] = fmaf(dq[bc], (float)ib[bc], facc[t][m][i]);
-                        if constexpr (PROBE) {
-                            const int64_t row = u.u * p.rb + lrow0 + p.gpw * i;
-                            if (mine && row < p.rows) {
-                                const int b = WB == 8 ? (cg >> 1) : (WB == 4 ? cg : 2 * cg + bc);
-                                p.probe[((orow[t] * NM + m) * p.rows + row) * (int64_t)(p.K / 32) + b] = ib[bc];
-                            }
-                        }
+                        const int bb = WB == 8 ? (c >> 1) : (WB == 4 ? c : 2 * c + bc);
+                        dq[bc] = dsc[bb];
+                        cb[bc] = cor[bb];
                     }
                 }
-            };
-            if constexpr (TOK_OUTER) {
-#pragma unroll
-                for (int t = 0; t < TP; ++t) {
-                    if (t < nt) {
-                        uint32_t d[NDIG][DW];
-                        float dq[NBC] = {};
-                        int cb[NBC] = {};
-                        load_dig(t, d);
-                        if constexpr (NDIG == 1) load_blk(t, dq, cb);
-#pragma unroll
-                        for (int m = 0; m < NM; ++m)
-#pragma unroll
-                            for (int i = 0; i < R; ++i) {
-                                uint32_t uw[4][UPW];
-                                unpack(m, i, uw);
-                                dot(t, m, i, uw, d, dq, cb);
-                            }
-                    }
-                }
-            } else {
-                uint32_t d[TP][NDIG][DW];
-                float dq[TP][NBC] = {};
-                int cb[TP][NBC] = {};
-#pragma unroll
-                for (int t = 0; t < TP; ++t)
-                    if (t < nt) {
-                        load_dig(t, d[t]);
-                        if constexpr (NDIG == 1) load_blk(t, dq[t], cb[t]);
-                    }
 #pragma unroll
                 for (int m = 0; m < NM; ++m)
 #pragma unroll
                     for (int i = 0; i < R; ++i) {
+                        const uint32_t ww[4] = {b[m][i].x, b[m][i].y, b[m][i].z, b[m][i].w};
                         uint32_t uw[4][UPW];
-                        unpack(m, i, uw);
 #pragma unroll
-                        for (int t = 0; t < TP; ++t)
-                            if (t < nt) dot(t, m, i, uw, d[t], dq[t], cb[t]);
+                        for (int wi = 0; wi < 4; ++wi) {
+                            if constexpr (HI16) {
+                                uw[wi][0] = (ww[wi] ^ 0x88888888u) & 0x0F0F0F0Fu;   // elements 0, 2, 4, 6 (code + 8)
+                                uw[wi][1] = (ww[wi] ^ 0x88888888u) & 0xF0F0F0F0u;   // elements 1, 3, 5, 7, x16
+                            } else {
+                                unpack_word<WB>(ww[wi], uw[wi]);
+                            }
+                        }
+                        if constexpr (NDIG == 3) {
+#pragma unroll
+                            for (int wi = 0; wi < 4; ++wi)
+#pragma unroll
+                                for (int jj = 0; jj < UPW; ++jj)
+#pragma unroll
+                                    for (int pl = 0; pl < 3; ++pl) {
+                                        int &acc = iacc[t][m][i][pl][HI16 ? jj : 0];
+                                        acc = HI16 ? g2_dp4a_us(uw[wi][jj], d[pl][wi * UPW + jj], acc)
+                                                   : dp4a(uw[wi][jj], d[pl][wi * UPW + jj], acc);
+                                    }
+                        } else {
+                            int ib[NBC], ibh = 0;
+#pragma unroll
+                            for (int bc = 0; bc < NBC; ++bc) ib[bc] = cb[bc];
+#pragma unroll
+                            for (int wi = 0; wi < 4; ++wi)
+#pragma unroll
+                                for (int jj = 0; jj < UPW; ++jj) {
+                                    const int bc = WB == 2 ? (wi >> 1) : 0;
+                                    if (HI16 && jj == 1) ibh = g2_dp4a_us(uw[wi][jj], d[0][wi * UPW + jj], ibh);
+                                    else ib[bc] = dp4a(uw[wi][jj], d[0][wi * UPW + jj], ib[bc]);
+                                }
+                            if constexpr (HI16) ib[0] += ibh >> 4;
+                            // int8: a block is two chunks, on lanes 2b and 2b + 1
+                            if constexpr (WB == 8) ib[0] += __shfl_xor_sync(0xffffffffu, ib[0], 1);
+                            const bool mine = WB != 8 || (c & 1) == 0;
+#pragma unroll
+                            for (int bc = 0; bc < NBC; ++bc) {
+                                if (mine) facc[t][m][i] = fmaf(dq[bc], (float)ib[bc], facc[t][m][i]);
+                                if constexpr (PROBE) {
+                                    const int64_t row = r0 + lrow0 + p.gpw * i;
+                                    if (mine && row < p.rows) {
+                                        const int bb = WB == 8 ? (c >> 1) : (WB == 4 ? c : 2 * c + bc);
+                                        p.probe[((orow[t] * NM + m) * p.rows + row) * (int64_t)(p.K / 32) + bb] = ib[bc];
+                                    }
+                                }
+                            }
+                        }
                     }
             }
-            if (j == p.nslice - 1) {
-                // ---- epilogue: lane partials -> row totals -> scales -> outputs
-                float v[V];
+        };
+        // the streaming loop: chunk j + 1's loads are issued before chunk j is computed
+        uint4 bufA[NM][R], bufB[NM][R];
+        load(0, bufA);
+#pragma unroll 1
+        for (int j = 0; j < nj; j += 2) {
+            if (j + 1 < nj) load(j + 1, bufB);
+            compute(j, bufA);
+            if (j + 2 < nj) load(j + 2, bufA);
+            if (j + 1 < nj) compute(j + 1, bufB);
+        }
+        // ---- epilogue: lane partials -> row totals -> scales -> outputs
+        float v[V];
 #pragma unroll
-                for (int t = 0; t < TP; ++t)
+        for (int t = 0; t < TP; ++t)
 #pragma unroll
-                    for (int i = 0; i < R; ++i)
+            for (int i = 0; i < R; ++i)
 #pragma unroll
-                        for (int m = 0; m < NM; ++m) {
-                            float x;
-                            if constexpr (NDIG == 3) {
-                                int P[3];
+                for (int m = 0; m < NM; ++m) {
+                    float x;
+                    if constexpr (NDIG == 3) {
+                        int P[3];
 #pragma unroll
-                                for (int pl = 0; pl < 3; ++pl)
-                                    P[pl] = (HI16 ? iacc[t][m][i][pl][0] + (iacc[t][m][i][pl][NA - 1] >> 4)
-                                                  : iacc[t][m][i][pl][0]) - corr[t][pl];
-                                x = fmaf(65536.f, (float)P[2], fmaf(256.f, (float)P[1], (float)P[0]));
-                            }
-                            else
-                                x = facc[t][m][i];
-                            v[(t * R + i) * NM + m] = t < nt ? x : 0.f;
-                        }
-                if (LPR == 32) g2_tr_reduce<V, 32>(v, lane);
-                else if (LPR == 16) g2_tr_reduce<V, 16>(v, lane);
-                else if (LPR == 8) g2_tr_reduce<V, 8>(v, lane);
-                else if (LPR == 4) g2_tr_reduce<V, 4>(v, lane);
-                else if (LPR == 2) g2_tr_reduce<V, 2>(v, lane);
-                // row scales of the unit, from the 16-byte boundary at or below its first row
-                const float *scl = reinterpret_cast<const float *>(stg + p.scale_off) + ((u.u * p.rb) & 3);
-                // total `tot` (and for gate/up the matching up total `upv`) of value idx
-                auto emit = [&](int idx, float tot, float upv) {
-                    const int t = idx / (NM * R), i = (idx / NM) % R;
-                    const int lrow = lrow0 + p.gpw * i;
-                    const int64_t row = u.u * p.rb + lrow;
-                    if (t >= nt || row >= p.rows) return;
-                    const int64_t o = g2_pick(orow, t);
-                    QRX_CHECK_OR(o >= 0 && o < n_out, return);
-                    const float sg = NDIG == 3 ? g2_pick(sig, t) : 1.f;
-                    if constexpr (GATEUP)
-                        p.out[o * p.out_ld + row] = silu_mul(scl[lrow] * (sg * tot), scl[p.sc_stride + lrow] * (sg * upv));
+                        for (int pl = 0; pl < 3; ++pl)
+                            P[pl] = (HI16 ? iacc[t][m][i][pl][0] + (iacc[t][m][i][pl][NA - 1] >> 4) : iacc[t][m][i][pl][0]) -
+                                    corr[t][pl];
+                        x = fmaf(65536.f, (float)P[2], fmaf(256.f, (float)P[1], (float)P[0]));
+                    }
                     else
-                        p.out[o * p.out_ld + row] = scl[lrow] * (sg * tot);
-                };
-                if (V <= LPR) {
-                    const int rep = LPR / V;
-                    const int idx = c / rep;
-                    const float upv = GATEUP ? __shfl_xor_sync(0xffffffffu, v[0], rep) : 0.f;
-                    if (c % rep == 0 && (!GATEUP || (idx & 1) == 0)) emit(idx, v[0], upv);
-                } else {
-                    const int nv = V / LPR;
-#pragma unroll
-                    for (int q = 0; q < V; q += NM)
-                        if (q < nv) emit(c * nv + q, v[q], GATEUP ? v[q + NM - 1] : 0.f);
+                        x = facc[t][m][i];
+                    v[(t * R + i) * NM + m] = t < nt ? x : 0.f;
                 }
+        if (LPR == 32) g2_tr_reduce<V, 32>(v, lane);
+        else if (LPR == 16) g2_tr_reduce<V, 16>(v, lane);
+        else if (LPR == 8) g2_tr_reduce<V, 8>(v, lane);
+        else if (LPR == 4) g2_tr_reduce<V, 4>(v, lane);
+        else if (LPR == 2) g2_tr_reduce<V, 2>(v, lane);
+        // value idx's total tot (gate/up: and its up total upv) to the output
+        auto emit = [&](int idx, float tot, float upv, float s0, float s1) {
+            const int t = idx / (NM * R), i = (idx / NM) % R;
+            const int row = r0 + lrow0 + p.gpw * i;
+            if (t >= nt || row >= p.rows) return;
+            const int64_t o = g2_pick(orow, t);
+            QRX_CHECK_OR(o >= 0 && o < n_out, return);
+            const float sg = NDIG == 3 ? g2_pick(sig, t) : 1.f;
+            if constexpr (GATEUP)
+                p.out[o * p.out_ld + row] = silu_mul(s0 * (sg * tot), s1 * (sg * upv));
+            else
+                p.out[o * p.out_ld + row] = s0 * (sg * tot);
+        };
+        if (V <= LPR) {
+            const float upv = GATEUP ? __shfl_xor_sync(0xffffffffu, v[0], rep) : 0.f;
+            if (writer) emit(my_idx, v[0], upv, sc0, sc1);
+        } else {
+            // few lanes per row (short rows): each lane holds V / LPR totals
+            const int nv = V / LPR;
+#pragma unroll
+            for (int q = 0; q < V; q += NM) {
+                if (q >= nv) break;
+                const int idx = cl * nv + q;
+                const int i = (idx / NM) % R;
+                const int row = min(r0 + lrow0 + p.gpw * i, p.rows - 1);
+                const float s0 = routed ? p.m[0].s[(int64_t)e * p.m[0].ss + row] : p.msh[0].s[row];
+                const float s1 = GATEUP ? (routed ? p.m[NM - 1].s[(int64_t)e * p.m[NM - 1].ss + row] : p.msh[NM - 1].s[row]) : 0.f;
+                emit(idx, v[q], GATEUP ? v[q + NM - 1] : 0.f, s0, s1);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(g2_smem(&empty[st]));
         }
         g2_units_next(u);
     }
@@ -898,58 +808,45 @@ struct G2Plan {
 };
 
 // Geometry for one projection: `nm` matrices of `rows` rows x K codes at wbits,
-// activations with ndig digit planes, calls of T <= G2_TMAX tokens.
+// activations with ndig digit planes, calls of T <= G2_TMAX tokens.  R (rows
+// per lane per matrix) is 2 for gate/up and 4 for down: four row chunks per
+// lane per step, double-buffered, keep ~64 KB of loads in flight per SM
+// (halved for several tokens with f32 / bf16 digits, or int2, to fit the
+// accumulators in registers).
 static inline bool g2_plan(G2Plan &pl, int wbits, int ndig, int K, int rows, int nm, int T, int maxslots)
 {
     G2P &p = pl.p;
     p = G2P{};
-    if (T < 1 || T > G2_TMAX) return false;
+    if (T < 1 || T > G2_TMAX || rows < 1) return false;
     pl.tp = T == 1 ? 1 : (T == 2 ? 2 : 4);
-    // rows per lane R: the integer accumulators (3 planes, x2 for int4's split
-    // halves; Q8_0: one f32) x matrices x R x TP stay within 48 registers
-    const int perrow = (ndig == 3 ? 3 * (wbits == 4 ? 2 : 1) : 1) * nm * pl.tp;
-    const int rmax = nm == 2 ? 4 : 8;
-    pl.r = 1;
-    while (pl.r * 2 <= rmax && pl.r * 2 * perrow <= 48) pl.r *= 2;
+    pl.r = nm == 2 ? 2 : 4;
+    if (pl.tp >= 2 && (ndig == 3 || wbits == 2)) pl.r /= 2;   // several tokens' sums, or int2's wide unpack
     p.K = K;
     p.rows = rows;
     p.row_bytes = K * wbits / 8;
     if (p.row_bytes % 16) return false;
     p.cpr = p.row_bytes / 16;
-    p.ks = p.row_bytes < G2_KS ? p.row_bytes : G2_KS;
-    if (p.row_bytes % p.ks) return false;
-    p.cps = p.ks / 16;
-    if (32 % p.cps != 0 && p.cps != 32) return false;
-    p.nslice = p.row_bytes / p.ks;
-    p.lpr = p.cps;
-    p.gpw = 32 / p.lpr;
+    if (p.cpr >= 32) {
+        if (p.cpr % 32) return false;
+        p.lpr = 32;
+        p.gpw = 1;
+        p.nj = p.cpr / 32;
+    } else {
+        if (32 % p.cpr) return false;
+        p.lpr = p.cpr;
+        p.gpw = 32 / p.cpr;
+        p.nj = 1;
+    }
     p.rw = pl.r * p.gpw;
     p.rb = G2_NW * p.rw;
     p.nrb = (rows + p.rb - 1) / p.rb;
-    if (rows % 4) return false;
-    // a TMA box spans at most 256 rows: rb is cut into equal boxes, each landing
-    // on a 128-byte boundary of shared memory
-    int nbox = (p.rb + 255) / 256;
-    while (p.rb % nbox) ++nbox;
-    p.box_rows = p.rb / nbox;
-    if ((p.box_rows * p.ks) % 128) return false;
-    p.scale_off = nm * p.rb * p.ks;
-    p.sc_stride = (p.rb + 7) & ~3;           // rb + up to 3 leading rows, rounded to 16 bytes
-    p.stage_bytes = (p.scale_off + nm * p.sc_stride * 4 + 127) & ~127;
-    p.rec_bytes = (g2_rec(ndig, K).bytes + 127) & ~127;
-    p.nrec = nm == 2 ? T : pl.tp;        // gate/up: every token; down: one slot's rows
-    const int fixed_tail = 128 /*barriers*/ + 256 /*scratch*/ + (maxslots + 2) * 8;
-    const int avail = G2_SMEM_MAX - p.nrec * p.rec_bytes - fixed_tail;
-    int stages = avail / p.stage_bytes;
-    if (stages > 8) stages = 8;
-    if (stages < 2) return false;
-    p.stages = stages;
-    int o = stages * p.stage_bytes;
+    p.rec_bytes = (g2_rec(ndig, K, p.cpr).bytes + 127) & ~127;
+    p.nrec = nm == 2 ? T : pl.tp;               // gate/up: every token; down: one slot's rows
+    int o = 0;
     p.rec_off = o;
     o += p.nrec * p.rec_bytes;
     p.bar_off = o;
-    o += 2 * stages * 8 + 16;
-    o = (o + 15) & ~15;
+    o += 16;
     p.red_off = o;
     o += 256;
     p.pre_off = o;
@@ -958,93 +855,8 @@ static inline bool g2_plan(G2Plan &pl, int wbits, int ndig, int K, int rows, int
     return o <= G2_SMEM_MAX;
 }
 
-// Tiled TMA map of one packed matrix of nexp experts: 8-byte elements, dims
-// (row_bytes/8, rows, nexp), box (ks/8, box_rows, 1), no swizzle (a box lands as
-// box_rows rows of ks bytes).  Encoded maps are kept in a small cache keyed by
-// every argument, so a call with the same experts encodes nothing.
-struct G2MapKey {
-    const void *q;
-    int64_t row_bytes, rows, nexp, stride, ks, box_rows;
-    bool operator==(const G2MapKey &o) const
-    {
-        return q == o.q && row_bytes == o.row_bytes && rows == o.rows && nexp == o.nexp && stride == o.stride &&
-               ks == o.ks && box_rows == o.box_rows;
-    }
-};
-
-static bool g2_map(CUtensorMap *m, const G2MapKey &k)
-{
-    constexpr int NC = 64;
-    static std::mutex mu;
-    static G2MapKey keys[NC];
-    static CUtensorMap maps[NC];
-    static int used = 0, next = 0;
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        for (int i = 0; i < used; ++i)
-            if (keys[i] == k) {
-                *m = maps[i];
-                return true;
-            }
-    }
-    const auto fn = tc_encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)(k.row_bytes / 8), (cuuint64_t)k.rows, (cuuint64_t)k.nexp};
-    const cuuint64_t strides[2] = {(cuuint64_t)k.row_bytes, (cuuint64_t)k.stride};
-    const cuuint32_t box[3] = {(cuuint32_t)(k.ks / 8), (cuuint32_t)k.box_rows, 1};
-    const cuuint32_t es[3] = {1, 1, 1};
-    CUtensorMap t{};
-    if (fn(&t, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void *>(k.q), dims, strides, box, es,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return false;
-    std::lock_guard<std::mutex> lock(mu);
-    keys[next] = k;
-    maps[next] = t;
-    next = (next + 1) % NC;
-    if (used < NC) ++used;
-    *m = t;
-    return true;
-}
-
-// The four maps of a launch: routed matrices 0/1 and the shared expert's 0/1
-// (down: one matrix each; unused maps are copies, never read).
-struct G2Maps {
-    CUtensorMap m0, m1, s0, s1;
-};
-
-static bool g2_maps(G2Maps &M, const G2P &p, int nm, const MatRef &r0, const MatRef &r1, const MatRef &sh0,
-                    const MatRef &sh1)
-{
-    M = G2Maps{};
-    const int64_t one = (int64_t)p.rows * p.row_bytes;
-    bool ok = true;
-    if (p.routed) {
-        ok = ok && g2_map(&M.m0, G2MapKey{r0.q, p.row_bytes, p.rows, p.E, p.E > 1 ? r0.sq : one, p.ks, p.box_rows});
-        if (nm == 2)
-            ok = ok && g2_map(&M.m1, G2MapKey{r1.q, p.row_bytes, p.rows, p.E, p.E > 1 ? r1.sq : one, p.ks, p.box_rows});
-    }
-    if (p.shared) {
-        ok = ok && g2_map(&M.s0, G2MapKey{sh0.q, p.row_bytes, p.rows, 1, one, p.ks, p.box_rows});
-        if (nm == 2) ok = ok && g2_map(&M.s1, G2MapKey{sh1.q, p.row_bytes, p.rows, 1, one, p.ks, p.box_rows});
-    }
-    if (nm == 1) {
-        M.m1 = M.m0;
-        M.s1 = M.s0;
-    }
-    if (!p.routed) {
-        M.m0 = M.s0;
-        M.m1 = M.s1;
-    }
-    if (!p.shared) {
-        M.s0 = M.m0;
-        M.s1 = M.m1;
-    }
-    return ok;
-}
-
 template <int WB, int ND, int TP, int R, bool GU, bool PR>
-static cudaError_t g2_go(const G2Maps &M, const G2P &p, int grid, cudaStream_t st)
+static cudaError_t g2_go(const G2P &p, int grid, cudaStream_t st)
 {
     auto kern = k_gemv2<WB, ND, TP, R, GU, PR>;
     static std::atomic<unsigned long long> configured{0};
@@ -1056,33 +868,23 @@ static cudaError_t g2_go(const G2Maps &M, const G2P &p, int grid, cudaStream_t s
         if (err != cudaSuccess) return err;
         if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_release);
     }
-    return launch_k(kern, dim3(grid), dim3(G2_THREADS), (size_t)p.smem, st, M.m0, M.m1, M.s0, M.s1, p);
+    return launch_k(kern, dim3(grid), dim3(G2_THREADS), (size_t)p.smem, st, p);
 }
 
 template <bool GU, bool PR>
-static cudaError_t g2_dispatch(const G2Maps &M, const G2Plan &pl, int wbits, int ndig, int grid, cudaStream_t st)
+static cudaError_t g2_dispatch(const G2Plan &pl, int wbits, int ndig, int grid, cudaStream_t st)
 {
+    constexpr int R1 = GU ? 2 : 4, R2 = R1 / 2;     // rows per lane: one token; several (halved)
 #define QRX_G2(WB, ND, TP, R) \
-    if (wbits == WB && ndig == ND && pl.tp == TP && pl.r == R) return g2_go<WB, ND, TP, R, GU, PR>(M, pl.p, grid, st);
-    // rows per lane R: the accumulators (NDIG or 1) x matrices x R x TP stay within 48
+    if (wbits == WB && ndig == ND && pl.tp == TP && pl.r == R) return g2_go<WB, ND, TP, R, GU, PR>(pl.p, grid, st);
     if constexpr (PR) {        // Q8_0 with the block-sum side output
-        if constexpr (GU) {
-            QRX_G2(4, 1, 1, 4) QRX_G2(4, 1, 2, 4) QRX_G2(4, 1, 4, 4)
-            QRX_G2(8, 1, 1, 4) QRX_G2(8, 1, 2, 4) QRX_G2(8, 1, 4, 4)
-            QRX_G2(2, 1, 1, 4) QRX_G2(2, 1, 2, 4) QRX_G2(2, 1, 4, 4)
-        } else {
-            QRX_G2(4, 1, 1, 8) QRX_G2(4, 1, 2, 8) QRX_G2(4, 1, 4, 8)
-            QRX_G2(8, 1, 1, 8) QRX_G2(8, 1, 2, 8) QRX_G2(8, 1, 4, 8)
-            QRX_G2(2, 1, 1, 8) QRX_G2(2, 1, 2, 8) QRX_G2(2, 1, 4, 8)
-        }
-    } else if constexpr (GU) {
-        QRX_G2(4, 3, 1, 4) QRX_G2(4, 3, 2, 2) QRX_G2(4, 3, 4, 1) QRX_G2(4, 1, 1, 4) QRX_G2(4, 1, 2, 4) QRX_G2(4, 1, 4, 4)
-        QRX_G2(8, 3, 1, 4) QRX_G2(8, 3, 2, 4) QRX_G2(8, 3, 4, 2) QRX_G2(8, 1, 1, 4) QRX_G2(8, 1, 2, 4) QRX_G2(8, 1, 4, 4)
-        QRX_G2(2, 3, 1, 4) QRX_G2(2, 3, 2, 4) QRX_G2(2, 3, 4, 2) QRX_G2(2, 1, 1, 4) QRX_G2(2, 1, 2, 4) QRX_G2(2, 1, 4, 4)
+        QRX_G2(4, 1, 1, R1) QRX_G2(4, 1, 2, R1) QRX_G2(4, 1, 4, R1)
+        QRX_G2(8, 1, 1, R1) QRX_G2(8, 1, 2, R1) QRX_G2(8, 1, 4, R1)
+        QRX_G2(2, 1, 1, R1) QRX_G2(2, 1, 2, R2) QRX_G2(2, 1, 4, R2)
     } else {
-        QRX_G2(4, 3, 1, 8) QRX_G2(4, 3, 2, 4) QRX_G2(4, 3, 4, 2) QRX_G2(4, 1, 1, 8) QRX_G2(4, 1, 2, 8) QRX_G2(4, 1, 4, 8)
-        QRX_G2(8, 3, 1, 8) QRX_G2(8, 3, 2, 8) QRX_G2(8, 3, 4, 4) QRX_G2(8, 1, 1, 8) QRX_G2(8, 1, 2, 8) QRX_G2(8, 1, 4, 8)
-        QRX_G2(2, 3, 1, 8) QRX_G2(2, 3, 2, 8) QRX_G2(2, 3, 4, 4) QRX_G2(2, 1, 1, 8) QRX_G2(2, 1, 2, 8) QRX_G2(2, 1, 4, 8)
+        QRX_G2(4, 3, 1, R1) QRX_G2(4, 3, 2, R2) QRX_G2(4, 3, 4, R2) QRX_G2(4, 1, 1, R1) QRX_G2(4, 1, 2, R1) QRX_G2(4, 1, 4, R1)
+        QRX_G2(8, 3, 1, R1) QRX_G2(8, 3, 2, R2) QRX_G2(8, 3, 4, R2) QRX_G2(8, 1, 1, R1) QRX_G2(8, 1, 2, R1) QRX_G2(8, 1, 4, R1)
+        QRX_G2(2, 3, 1, R1) QRX_G2(2, 3, 2, R2) QRX_G2(2, 3, 4, R2) QRX_G2(2, 1, 1, R1) QRX_G2(2, 1, 2, R2) QRX_G2(2, 1, 4, R2)
     }
 #undef QRX_G2
     return cudaErrorInvalidValue;
@@ -1106,7 +908,7 @@ static inline G2Mat g2_mat(const MatRef &m) { return G2Mat{m.q, m.s, m.sq, m.ss}
 
 bool g2_use(const FfnArgs &a)
 {
-    if (a.T < 1 || a.T > G2_TMAX || !tc_encode_fn()) return false;
+    if (a.T < 1 || a.T > G2_TMAX) return false;
     const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
     G2Plan pg, pd;
     return g2_plan(pg, a.wbits, ndig, a.H, a.I, 2, a.T, a.E + 1) && g2_plan(pd, a.wbits, ndig, a.I, a.H, 1, a.T, a.E + 1);
@@ -1133,10 +935,8 @@ cudaError_t launch_g2_gateup(const FfnArgs &a, int num_sms, cudaStream_t st, int
     p.out_ld = a.h_ld;
     p.sh_out_row0 = a.sh_h_row0;
     p.probe = probe;
-    G2Maps M;
-    if (!g2_maps(M, p, 2, a.gate, a.up, a.gate_sh, a.up_sh)) return cudaErrorInvalidValue;
-    if (probe) return ndig == 1 ? g2_dispatch<true, true>(M, pl, a.wbits, ndig, num_sms, st) : cudaErrorInvalidValue;
-    return g2_dispatch<true, false>(M, pl, a.wbits, ndig, num_sms, st);
+    if (probe) return ndig == 1 ? g2_dispatch<true, true>(pl, a.wbits, ndig, num_sms, st) : cudaErrorInvalidValue;
+    return g2_dispatch<true, false>(pl, a.wbits, ndig, num_sms, st);
 }
 
 cudaError_t launch_g2_down(const FfnArgs &a, int num_sms, cudaStream_t st, int32_t *probe)
@@ -1158,10 +958,8 @@ cudaError_t launch_g2_down(const FfnArgs &a, int num_sms, cudaStream_t st, int32
     p.out_ld = a.y_ld;
     p.sh_out_row0 = a.sh_y_row0;
     p.probe = probe;
-    G2Maps M;
-    if (!g2_maps(M, p, 1, a.down, a.down, a.down_sh, a.down_sh)) return cudaErrorInvalidValue;
-    if (probe) return ndig == 1 ? g2_dispatch<false, true>(M, pl, a.wbits, ndig, num_sms, st) : cudaErrorInvalidValue;
-    return g2_dispatch<false, false>(M, pl, a.wbits, ndig, num_sms, st);
+    if (probe) return ndig == 1 ? g2_dispatch<false, true>(pl, a.wbits, ndig, num_sms, st) : cudaErrorInvalidValue;
+    return g2_dispatch<false, false>(pl, a.wbits, ndig, num_sms, st);
 }
 
 }  // namespace qrx

@@ -244,6 +244,115 @@ __device__ __forceinline__ void select_token_warp(const RouterArgs &a, int t, in
     }
 }
 
+// The same selection with every value in registers, for E a multiple of 32
+// (at most 32 * NE) and groups of a multiple of 32 experts: lane l holds
+// experts l + 32 i.  Group top-2 sums come from a butterfly over (top1, top2)
+// pairs, all groups at once; the kept groups are ranked in registers; the k
+// picks are warp arg-max rounds (ties to the lower expert); the weight sum is
+// taken in double in pick order.  Same results as select_token_warp.
+template <int NE>
+__device__ __forceinline__ void select_token_warp_reg(const RouterArgs &a, int t, int lane)
+{
+    const int E = a.E, G = a.G, gs = E / G, ne = E / 32, gi = gs / 32;   // gi: i's per group
+    float s[NE], sc[NE];
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+        s[i] = 0.f;
+        sc[i] = -INFINITY;
+        if (i < ne) {
+            const int e = lane + 32 * i;
+            const float lg = a.logits[(int64_t)t * E + e];
+            s[i] = (float)(1.0 / (1.0 + exp(-(double)lg)));
+            sc[i] = __fadd_rn(s[i], a.bias[e]);
+        }
+    }
+    // group scores: group g holds i in [g*gi, (g+1)*gi) of every lane
+    float gsc[NE];
+#pragma unroll
+    for (int g = 0; g < NE; ++g) {
+        float t1 = -INFINITY, t2 = -INFINITY;
+        if (g < G) {
+#pragma unroll
+            for (int i = 0; i < NE; ++i)
+                if (i >= g * gi && i < (g + 1) * gi) {
+                    const float v = sc[i];
+                    if (v > t1) { t2 = t1; t1 = v; }
+                    else if (v > t2) { t2 = v; }
+                }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            const float b1 = __shfl_xor_sync(0xffffffffu, t1, o), b2 = __shfl_xor_sync(0xffffffffu, t2, o);
+            const float hi = fmaxf(t1, b1), lo = fmaxf(fminf(t1, b1), fmaxf(t2, b2));
+            t1 = hi;
+            t2 = lo;
+        }
+        gsc[g] = gs >= 2 ? __fadd_rn(t1, t2) : t1;
+    }
+    // kept groups: rank among the G scores (ties to the lower group)
+    uint32_t kept = 0;
+#pragma unroll
+    for (int g = 0; g < NE; ++g) {
+        if (g >= G) continue;
+        int rank = 0;
+#pragma unroll
+        for (int h = 0; h < NE; ++h)
+            if (h < G) rank += (gsc[h] > gsc[g]) || (gsc[h] == gsc[g] && h < g);
+        if (rank < a.Gk) kept |= 1u << g;
+    }
+    uint32_t avail = 0;       // bit i: expert lane + 32 i is a candidate not yet taken
+#pragma unroll
+    for (int i = 0; i < NE; ++i)
+        if (i < ne && (kept >> (i / gi) & 1u)) avail |= 1u << i;
+    int my_e = 0;
+    float my_w = 0.f;
+    double ssum = 0.0;
+    for (int j = 0; j < a.k; ++j) {
+        float best = -INFINITY;
+        int be = 0x7fffffff, bi = -1;
+#pragma unroll
+        for (int i = 0; i < NE; ++i)
+            if (avail >> i & 1u) {
+                const int e = lane + 32 * i;
+                if (be == 0x7fffffff || sc[i] > best) { best = sc[i]; be = e; bi = i; }
+            }
+        float bs = 0.f;       // the unbiased score of this lane's best candidate
+#pragma unroll
+        for (int i = 0; i < NE; ++i)
+            if (i == bi) bs = s[i];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+            const bool better = (oe != 0x7fffffff) && (be == 0x7fffffff || ob > best || (ob == best && oe < be));
+            if (better) { best = ob; be = oe; bs = os; }
+        }
+        if (be == 0x7fffffff) {      // cannot happen for a validated configuration
+            if (lane == 0) raise_status(DERR_BOUNDS);
+            return;
+        }
+        if ((be & 31) == lane) avail &= ~(1u << (be >> 5));
+        ssum += (double)bs;
+        if (lane == j) {
+            my_e = be;
+            my_w = bs;
+        }
+    }
+    const float wv = lane < a.k ? (float)((double)my_w / ssum * (double)a.rsf) : 0.f;
+    const bool keep = a.topp_thr > 0.0 ? warp_topp_keep(lane, a.k, wv, a.topp_thr) : true;
+    if (lane < a.k) {
+        a.idx[(int64_t)t * a.k + lane] = keep ? my_e : -1;
+        a.w[(int64_t)t * a.k + lane] = keep ? wv : 0.f;
+    }
+}
+
+// Whether select_token_warp_reg<8> takes this configuration.
+__host__ __device__ inline bool select_reg_ok(int E, int G)
+{
+    return E % 32 == 0 && E <= 256 && G > 0 && E % G == 0 && (E / G) % 32 == 0;
+}
+
 __global__ void __launch_bounds__(256) k_router_select(RouterArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -252,7 +361,8 @@ __global__ void __launch_bounds__(256) k_router_select(RouterArgs a)
     pdl_wait();
     pdl_trigger();
     if (t >= a.T) return;
-    select_token_warp(a, t, lane, smem_raw + select_smem_per_warp(a.E, a.G) * wid);
+    if (select_reg_ok(a.E, a.G)) select_token_warp_reg<8>(a, t, lane);
+    else select_token_warp(a, t, lane, smem_raw + select_smem_per_warp(a.E, a.G) * wid);
 }
 
 // Selection and batch-union permutation of a small batch in one CTA of 1024
@@ -264,7 +374,10 @@ __global__ void __launch_bounds__(1024, 1) k_select_permute(RouterArgs a, qrx_pe
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     pdl_wait();
     pdl_trigger();
-    if (wid < a.T) select_token_warp(a, wid, lane, smem_raw + select_smem_per_warp(a.E, a.G) * wid);
+    if (wid < a.T) {
+        if (select_reg_ok(a.E, a.G)) select_token_warp_reg<8>(a, wid, lane);
+        else select_token_warp(a, wid, lane, smem_raw + select_smem_per_warp(a.E, a.G) * wid);
+    }
     __syncthreads();        // the selection (global a.idx) is visible to the whole CTA
     permute_cta(a.idx, a.T * a.k, a.E, p, usage, reinterpret_cast<int *>(smem_raw));
 }
