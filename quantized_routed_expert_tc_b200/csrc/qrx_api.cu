@@ -65,7 +65,7 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 // Workspace regions for T tokens.
 struct Ws {
     size_t logits, counts, offsets, sorted, inv, uids, nu, xq, xd, xrec, hrec, xperm, hperm, h, y,
-        xdev, outdev, idx, w, total;
+        xdev, outdev, idx, w, g2tab, g2cnt, total;
 };
 
 Ws ws_layout(const qrx_cfg *c, int T)
@@ -98,6 +98,8 @@ Ws ws_layout(const qrx_cfg *c, int T)
     L.outdev = take((size_t)T * H * 4);
     L.idx = take(A * 4);
     L.w = take(A * 4);
+    L.g2tab = take((size_t)(4 + 4 * (std::min<int64_t>(E, A) + 1)) * 4);   // decode path: slot table
+    L.g2cnt = take((size_t)H * 4);                                          // decode path: combine counters
     L.total = off;
     return L;
 }
@@ -561,14 +563,6 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     qrx_perm perm{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.sorted),
                   at<int32_t>(ws, L.inv), at<int32_t>(ws, L.uids), at<int32_t>(ws, L.nu)};
     const RouterArgs ra = router_args(c, x, T, Wr, bias, topk_idx, topk_w, ws, topp_thr);
-    // small batches: selection and permutation in one kernel after the logits
-    const bool fused = select_permute_fused_ok(T, c->n_experts, c->n_group);
-    e = launch_router(ra, st, !fused);
-    g_pdl = true;
-    if (e != cudaSuccess || !mark(2)) return QRX_ECUDA;
-    e = fused ? launch_select_permute(ra, perm, usage, st)
-              : launch_permute(topk_idx, T, c->top_k, c->n_experts, perm, st, usage);
-    if (e != cudaSuccess || !mark(3)) return QRX_ECUDA;
     float *h = at<float>(ws, L.h), *y = at<float>(ws, L.y);
     set_routed(a, routed, &perm);
     if (shared) set_shared(a, shared);
@@ -579,6 +573,40 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     a.y_ld = c->hidden;
     a.sh_h_row0 = A;
     a.sh_y_row0 = A;
+    // decode GEMV: the gate/up kernel also selects and permutes, the down kernel also combines
+    if (!tc && g2_fuse_ok(a, c->n_group, c->topk_group)) {
+        e = launch_router(ra, st, false);
+        g_pdl = true;
+        if (e != cudaSuccess || !mark(2) || !mark(3)) return QRX_ECUDA;
+        G2Fuse f{};
+        f.logits = ra.logits;
+        f.bias = bias;
+        f.G = c->n_group;
+        f.Gk = c->topk_group;
+        f.rsf = c->routed_scaling_factor;
+        f.topp_thr = topp_thr;
+        f.idx = topk_idx;
+        f.w = topk_w;
+        f.usage = usage;
+        f.counts = perm.counts;
+        f.inv = perm.inv;
+        f.tab = at<int32_t>(ws, L.g2tab);
+        f.cnt = at<int32_t>(ws, L.g2cnt);
+        f.out = out;
+        e = launch_g2_gateup_fused(a, f, sms, st);
+        if (e != cudaSuccess || !mark(4)) return QRX_ECUDA;
+        e = launch_g2_down_fused(a, f, sms, st);
+        if (e != cudaSuccess || !mark(5) || !mark(6)) return QRX_ECUDA;
+        return QRX_OK;
+    }
+    // small batches: selection and permutation in one kernel after the logits
+    const bool fused = select_permute_fused_ok(T, c->n_experts, c->n_group);
+    e = launch_router(ra, st, !fused);
+    g_pdl = true;
+    if (e != cudaSuccess || !mark(2)) return QRX_ECUDA;
+    e = fused ? launch_select_permute(ra, perm, usage, st)
+              : launch_permute(topk_idx, T, c->top_k, c->n_experts, perm, st, usage);
+    if (e != cudaSuccess || !mark(3)) return QRX_ECUDA;
     e = launch_ffn_gateup(a, sms, st);
     if (e != cudaSuccess || !mark(4)) return QRX_ECUDA;
     e = launch_ffn_down(a, sms, st);

@@ -112,6 +112,26 @@ cudaError_t launch_ffn_down(const FfnArgs &a, int num_sms, cudaStream_t st);
 bool g2_use(const FfnArgs &a);
 cudaError_t launch_g2_gateup(const FfnArgs &a, int num_sms, cudaStream_t st, int32_t *probe = nullptr);
 cudaError_t launch_g2_down(const FfnArgs &a, int num_sms, cudaStream_t st, int32_t *probe = nullptr);
+// Layer forward with the decode GEMV: the gate/up launch also makes the
+// selection and the permutation from the router logits, and the down launch
+// also applies the weighted combine.
+struct G2Fuse {
+    const float *logits, *bias;   // router logits [T][E], score-correction bias [E]
+    int G, Gk;
+    float rsf;
+    double topp_thr;              // adaptive top-p threshold p * rsf (0: off)
+    int32_t *idx;                 // [T][k] chosen experts (out)
+    float *w;                     // [T][k] weights (out)
+    uint64_t *usage;              // per-expert counters (may be null)
+    int32_t *counts, *inv;        // permutation outputs besides those in FfnArgs
+    int32_t *tab;                 // compact slot table: 4 + 4 * (min(E, T*k) + 1) ints
+    int32_t *cnt;                 // combine counters: g2_down_groups() ints
+    float *out;                   // [T][H] layer output (down launch; null: no combine)
+};
+bool g2_fuse_ok(const FfnArgs &a, int G, int Gk);
+int g2_down_groups(const FfnArgs &a);
+cudaError_t launch_g2_gateup_fused(const FfnArgs &a, const G2Fuse &f, int num_sms, cudaStream_t st);
+cudaError_t launch_g2_down_fused(const FfnArgs &a, const G2Fuse &f, int num_sms, cudaStream_t st);
 
 cudaError_t launch_combine(const float *y_sorted, const float *y_sh, const float *w,
                            const int32_t *inv, int T, int k, int H, float *out,
