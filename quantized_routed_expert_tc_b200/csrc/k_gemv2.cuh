@@ -62,6 +62,7 @@ constexpr int G2_THREADS = 32 * G2_NW;
 constexpr int G2_TMAX = 4;                        // tokens per call
 constexpr int G2_SMEM_MAX = 227 * 1024;
 constexpr int G2_CLIST = 1024;                    // combine: row groups a CTA lists in shared memory
+constexpr int64_t G2_BW = 4;                      // cost of a warp-unit: G2_BW for its bytes, plus one per token
 
 // ---------------------------------------------------------------- records
 // Record of one input row of K codes, in shared memory:
@@ -103,7 +104,7 @@ struct G2P {
     int rec_bytes, nrec, slot_cap;   // record size, records held, slots per phase (down)
     int ms;                          // slot capacity of the tables (routed slots + 1)
     // shared-memory offsets (bytes)
-    int o_sl, o_srt, o_pre, o_seg, o_rmax, o_route, o_rec, smem;
+    int o_sl, o_srt, o_pre, o_seg, o_hmx, o_rmax, o_route, o_rec, smem;
     G2Mat m[2], msh[2];              // gate/up: m[0] gate, m[1] up; down: m[0] down
     int routed, shared;
     int32_t *counts, *offsets, *sorted, *inv, *union_ids, *n_union;   // the permutation
@@ -135,6 +136,9 @@ struct G2P {
     const float *cw;                 // [T][k] weights
     const int32_t *cinv;             // [T][k] positions (-1: none)
     float *cout;                     // [T][H]
+    // largest |h| per h row, as f32 bits (fused path; zeroed before the gate/up
+    // launch): gate/up raises it for every h value it writes, down reads it
+    uint32_t *hmax;
 };
 
 // ---------------------------------------------------------------- small helpers
@@ -272,11 +276,13 @@ __device__ void g2_build(const G2P &p, unsigned char *recs, int n, SrcFn src, bo
                      : static_cast<const void *>(static_cast<const float *>(p.x) + row * p.in_ld);
     };
     if constexpr (NDIG == 3) {
+        // the row maxima of h are known (fused down projection): one pass
+        const bool known = !gateup && p.hmax != nullptr;
         // pass 1: every row's largest magnitude; a thread's first two (row, item)
         // values stay in registers for pass 2 (item it = tid + q * threads in both)
         const int nq = (nitem + G2_THREADS - 1) / G2_THREADS;
         float cache[2][EW];
-        for (int i = 0; i < n; ++i) {
+        for (int i = 0; i < n && !known; ++i) {
             int64_t row;
             if (!src(i, row)) continue;
             const void *rp = row_ptr(row);
@@ -295,7 +301,7 @@ __device__ void g2_build(const G2P &p, unsigned char *recs, int n, SrcFn src, bo
             am = warp_max(am);
             if (lane == 0) rmax[i * G2_NW + warp] = am;
         }
-        __syncthreads();
+        if (!known) __syncthreads();
         // pass 2: digits and chunk digit sums
         for (int i = 0; i < n; ++i) {
             int64_t row;
@@ -303,8 +309,13 @@ __device__ void g2_build(const G2P &p, unsigned char *recs, int n, SrcFn src, bo
             const void *rp = row_ptr(row);
             unsigned char *rec = recs + (size_t)i * p.rec_bytes;
             float am = 0.f;
+            if (known) {
+                am = __uint_as_float(p.hmax[row]);
+                if (rnd) am = __bfloat162float(__float2bfloat16_rn(am));
+            } else {
 #pragma unroll
-            for (int w = 0; w < G2_NW; ++w) am = fmaxf(am, rmax[i * G2_NW + w]);
+                for (int w = 0; w < G2_NW; ++w) am = fmaxf(am, rmax[i * G2_NW + w]);
+            }
             const int sh = am != 0.f ? fixed_shift(am) : 0;
             const bool fast = sh >= -126 && sh <= 127;
             const float mul = fast ? __int_as_float((sh + 127) << 23) : 0.f;
@@ -313,7 +324,7 @@ __device__ void g2_build(const G2P &p, unsigned char *recs, int n, SrcFn src, bo
                 const bool act = it < nitem;
                 const int c = it >> 2, wi = it & 3, slot = i * nq + q;
                 float v[EW];
-                if (act && (!CACHE || slot >= 2)) g2_vals<EW>(rp, bf_in, rnd, it * EW, v);
+                if (act && (!CACHE || known || slot >= 2)) g2_vals<EW>(rp, bf_in, rnd, it * EW, v);
                 else
 #pragma unroll
                     for (int e = 0; e < EW; ++e) v[e] = !act ? 0.f : slot == 0 ? cache[0][e] : cache[1][e];
@@ -476,6 +487,49 @@ struct G2RouteSm {
     }
 };
 
+// CTA 0 publishes the route: choice, permutation, usage, the compact slot
+// table; and zeroes the combine counters.  Every thread of the CTA calls it.
+__device__ void g2_publish(const G2P &p, const G2RouteSm &r, G2Slots sl, int A, int nu, int nslots)
+{
+    const int tid = threadIdx.x, E = p.E;
+    {
+        for (int a = tid; a < A; a += G2_THREADS) {
+            p.idx[a] = r.ridx[a];
+            p.w[a] = r.rw[a];
+            p.inv[a] = r.pos[a];
+            if (r.pos[a] >= 0) p.sorted[r.pos[a]] = a;
+            if (r.lead[a] && p.usage)
+                atomicAdd(reinterpret_cast<unsigned long long *>(p.usage + r.ridx[a]), (unsigned long long)r.cnt[a]);
+        }
+        for (int e = tid; e <= E; e += G2_THREADS) {
+            int less = 0, cnt = 0;
+            for (int b = 0; b < A; ++b) {
+                const int f = r.ridx[b];
+                if (f < 0) continue;
+                less += f < e;
+                cnt += f == e;
+            }
+            p.offsets[e] = less;
+            if (e < E) p.counts[e] = cnt;
+        }
+        for (int u = tid; u < nu; u += G2_THREADS) p.union_ids[u] = sl.e[u];
+        for (int s = tid; s < nslots; s += G2_THREADS) {
+            p.tab_out[G2_TAB_HDR + 4 * s] = sl.e[s];
+            p.tab_out[G2_TAB_HDR + 4 * s + 1] = sl.p0[s];
+            p.tab_out[G2_TAB_HDR + 4 * s + 2] = sl.nt[s];
+            p.tab_out[G2_TAB_HDR + 4 * s + 3] = 0;
+        }
+        if (tid == 0) {
+            *p.n_union = nu;
+            p.tab_out[0] = nslots;
+            p.tab_out[1] = nu;
+            p.tab_out[2] = 0;
+            p.tab_out[3] = 0;
+        }
+        for (int i = tid; i < p.ncnt; i += G2_THREADS) p.cnt[i] = 0;
+    }
+}
+
 // The call's expert choice and batch-union permutation, made by every CTA in
 // shared memory.  Selection (README "JustVugg/colibri", section "已实现的功能":
 // DeepSeek-V3-style sigmoid router, noaux_tc): s = sigmoid(logit) in double
@@ -619,43 +673,129 @@ __device__ void g2_route(const G2P &p, int *rsm, G2Slots sl, int *srt)
         }
     }
     __syncthreads();
-    if (blockIdx.x == 0) {
-        // publish: choice, permutation, usage, the compact slot table; zero the combine counters
-        for (int a = tid; a < A; a += G2_THREADS) {
-            p.idx[a] = r.ridx[a];
-            p.w[a] = r.rw[a];
-            p.inv[a] = r.pos[a];
-            if (r.pos[a] >= 0) p.sorted[r.pos[a]] = a;
-            if (r.lead[a] && p.usage)
-                atomicAdd(reinterpret_cast<unsigned long long *>(p.usage + r.ridx[a]), (unsigned long long)r.cnt[a]);
-        }
-        for (int e = tid; e <= E; e += G2_THREADS) {
-            int less = 0, cnt = 0;
-            for (int b = 0; b < A; ++b) {
-                const int f = r.ridx[b];
-                if (f < 0) continue;
-                less += f < e;
-                cnt += f == e;
-            }
-            p.offsets[e] = less;
-            if (e < E) p.counts[e] = cnt;
-        }
-        for (int u = tid; u < nu; u += G2_THREADS) p.union_ids[u] = sl.e[u];
-        for (int s = tid; s < nslots; s += G2_THREADS) {
-            p.tab_out[G2_TAB_HDR + 4 * s] = sl.e[s];
-            p.tab_out[G2_TAB_HDR + 4 * s + 1] = sl.p0[s];
-            p.tab_out[G2_TAB_HDR + 4 * s + 2] = sl.nt[s];
-            p.tab_out[G2_TAB_HDR + 4 * s + 3] = 0;
-        }
-        if (tid == 0) {
-            *p.n_union = nu;
-            p.tab_out[0] = nslots;
-            p.tab_out[1] = nu;
-            p.tab_out[2] = 0;
-            p.tab_out[3] = 0;
-        }
-        for (int i = tid; i < p.ncnt; i += G2_THREADS) p.cnt[i] = 0;
+    if (blockIdx.x == 0) g2_publish(p, r, sl, A, nu, nslots);
+}
+
+// One token, groups of a multiple of 32 experts: the choice in four CTA steps
+// (the same arithmetic and ties as g2_route).  (1) s and the biased scores sc
+// of every expert; (2) one warp per group: the top-2 sum by a butterfly;
+// (3) every expert of a kept group (rank of its group < Gk, ties to the lower
+// group) counts, over the kept groups' experts, those with a larger sc or an
+// equal sc and a lower index -- two threads per expert, half the members
+// each -- and if the count is below k it is the pick of that rank; (4) warp 0:
+// the weight sum in double in pick order, the weights, top-p, and the sort of
+// the kept picks into the slot table.  CTA 0 publishes.  Ends with __syncthreads.
+__host__ __device__ inline bool g2_route1_ok(int T, int E, int G, int k)
+{
+    return T == 1 && G >= 1 && G <= 32 && E % G == 0 && (E / G) % 32 == 0 && k <= 32;
+}
+
+__device__ void g2_route1(const G2P &p, int *rsm, G2Slots sl, int *srt)
+{
+    const int E = p.E, G = p.G, Gk = p.Gk, k = p.k, gs = E / G;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    G2RouteSm r(rsm, 1, E, G, Gk, k);
+    float *ps = r.csc;                        // s of the pick of each rank
+    for (int e = tid; e < E; e += G2_THREADS) {
+        const float s = (float)(1.0 / (1.0 + exp(-(double)p.logits[e])));
+        r.s[e] = s;
+        r.sc[e] = __fadd_rn(s, p.bias[e]);
     }
+    __syncthreads();
+    for (int g = warp; g < G; g += G2_NW) {
+        float t1 = -INFINITY, t2 = -INFINITY;
+        for (int e = g * gs + lane; e < (g + 1) * gs; e += 32) {
+            const float v = r.sc[e];
+            if (v > t1) { t2 = t1; t1 = v; }
+            else if (v > t2) { t2 = v; }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            const float b1 = __shfl_xor_sync(0xffffffffu, t1, o), b2 = __shfl_xor_sync(0xffffffffu, t2, o);
+            const float hi = fmaxf(t1, b1), lo = fmaxf(fminf(t1, b1), fmaxf(t2, b2));
+            t1 = hi;
+            t2 = lo;
+        }
+        if (lane == 0) r.gsc[g] = __fadd_rn(t1, t2);        // gs >= 32: two members at least
+    }
+    __syncthreads();
+    // kept groups as a bit mask (every thread the same)
+    uint32_t kept = 0;
+    for (int g = 0; g < G; ++g) {
+        const float v = r.gsc[g];
+        int rank = 0;
+        for (int h = 0; h < G; ++h) {
+            const float u = r.gsc[h];
+            rank += (u > v) || (u == v && h < g);
+        }
+        if (rank < Gk) kept |= 1u << g;
+    }
+    for (int q = tid; q < 2 * E; q += G2_THREADS) {       // (expert, half) pairs on neighbouring lanes
+        const int e = q >> 1, half = q & 1;
+        const bool mine = kept >> (e / gs) & 1u;
+        int cnt = 0;
+        if (mine) {
+            const float v = r.sc[e];
+            for (uint32_t km = kept; km; km &= km - 1) {
+                const int g = __ffs(km) - 1;
+                const int b0 = g * gs + half * (gs / 2), b1 = b0 + gs / 2;
+#pragma unroll 4
+                for (int e2 = b0; e2 < b1; ++e2) {
+                    const float u = r.sc[e2];
+                    cnt += (u > v) || (u == v && e2 < e);
+                }
+            }
+        }
+        cnt += __shfl_xor_sync(0xffffffffu, cnt, 1);
+        if (mine && half == 0 && cnt < k) {
+            r.pick[cnt] = e;
+            ps[cnt] = r.s[e];
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int my_e = lane < k ? r.pick[lane] : 0;
+        const float my_s = lane < k ? ps[lane] : 0.f;
+        double ssum = 0.0;
+        for (int j = 0; j < k; ++j) ssum += (double)__shfl_sync(0xffffffffu, my_s, j);
+        const float wv = lane < k ? (float)((double)my_s / ssum * (double)p.rsf) : 0.f;
+        const bool keep = p.topp_thr > 0.0 ? warp_topp_keep(lane, k, wv, p.topp_thr) : true;
+        const bool valid = lane < k && keep;
+        const int e = valid ? my_e : -1;
+        // permutation: the kept experts are distinct; position = kept experts below
+        const unsigned vm = __ballot_sync(0xffffffffu, valid);
+        int pos = 0;
+        for (int j = 0; j < k; ++j) {
+            const int ej = __shfl_sync(0xffffffffu, e, j);
+            pos += (vm >> j & 1u) && ej < e;
+        }
+        const int nu = __popc(vm);
+        if (lane < k) {
+            r.ridx[lane] = e;
+            r.rw[lane] = keep ? wv : 0.f;
+            r.pos[lane] = valid ? pos : -1;
+            r.lead[lane] = valid;
+            r.cnt[lane] = valid ? 1 : 0;
+        }
+        if (valid) {
+            srt[pos] = lane;
+            sl.e[pos] = e;
+            sl.p0[pos] = pos;
+            sl.nt[pos] = 1;
+        }
+        if (lane == 0) {
+            const int nslots = nu + (p.shared ? 1 : 0);
+            sl.hdr[0] = nslots;
+            sl.hdr[1] = nu;
+            if (p.shared) {
+                sl.e[nu] = -1;
+                sl.p0[nu] = 0;
+                sl.nt[nu] = 1;
+            }
+        }
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) g2_publish(p, r, sl, k, sl.hdr[1], sl.hdr[0]);
 }
 
 // Slot table from a permutation in memory (gate/up without fusing; down
@@ -720,13 +860,81 @@ __device__ void g2_slots_from_perm(const G2P &p, G2Slots sl, int *srt, bool gate
     __syncthreads();
 }
 
+// This CTA's segments: its range of the slots' total cost cut into (slot,
+// first warp-unit, end warp-unit) triples, seg[0] the count.  A slot's
+// warp-units cost G2_BW + its tokens (at most TP) each.  Run by one warp; when
+// every slot costs the same the prefix is a product, else a scan into pre.
+template <int TP>
+__device__ void g2_segments(const G2P &p, G2Slots sl, int nslots, int64_t *pre, int *seg)
+{
+    const int lane = threadIdx.x & 31;
+    const int nt0 = nslots > 0 ? min(sl.nt[0], TP) : 0;
+    bool same = true;
+    for (int s = lane; s < nslots; s += 32) same = same && min(sl.nt[s], TP) == nt0;
+    same = __all_sync(0xffffffffu, same) && nt0 > 0;
+    const int64_t C = (int64_t)p.nwu * (G2_BW + nt0);          // the cost of one slot when all are the same
+    int64_t Ctot;
+    if (same) {
+        Ctot = C * nslots;
+    } else {
+        int64_t run = 0;
+        for (int s0 = 0; s0 < nslots; s0 += 32) {
+            const int s = s0 + lane;
+            int64_t cost = 0;
+            if (s < nslots) {
+                const int nt = sl.nt[s];
+                cost = nt > 0 ? (int64_t)p.nwu * (G2_BW + min(nt, TP)) : 0;
+            }
+            int64_t inc = cost;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int64_t v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            if (s < nslots) pre[s] = run + inc - cost;
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) pre[nslots] = run;
+        __syncwarp();
+        Ctot = run;
+    }
+    int64_t c0, c1;
+    if (Ctot < (int64_t)(0x7fffffff / gridDim.x)) {        // 32-bit arithmetic is exact
+        c0 = (int)Ctot * (int)blockIdx.x / (int)gridDim.x;
+        c1 = (int)Ctot * (int)(blockIdx.x + 1) / (int)gridDim.x;
+    } else {
+        c0 = Ctot * blockIdx.x / gridDim.x;
+        c1 = Ctot * (blockIdx.x + 1) / gridDim.x;
+    }
+    int nseg = 0;
+    for (int s0 = 0; s0 < nslots; s0 += 32) {
+        const int s = s0 + lane;
+        int bf = 0, be = 0;
+        if (s < nslots && sl.nt[s] > 0) {
+            const int cu = (int)G2_BW + min(sl.nt[s], TP);       // cost of one of the slot's warp-units
+            const int64_t g0 = same ? C * s : pre[s], g1 = same ? g0 + C : pre[s + 1];
+            // first unit whose cost interval starts at or after c0, and likewise for c1
+            bf = c0 <= g0 ? 0 : (c0 >= g1 ? p.nwu : ((int)(c0 - g0) + cu - 1) / cu);
+            be = c1 <= g0 ? 0 : (c1 >= g1 ? p.nwu : ((int)(c1 - g0) + cu - 1) / cu);
+        }
+        const bool has = be > bf;
+        const unsigned m = __ballot_sync(0xffffffffu, has);
+        if (has) {
+            const int i = nseg + __popc(m & ((1u << lane) - 1u));
+            seg[1 + 3 * i] = s;
+            seg[2 + 3 * i] = bf;
+            seg[3 + 3 * i] = be;
+        }
+        nseg += __popc(m);
+    }
+    if (lane == 0) seg[0] = nseg;
+}
+
 // ---------------------------------------------------------------- kernel
-// Cost of a warp-unit: G2_BW for streaming its rows plus one per token (dot work).
-constexpr int64_t G2_BW = 4;
 
 // Shared memory (offsets in G2P): slot table, srt, cost prefix, the CTA's
 // segments (slot, first and end warp-unit), row maxima, route scratch, records.
-template <int WB, int NDIG, int TP, int R, bool GATEUP, bool PROBE>
+template <int WB, int NDIG, int TP, int R, bool GATEUP, bool PROBE, int NJ>
 __global__ void __launch_bounds__(G2_THREADS, 1) k_gemv2(const __grid_constant__ G2P p)
 {
     using F = Fmt<WB>;
@@ -756,67 +964,28 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gemv2(const __grid_constant__
     }
     pdl_wait();            // gate/up: the logits or the permutation; down: h, from the kernels before
     pdl_trigger();
-    if (GATEUP && p.fuse) g2_route(p, reinterpret_cast<int *>(sm + p.o_route), sl, srt);
-    else g2_slots_from_perm(p, sl, srt, GATEUP);
+    if (GATEUP && p.fuse) {
+        if (g2_route1_ok(p.T, p.E, p.G, p.k)) g2_route1(p, reinterpret_cast<int *>(sm + p.o_route), sl, srt);
+        else g2_route(p, reinterpret_cast<int *>(sm + p.o_route), sl, srt);
+    } else {
+        g2_slots_from_perm(p, sl, srt, GATEUP);
+    }
     const int nslots = sl.hdr[0], nu = sl.hdr[1];
-    if (warp == 0) {       // cost prefix over slots, and this CTA's cost range -> segments
-        int64_t run = 0;
-        for (int s0 = 0; s0 < nslots; s0 += 32) {
-            const int s = s0 + lane;
-            int64_t cost = 0;
-            if (s < nslots) {
-                const int nt = sl.nt[s];
-                cost = nt > 0 ? (int64_t)p.nwu * (G2_BW + min(nt, TP)) : 0;
-            }
-            int64_t inc = cost;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int64_t v = __shfl_up_sync(0xffffffffu, inc, o);
-                if (lane >= o) inc += v;
-            }
-            if (s < nslots) pre[s] = run + inc - cost;
-            run += __shfl_sync(0xffffffffu, inc, 31);
+    uint32_t *hmx = reinterpret_cast<uint32_t *>(sm + p.o_hmx);
+    if (warp == 0) {
+        g2_segments<TP>(p, sl, nslots, pre, seg);
+        if (GATEUP && p.hmax) {
+            __syncwarp();
+            for (int i = lane; i < seg[0] * TP; i += 32) hmx[i] = 0u;
         }
-        if (lane == 0) pre[nslots] = run;
-        __syncwarp();
-        const int64_t Ctot = pre[nslots];
-        int64_t c0, c1;
-        if (Ctot < (int64_t)(0x7fffffff / gridDim.x)) {        // 32-bit arithmetic is exact
-            c0 = (int)Ctot * (int)blockIdx.x / (int)gridDim.x;
-            c1 = (int)Ctot * (int)(blockIdx.x + 1) / (int)gridDim.x;
-        } else {
-            c0 = Ctot * blockIdx.x / gridDim.x;
-            c1 = Ctot * (blockIdx.x + 1) / gridDim.x;
-        }
-        int nseg = 0;
-        for (int s0 = 0; s0 < nslots; s0 += 32) {
-            const int s = s0 + lane;
-            int bf = 0, be = 0;
-            if (s < nslots && sl.nt[s] > 0) {
-                const int cu = (int)G2_BW + min(sl.nt[s], TP);       // cost of one of the slot's warp-units
-                const int64_t g0 = pre[s], g1 = pre[s + 1];
-                // first unit whose cost interval starts at or after c0, and likewise for c1
-                bf = c0 <= g0 ? 0 : (c0 >= g1 ? p.nwu : ((int)(c0 - g0) + cu - 1) / cu);
-                be = c1 <= g0 ? 0 : (c1 >= g1 ? p.nwu : ((int)(c1 - g0) + cu - 1) / cu);
-            }
-            const bool has = be > bf;
-            const unsigned m = __ballot_sync(0xffffffffu, has);
-            if (has) {
-                const int i = nseg + __popc(m & ((1u << lane) - 1u));
-                seg[1 + 3 * i] = s;
-                seg[2 + 3 * i] = bf;
-                seg[3 + 3 * i] = be;
-            }
-            nseg += __popc(m);
-        }
-        if (lane == 0) seg[0] = nseg;
     }
     __syncthreads();
     const int nseg = seg[0];
     QRX_CHECK_ONLY(const int64_t n_pos = p.routed ? (int64_t)p.T * p.k : 0;)
     QRX_CHECK_ONLY(const int64_t n_out = max(n_pos, p.shared ? p.sh_out_row0 + p.T : (int64_t)0);)
 
-    const int LPR = p.lpr, nj = p.nj;
+    // NJ > 0: rows of 32 * NJ chunks, fixed at compile time (LPR = 32)
+    const int LPR = NJ > 0 ? 32 : p.lpr, nj = NJ > 0 ? NJ : p.nj;
     const int cl = lane % LPR, grp = lane / LPR;
     const G2Rec RL = g2_rec(NDIG, p.K, p.cpr);
     // after the butterfly (V <= LPR) lane cl holds value cl / rep: that value's
@@ -1109,9 +1278,11 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gemv2(const __grid_constant__
                 const int64_t o = g2_pick(orow, t);
                 QRX_CHECK_OR(o >= 0 && o < n_out, return);
                 const float sg = NDIG == 3 ? g2_pick(sig, t) : 1.f;
-                if constexpr (GATEUP)
-                    p.out[o * p.out_ld + row] = silu_mul(s0 * (sg * tot), s1 * (sg * upv));
-                else
+                if constexpr (GATEUP) {
+                    const float hv = silu_mul(s0 * (sg * tot), s1 * (sg * upv));
+                    p.out[o * p.out_ld + row] = hv;
+                    if (p.hmax) atomicMax(hmx + j * TP + t, __float_as_uint(fabsf(hv)));
+                } else
                     p.out[o * p.out_ld + row] = s0 * (sg * tot);
             };
             if (V <= LPR) {
@@ -1130,6 +1301,18 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gemv2(const __grid_constant__
                     const float s1 = GATEUP ? (routed ? p.m[NM - 1].s[(int64_t)e * p.m[NM - 1].ss + row] : p.msh[NM - 1].s[row]) : 0.f;
                     emit(idx, v[q], GATEUP ? v[q + NM - 1] : 0.f, s0, s1);
                 }
+            }
+        }
+    }
+    if constexpr (GATEUP) {
+        if (p.hmax) {
+            // the CTA's row maxima of h, one global raise per (segment, token)
+            __syncthreads();
+            for (int q = tid; q < nseg * TP; q += G2_THREADS) {
+                const int s = seg[1 + 3 * (q / TP)], t = q % TP;
+                if (t >= min(sl.nt[s], TP) || hmx[q] == 0u) continue;
+                const int64_t o = s < nu ? (int64_t)sl.p0[s] + t : p.sh_out_row0 + t;
+                atomicMax(p.hmax + o, hmx[q]);
             }
         }
     }
@@ -1236,6 +1419,8 @@ static inline bool g2_plan(G2Plan &pl, int wbits, int ndig, int K, int rows, int
     o = al(o + (p.ms + 1) * 8, 16);
     p.o_seg = o;
     o = al(o + (1 + 3 * p.ms) * 4, 16);
+    p.o_hmx = o;                                   // gate/up: largest |h| per (segment, token)
+    o = al(o + p.ms * pl.tp * 4, 16);
     p.o_route = o;
     if (G > 0) o = al(o + G2RouteSm::ints(T, E, G, Gk, k) * 4, 16);
     else if (nm == 1) o = al(o + (1 + G2_CLIST) * 4, 16);         // down: the combine's list
@@ -1259,10 +1444,10 @@ static inline bool g2_plan(G2Plan &pl, int wbits, int ndig, int K, int rows, int
     return o <= G2_SMEM_MAX;
 }
 
-template <int WB, int ND, int TP, int R, bool GU, bool PR>
+template <int WB, int ND, int TP, int R, bool GU, bool PR, int NJ = 0>
 static cudaError_t g2_go(const G2P &p, int grid, cudaStream_t st)
 {
-    auto kern = k_gemv2<WB, ND, TP, R, GU, PR>;
+    auto kern = k_gemv2<WB, ND, TP, R, GU, PR, NJ>;
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -1281,6 +1466,13 @@ static cudaError_t g2_dispatch(const G2Plan &pl, int wbits, int ndig, int grid, 
     constexpr int R1 = GU ? 2 : 4, R2 = R1 / 2;     // rows per lane: one token; several (halved)
 #define QRX_G2(WB, ND, TP, R) \
     if (wbits == WB && ndig == ND && pl.tp == TP && pl.r == R) return g2_go<WB, ND, TP, R, GU, PR>(pl.p, grid, st);
+    // rows of the common shapes (hidden 6144, expert intermediate 2048) with the chunk count fixed
+    if constexpr (!PR) {
+        if (pl.p.lpr == 32 && wbits == 4 && ndig == 3 && pl.tp == 1 && pl.r == R1) {
+            if (pl.p.nj == 6) return g2_go<4, 3, 1, R1, GU, PR, 6>(pl.p, grid, st);
+            if (pl.p.nj == 2) return g2_go<4, 3, 1, R1, GU, PR, 2>(pl.p, grid, st);
+        }
+    }
     if constexpr (PR) {        // Q8_0 with the block-sum side output
         QRX_G2(4, 1, 1, R1) QRX_G2(4, 1, 2, R1) QRX_G2(4, 1, 4, R1)
         QRX_G2(8, 1, 1, R1) QRX_G2(8, 1, 2, R1) QRX_G2(8, 1, 4, R1)
@@ -1410,6 +1602,7 @@ cudaError_t launch_g2_gateup_fused(const FfnArgs &a, const G2Fuse &f, int num_sm
     p.counts = f.counts;
     p.inv = f.inv;
     p.tab_out = f.tab;
+    p.hmax = f.hmax;
     p.cnt = f.cnt;
     p.ncnt = f.cnt ? g2_down_groups(a) : 0;
     return g2_dispatch<true, false>(pl, a.wbits, ndig, num_sms, st);
@@ -1423,6 +1616,7 @@ cudaError_t launch_g2_down_fused(const FfnArgs &a, const G2Fuse &f, int num_sms,
     G2P &p = pl.p;
     g2_down_args(p, a, nullptr);
     p.tab = f.tab;
+    p.hmax = f.hmax;
     if (f.out) {
         p.comb = 1;
         p.cnt = f.cnt;

@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(256) k_router_gemv(RouterArgs a)
 {
     __shared__ double part[RG_ROWS][4][RG_TMAX];
     pdl_trigger();                       // reads only inputs; waits before it exits
+    if (blockIdx.x == 0 && a.zero)
+        for (int i = threadIdx.x; i < a.nzero; i += blockDim.x) a.zero[i] = 0u;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int rl = w >> 2, q = w & 3;
     const int e = blockIdx.x * RG_ROWS + rl;
@@ -100,6 +102,8 @@ __global__ void __launch_bounds__(256) k_router_tile(RouterArgs a)
     __shared__ double xs[RT_T][RT_KC + 1];
     __shared__ double wsm[RT_E][RT_KC + 1];
     pdl_trigger();                       // reads only inputs; waits before it exits
+    if (blockIdx.x == 0 && blockIdx.y == 0 && a.zero)
+        for (int i = threadIdx.x; i < a.nzero; i += blockDim.x) a.zero[i] = 0u;
     const int tid = threadIdx.x;
     const int e0 = blockIdx.x * RT_E, t0 = blockIdx.y * RT_T;
     const int c0 = 0, c1 = a.H / RT_KC;

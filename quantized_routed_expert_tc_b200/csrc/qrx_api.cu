@@ -65,7 +65,7 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 // Workspace regions for T tokens.
 struct Ws {
     size_t logits, counts, offsets, sorted, inv, uids, nu, xq, xd, xrec, hrec, xperm, hperm, h, y,
-        xdev, outdev, idx, w, g2tab, g2cnt, total;
+        xdev, outdev, idx, w, g2tab, g2cnt, g2hmax, total;
 };
 
 Ws ws_layout(const qrx_cfg *c, int T)
@@ -100,6 +100,7 @@ Ws ws_layout(const qrx_cfg *c, int T)
     L.w = take(A * 4);
     L.g2tab = take((size_t)(4 + 4 * (std::min<int64_t>(E, A) + 1)) * 4);   // decode path: slot table
     L.g2cnt = take((size_t)H * 4);                                          // decode path: combine counters
+    L.g2hmax = take((size_t)(A + T) * 4);                                   // decode path: largest |h| per row
     L.total = off;
     return L;
 }
@@ -575,7 +576,10 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     a.sh_y_row0 = A;
     // decode GEMV: the gate/up kernel also selects and permutes, the down kernel also combines
     if (!tc && g2_fuse_ok(a, c->n_group, c->topk_group)) {
-        e = launch_router(ra, st, false);
+        RouterArgs rz = ra;
+        rz.zero = at<uint32_t>(ws, L.g2hmax);
+        rz.nzero = (int)(A + T);
+        e = launch_router(rz, st, false);
         g_pdl = true;
         if (e != cudaSuccess || !mark(2) || !mark(3)) return QRX_ECUDA;
         G2Fuse f{};
@@ -593,6 +597,7 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
         f.tab = at<int32_t>(ws, L.g2tab);
         f.cnt = at<int32_t>(ws, L.g2cnt);
         f.out = out;
+        f.hmax = rz.zero;
         e = launch_g2_gateup_fused(a, f, sms, st);
         if (e != cudaSuccess || !mark(4)) return QRX_ECUDA;
         e = launch_g2_down_fused(a, f, sms, st);

@@ -54,6 +54,8 @@ struct RouterArgs {
     int32_t *idx;           // [T][k]
     float *w;               // [T][k]
     double topp_thr;        // adaptive top-p: p * rsf; 0 = off
+    uint32_t *zero;         // if set: zero[0, nzero) cleared by the logits kernel (scratch of the next kernels)
+    int nzero;
 };
 // the logits kernel, then (select) the selection kernel
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t st, bool select = true);
@@ -127,6 +129,7 @@ struct G2Fuse {
     int32_t *tab;                 // compact slot table: 4 + 4 * (min(E, T*k) + 1) ints
     int32_t *cnt;                 // combine counters: g2_down_groups() ints
     float *out;                   // [T][H] layer output (down launch; null: no combine)
+    uint32_t *hmax;               // [T*k + T] largest |h| per h row (bits), zeroed by the logits kernel
 };
 bool g2_fuse_ok(const FfnArgs &a, int G, int Gk);
 int g2_down_groups(const FfnArgs &a);
