@@ -933,6 +933,7 @@ cudaError_t launch_act_digits(const FfnArgs &a, cudaStream_t st)
 cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
 {
     if (ffn_use_tc(a)) return launch_ffn_tc_gateup(a, num_sms, st);
+    if (a.T >= 2 && gm_use(a)) return launch_gm_gateup(a, num_sms, st);
     if (g2_use(a)) return launch_g2_gateup(a, num_sms, st);
     const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
     GemvPlan pl;
@@ -966,6 +967,7 @@ cudaError_t launch_ffn_gateup(const FfnArgs &a, int num_sms, cudaStream_t st)
 cudaError_t launch_ffn_down(const FfnArgs &a, int num_sms, cudaStream_t st)
 {
     if (ffn_use_tc(a)) return launch_ffn_tc_down(a, num_sms, st);
+    if (a.T >= 2 && gm_use(a)) return launch_gm_down(a, num_sms, st);
     if (g2_use(a)) return launch_g2_down(a, num_sms, st);
     const int ndig = a.afmt == QRX_A_Q8_0 ? 1 : 3;
     GemvPlan pl;

@@ -19,6 +19,7 @@
 #include "k_ffn_gemv.cuh"
 #include "k_ffn_tc.cuh"
 #include "k_gemv2.cuh"
+#include "k_gmma.cuh"
 #include "k_combine.cuh"
 
 using namespace qrx;
@@ -555,7 +556,7 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     a.hperm_ready = 1;
     if (!mark(0)) return QRX_ECUDA;
     // the tensor-core path needs no digit records; the decode GEMV builds its own
-    const bool tc = ffn_use_tc(a), own_records = tc || g2_use(a);
+    const bool tc = ffn_use_tc(a), own_records = tc || g2_use(a) || gm_use(a);
     cudaError_t e = own_records ? cudaSuccess : launch_act_digits(a, st);
     if (e != cudaSuccess || !mark(1)) return QRX_ECUDA;
     // 2.. the rest chained with programmatic dependent launch (the first kernel
@@ -575,7 +576,7 @@ int moe_forward_impl(const qrx_cfg *c, const void *x, int32_t T, const float *Wr
     a.sh_h_row0 = A;
     a.sh_y_row0 = A;
     // decode GEMV: the gate/up kernel also selects and permutes, the down kernel also combines
-    if (!tc && g2_fuse_ok(a, c->n_group, c->topk_group)) {
+    if (!tc && T == 1 && g2_fuse_ok(a, c->n_group, c->topk_group)) {
         RouterArgs rz = ra;
         rz.zero = at<uint32_t>(ws, L.g2hmax);
         rz.nzero = (int)(A + T);

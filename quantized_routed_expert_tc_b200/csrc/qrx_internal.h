@@ -132,6 +132,10 @@ struct G2Fuse {
     uint32_t *hmax;               // [T*k + T] largest |h| per h row (bits), zeroed by the logits kernel
 };
 bool g2_fuse_ok(const FfnArgs &a, int G, int Gk);
+// multi-token GEMV on tensor cores (2 <= T <= 64, int4 / int8 weights)
+bool gm_use(const FfnArgs &a);
+cudaError_t launch_gm_gateup(const FfnArgs &a, int num_sms, cudaStream_t st);
+cudaError_t launch_gm_down(const FfnArgs &a, int num_sms, cudaStream_t st);
 int g2_down_groups(const FfnArgs &a);
 cudaError_t launch_g2_gateup_fused(const FfnArgs &a, const G2Fuse &f, int num_sms, cudaStream_t st);
 cudaError_t launch_g2_down_fused(const FfnArgs &a, const G2Fuse &f, int num_sms, cudaStream_t st);
