@@ -25,7 +25,8 @@ namespace qrx {
 constexpr int RT_T = 32, RT_E = 64, RT_KC = 32;
 
 constexpr int RG_ROWS = 2;           // experts per CTA in k_router_gemv
-constexpr int RG_TMAX = 64;          // tokens handled by k_router_gemv
+constexpr int RG_TMAX = 64;          // tokens k_router_gemv can handle
+constexpr int RG_TSPLIT = 4;         // tokens above which the split-K tile kernel is used (when given its scratch)
 
 template <bool XBF16>
 __device__ __forceinline__ float4 load_x4(const void *x, int64_t off)
@@ -162,6 +163,117 @@ __global__ void __launch_bounds__(256) k_router_tile(RouterArgs a)
             if (t < a.T && e < a.E) a.logits[(int64_t)t * a.E + e] = (float)acc[i][j];
         }
     pdl_wait();
+}
+
+
+// Many tokens, split over K: a CTA computes the f64 partial dots of 64
+// tokens x 64 experts over one K slice (32-wide chunks of x and Wr staged in
+// shared memory, 4 x 4 outputs per thread); the CTA that finishes a tile's
+// last slice (a per-tile counter that it resets) adds the slices' partials in
+// slice order and rounds each logit to f32 once.  Slices keep the grid near
+// two CTAs per SM when there are few token tiles.
+constexpr int RS_T = 64, RS_E = 64, RS_KC = 32;
+
+template <bool XBF16>
+__global__ void __launch_bounds__(256) k_router_split(RouterArgs a, int nslice, double *part, int *tilecnt)
+{
+    __shared__ double xs[RS_KC][RS_T + 1];
+    __shared__ double wsm[RS_KC][RS_E + 1];
+    __shared__ int last;
+    pdl_trigger();                       // reads only inputs; waits before it exits
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && a.zero)
+        for (int i = threadIdx.x; i < a.nzero; i += blockDim.x) a.zero[i] = 0u;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int e0 = blockIdx.x * RS_E, t0 = blockIdx.y * RS_T, sl = blockIdx.z;
+    const int kper = a.H / nslice, kb0 = sl * kper;
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int kb = kb0; kb < kb0 + kper; kb += RS_KC) {
+        // x: 64 tokens x 32 k, 8 per thread; Wr: 64 experts x 32 k, 8 per thread
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int idx = tid + 256 * q;
+            const int rr = idx >> 5, kk = idx & 31;
+            const int t = t0 + rr, e = e0 + rr;
+            double xv = 0.0;
+            if (t < a.T) {
+                if constexpr (XBF16)
+                    xv = (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(a.x)[(int64_t)t * a.H + kb + kk]);
+                else
+                    xv = (double)reinterpret_cast<const float *>(a.x)[(int64_t)t * a.H + kb + kk];
+            }
+            xs[kk][rr] = xv;
+            wsm[kk][rr] = e < a.E ? (double)a.Wr[(int64_t)e * a.H + kb + kk] : 0.0;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int kk = 0; kk < RS_KC; ++kk) {
+            double xv[4], wv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xv[i] = xs[kk][ty + 16 * i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) wv[j] = wsm[kk][tx + 16 * j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fma(xv[i], wv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+    if (nslice == 1) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int t = t0 + ty + 16 * i, e = e0 + tx + 16 * j;
+                if (t < a.T && e < a.E) a.logits[(int64_t)t * a.E + e] = (float)acc[i][j];
+            }
+        pdl_wait();
+        return;
+    }
+    const int64_t TE = (int64_t)a.T * a.E;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = t0 + ty + 16 * i, e = e0 + tx + 16 * j;
+            if (t < a.T && e < a.E) part[sl * TE + (int64_t)t * a.E + e] = acc[i][j];
+        }
+    __threadfence();
+    __syncthreads();
+    const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+    if (tid == 0) {
+        const int done = atomicAdd(tilecnt + tile, 1);
+        last = done == nslice - 1;
+        if (last) tilecnt[tile] = 0;             // ready for the next call
+    }
+    __syncthreads();
+    if (last) {
+        __threadfence();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int t = t0 + ty + 16 * i, e = e0 + tx + 16 * j;
+                if (t >= a.T || e >= a.E) continue;
+                double sum = 0.0;
+                for (int q = 0; q < nslice; ++q) sum += __ldcg(part + q * TE + (int64_t)t * a.E + e);
+                a.logits[(int64_t)t * a.E + e] = (float)sum;
+            }
+    }
+    pdl_wait();
+}
+
+// Slices for the split kernel: about two CTAs per SM, K slices of whole chunks.
+inline int router_slices(int T, int E, int H)
+{
+    const int tiles = ((E + RS_E - 1) / RS_E) * ((T + RS_T - 1) / RS_T);
+    int s = 1;
+    while (tiles * s * 2 <= 2 * 148 && (H / RS_KC) % (s * 2) == 0 && s * 2 <= 64) s *= 2;
+    return s;
 }
 
 // One warp per token.  Dynamic shared memory per warp: s[E], sc[E] (f32),
@@ -429,10 +541,19 @@ cudaError_t launch_topp_prune(int32_t *idx, float *w, int T, int k, double thr, 
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t st, bool select)
 {
     cudaError_t err;
-    if (a.T <= RG_TMAX && a.H <= 16 * 32 * RG_W4) {
+    if (a.T <= RG_TSPLIT && a.H <= 16 * 32 * RG_W4) {
         const unsigned grid = (unsigned)((a.E + RG_ROWS - 1) / RG_ROWS);
         err = launch_k(a.x_bf16 ? k_router_gemv<true> : k_router_gemv<false>, dim3(grid), dim3(256), 0,
                        st, a);
+    } else if (a.part && a.tilecnt && a.H % RS_KC == 0) {
+        const int ns = router_slices(a.T, a.E, a.H);
+        dim3 grid((a.E + RS_E - 1) / RS_E, (a.T + RS_T - 1) / RS_T, ns);
+        if (ns > 1) {                            // the tile counters start at zero (the workspace is not cleared)
+            err = cudaMemsetAsync(a.tilecnt, 0, sizeof(int) * grid.x * grid.y, st);
+            if (err != cudaSuccess) return err;
+        }
+        err = launch_k(a.x_bf16 ? k_router_split<true> : k_router_split<false>, grid, dim3(256), 0, st, a, ns,
+                       a.part, a.tilecnt);
     } else {
         dim3 grid((a.E + RT_E - 1) / RT_E, (a.T + RT_T - 1) / RT_T);
         err = launch_k(a.x_bf16 ? k_router_tile<true> : k_router_tile<false>, grid, dim3(256), 0, st, a);

@@ -66,7 +66,7 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 // Workspace regions for T tokens.
 struct Ws {
     size_t logits, counts, offsets, sorted, inv, uids, nu, xq, xd, xrec, hrec, xperm, hperm, h, y,
-        xdev, outdev, idx, w, g2tab, g2cnt, g2hmax, total;
+        xdev, outdev, idx, w, g2tab, g2cnt, g2hmax, rpart, rcnt, total;
 };
 
 Ws ws_layout(const qrx_cfg *c, int T)
@@ -102,6 +102,11 @@ Ws ws_layout(const qrx_cfg *c, int T)
     L.g2tab = take((size_t)(4 + 4 * (std::min<int64_t>(E, A) + 1)) * 4);   // decode path: slot table
     L.g2cnt = take((size_t)H * 4);                                          // decode path: combine counters
     L.g2hmax = take((size_t)(A + T) * 4);                                   // decode path: largest |h| per row
+    {
+        const int ns = router_slices(T, (int)E, (int)H);
+        L.rpart = take(ns > 1 ? (size_t)ns * T * E * 8 : 8);                 // router split-K partials
+    }
+    L.rcnt = take((size_t)((E + 63) / 64) * ((T + 63) / 64) * 4);          // router split-K tile counters
     L.total = off;
     return L;
 }
@@ -328,6 +333,8 @@ static RouterArgs router_args(const qrx_cfg *c, const void *x, int32_t T, const 
     a.k = c->top_k;
     a.rsf = c->routed_scaling_factor;
     a.logits = at<float>(ws, L.logits);
+    a.part = at<double>(ws, L.rpart);
+    a.tilecnt = at<int>(ws, L.rcnt);
     a.idx = topk_idx;
     a.w = topk_w;
     a.topp_thr = topp_thr;

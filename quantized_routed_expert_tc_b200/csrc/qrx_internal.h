@@ -56,6 +56,8 @@ struct RouterArgs {
     double topp_thr;        // adaptive top-p: p * rsf; 0 = off
     uint32_t *zero;         // if set: zero[0, nzero) cleared by the logits kernel (scratch of the next kernels)
     int nzero;
+    double *part;           // split-K scratch: slices x T x E doubles (null: no split kernel)
+    int *tilecnt;           // split-K per-tile counters, zero between calls
 };
 // the logits kernel, then (select) the selection kernel
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t st, bool select = true);
