@@ -92,26 +92,54 @@ def uses_tensor_cores(wl) -> bool:
     return wl.afmt == 2 and wl.wbits == 4 and wl.T >= TC_MIN_T
 
 
-DECODE_T_MAX = 4        # calls of up to this many tokens run the decode GEMV (k_gemv2)
-
-
 def uses_decode_gemv(wl) -> bool:
-    return not uses_tensor_cores(wl) and wl.T <= DECODE_T_MAX
+    """One-token calls: the decode GEMV (k_gemv2), with the selection and the
+    permutation fused into its gate/up launch and the combine into its down."""
+    return not uses_tensor_cores(wl) and wl.T == 1
+
+
+def uses_mma_gemv(wl) -> bool:
+    """Calls of 2..64 tokens over int4 / int8 weights: the multi-token GEMV on
+    tensor cores (k_gmma)."""
+    return not uses_tensor_cores(wl) and 2 <= wl.T <= 64 and wl.wbits in (4, 8)
+
+
+def gemv_kernel(wl) -> str:
+    return "k_gemv2" if uses_decode_gemv(wl) else ("k_gmma" if uses_mma_gemv(wl) else "k_ffn_gemv")
+
+
+def launches_per_call(wl) -> int:
+    """Library kernels per layer call (top-p and usage add none):
+    one token: logits, gate/up (+ selection, permutation), down (+ combine) = 3;
+    2..32 tokens: logits, selection + permutation, gate/up, down, combine = 5
+    (64 tokens: selection and permutation apart, 6); tensor-core engine:
+    logits, selection, permutation, token gather, gate/up, down, combine = 7;
+    other GEMV shapes: activation records, logits, selection, permutation,
+    gate/up, h records, down, combine = 8."""
+    if uses_tensor_cores(wl):
+        return 7
+    if uses_decode_gemv(wl):
+        return 3
+    if uses_mma_gemv(wl):
+        return 5 if wl.T <= 32 else 6
+    return 8
 
 
 def dtype_label(wl) -> str:
     """The arithmetic the expert FFN computes in.  GEMV engines: exact int32 sums
     of int8 activation digits times the packed codes -- f32 / bf16 activations as
     three int8 digit planes of a 22-bit fixed point (one power-of-two scale per
-    row in the decode GEMV, per 32-block in the multi-token GEMV), Q8_0 as its
+    row in the decode and multi-token GEMVs, per 32-block in the older GEMV
+    engine), Q8_0 as its
     int8 codes with f32 block scales; the tensor-core engine: bf16 x bf16 -> f32."""
     if uses_tensor_cores(wl):
         return "bf16"
     w = f"int{wl.wbits}"
+    mma = ", tensor-core mma" if uses_mma_gemv(wl) else ""
     if wl.afmt == 1:
-        return f"int8 (Q8_0) x {w} -> int32"
+        return f"int8 (Q8_0) x {w} -> int32{mma}"
     src = "bf16" if wl.afmt == 2 else "f32"
-    return f"int8x3 digit planes (22-bit fixed point of {src}) x {w} -> int32"
+    return f"int8x3 digit planes (22-bit fixed point of {src}) x {w} -> int32{mma}"
 
 
 # How the dominant kernel's duration is taken: events placed between the layer's
@@ -163,6 +191,7 @@ def kernel_source_hash(kernel: str = "k_gemv2_gateup") -> str:
     h = hashlib.sha256()
     files = ("k_ffn_tc.cuh", "qrx_dev.cuh") if kernel.startswith("k_ffn_tc") else \
         ("k_gemv2.cuh", "qrx_dev.cuh") if kernel.startswith("k_gemv2") else \
+        ("k_gmma.cuh", "k_gemv2.cuh", "qrx_dev.cuh") if kernel.startswith("k_gmma") else \
         ("k_ffn_gemv.cuh", "qrx_dev.cuh")
     for f in files:
         with open(os.path.join(ROOT, "quantized_routed_expert_tc_b200", "csrc", f), encoding="utf-8") as fh:
@@ -540,8 +569,7 @@ def run_qrx(args, wl, rank, world, local_rank):
         tc_peak, tc_peak_kind = tensor_peak()
     nu_all = np.array([unions[i % npool] for i in range(args.steps)], dtype=np.float64)
     weight_gbs = float(((nu_all + 1) * exp_bytes).mean() / (ms_step / 1e3) / 1e9)
-    decode = uses_decode_gemv(wl)
-    gv_kernel = "k_gemv2" if decode else "k_ffn_gemv"
+    gv_kernel = gemv_kernel(wl)
     traffic = recorded_traffic("k_ffn_tc_gateup" if tc else f"{gv_kernel}_gateup", wl.name)
 
     e2e = None
@@ -582,12 +610,7 @@ def run_qrx(args, wl, rank, world, local_rank):
 
     if rank == 0:
         stages = ["act_records", "router", "permute", "gateup", "down", "combine"]
-        # library kernels per layer call: decode GEMV (T <= 4): router (dot +
-        # selection), permutation, gate/up, down, combine = 6; multi-token GEMV:
-        # activation records, router (2), permutation, gate/up, h records, down,
-        # combine = 8; tensor-core engine: router (2), permutation, token gather,
-        # gate/up, down, combine = 7 (top-p and usage add none)
-        launches_per_step = 7 if tc else (6 if decode else 8)
+        launches_per_step = launches_per_call(wl)
         line = {
             "metric": METRIC, "value": T * world / (ms_step / 1e3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -604,7 +627,9 @@ def run_qrx(args, wl, rank, world, local_rank):
             "reuse_ratio": float(np.mean(T * k / nu)),
             "stage_us": {s: float(per[:, j].mean() * 1e3) for j, s in enumerate(stages)},
             "stage_note": "from qrx_moe_forward_profiled: events between kernels disable the "
-                          "launch overlap, so the stages sum to more than ms_per_step",
+                          "launch overlap, so the stages sum to more than ms_per_step" +
+                          ("; one-token calls fuse the selection and permutation into gate/up "
+                           "and the combine into down" if uses_decode_gemv(wl) else ""),
             "roofline": ({"kernel": "k_ffn_tc (gate/up + SwiGLU, tcgen05)", "bound": "tensor",
                           "achieved": tc_achieved, "peak": tc_peak, "unit": "TFLOP/s",
                           "frac": tc_achieved / tc_peak, "peak_kind": tc_peak_kind,
