@@ -102,7 +102,8 @@ struct G2P {
     int lpr, gpw, nj;                // lanes per row, row groups per warp, chunks per lane per row
     int rw, nwu;                     // rows per warp-unit (per matrix), warp-units per slot
     int rec_bytes, nrec, slot_cap;   // record size, records held, slots per phase (down)
-    int ntile;                       // multi-token kernel: bytes of a warp's tile
+    int ntile;                       // multi-token kernel: bytes of a warp's tile ring
+    int allrec;                      // multi-token gate/up: one record per token of the call, built once
     int ms;                          // slot capacity of the tables (routed slots + 1)
     // shared-memory offsets (bytes)
     int o_sl, o_srt, o_pre, o_seg, o_hmx, o_rmax, o_route, o_rec, smem;

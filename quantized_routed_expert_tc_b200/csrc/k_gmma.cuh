@@ -44,6 +44,15 @@ constexpr int GM_ROWS = 16;                       // rows of each matrix per war
 constexpr int GM_SCB = 64;                        // bytes of a row per streaming step
 constexpr int GM_TSTRIDE = 80;                    // bytes per row of a warp's tile (64 + 16: ldmatrix without bank conflicts)
 constexpr int GM_COST_ROWS = 16;                  // cost of a warp-unit: 16 for its bytes, plus one per token
+constexpr int GM_STAGES = 3;                      // tiles in a warp's copy ring
+
+__device__ __forceinline__ void gm_cp16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void gm_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void gm_wait_groups() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ void gm_mma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                        uint32_t b1, bool uns)
@@ -179,6 +188,27 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
     const uint32_t tile_s = (uint32_t)__cvta_generic_to_shared(tile);
     const G2Rec RL = g2_rec(NDIG, p.K, p.cpr);
 
+    // OFF times each record's digit total per plane (fixed point, int4), records [i0, i1)
+    auto totals = [&](int i0, int i1) {
+        if constexpr (NDIG == 3 && WB == 4) {
+            for (int q = warp; q < (i1 - i0) * 3; q += G2_NW) {
+                const int i = i0 + q / 3, pl = q % 3;
+                const unsigned char *rec = recs + (size_t)i * p.rec_bytes;
+                int sacc = 0;
+                for (int c = lane; c < p.cpr; c += 32) sacc += reinterpret_cast<const int *>(rec + RL.csum + (size_t)c * 16)[pl];
+#pragma unroll
+                for (int o = 16; o; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
+                if (lane == 0) tot[i * 4 + pl] = F::OFF * sacc;
+            }
+            __syncthreads();
+        }
+    };
+    const bool allrec = GATEUP && p.allrec;
+    if (allrec) {
+        // every token's record, before the dependency wait: x is an input of the call
+        g2_build<WB, NDIG, false>(p, recs, p.T, [](int i, int64_t &row) { row = i; return true; }, true, rmax);
+        totals(0, p.T);
+    }
     pdl_wait();            // the permutation and (down) h, from the kernels before
     pdl_trigger();
     g2_slots_from_perm(p, sl, srt, GATEUP);
@@ -191,12 +221,13 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
     QRX_CHECK_ONLY(const int64_t n_pos = p.routed ? (int64_t)p.T * p.k : 0;)
     QRX_CHECK_ONLY(const int64_t n_out = max(n_pos, p.shared ? p.sh_out_row0 + p.T : (int64_t)0);)
 
-    for (int ph0 = 0; ph0 < nseg; ph0 += p.slot_cap) {
-        const int ph1 = min(nseg, ph0 + p.slot_cap);
+    const int plen = allrec ? nseg : p.slot_cap;
+    for (int ph0 = 0; ph0 < nseg; ph0 += plen) {
+        const int ph1 = min(nseg, ph0 + plen);
         if (ph0 > 0) __syncthreads();                     // every warp is done with the last phase's records
         // records of the phase's tokens: instance j's token i at record (j - ph0) * NTOK + i
         bool ok = true;
-        g2_build<WB, NDIG, false>(p, recs, (ph1 - ph0) * NTOK,
+        if (!allrec) g2_build<WB, NDIG, false>(p, recs, (ph1 - ph0) * NTOK,
                                   [&](int i, int64_t &row) {
                                       const int s = seg[1 + 3 * (ph0 + i / NTOK)], tk = i % NTOK;
                                       if (tk >= sl.nt[s]) return false;
@@ -216,19 +247,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                                   },
                                   GATEUP, rmax);
         if (!ok) return;
-        if constexpr (NDIG == 3 && WB == 4) {
-            // per record and plane: OFF times the digit total over all chunks
-            for (int q = warp; q < (ph1 - ph0) * NTOK * 3; q += G2_NW) {
-                const int i = q / 3, pl = q % 3;
-                const unsigned char *rec = recs + (size_t)i * p.rec_bytes;
-                int sacc = 0;
-                for (int c = lane; c < p.cpr; c += 32) sacc += reinterpret_cast<const int *>(rec + RL.csum + (size_t)c * 16)[pl];
-#pragma unroll
-                for (int o = 16; o; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
-                if (lane == 0) tot[i * 4 + pl] = F::OFF * sacc;
-            }
-            __syncthreads();
-        }
+        if (!allrec) totals(0, (ph1 - ph0) * NTOK);
         int ntot = 0;
         for (int j = ph0; j < ph1; ++j) ntot += seg[3 + 3 * j] - seg[2 + 3 * j];
         const int f0 = (int)((int64_t)ntot * warp / G2_NW), f1 = (int)((int64_t)ntot * (warp + 1) / G2_NW);
@@ -243,6 +262,11 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
             const int e = routed ? sl.e[s] : 0;
             const int p0 = sl.p0[s], nt = min(sl.nt[s], NTOK);
             const int rbase = (j - ph0) * NTOK;              // the instance's first record
+            // record of the instance's token tk: the token's own (allrec) or the phase's
+            auto recidx = [&](int tk) -> int {
+                if (!allrec) return rbase + tk;
+                return routed ? srt[p0 + tk] / p.k : p0 + tk;
+            };
             const int r0 = u * GM_ROWS;
             // this lane's two rows of each matrix, 16 bytes at 16 t of every 64-byte step
             const uint8_t *wa[NM], *wb[NM];
@@ -258,7 +282,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
             for (int jj = 0; jj < NTL; ++jj) {
                 const int col = 8 * jj + g;
                 const int tk = NDIG == 3 ? col / 3 : col, pl = NDIG == 3 ? col % 3 : 0;
-                boff[jj] = tk < nt ? p.o_rec + (rbase + tk) * p.rec_bytes + pl * NQ * p.cpr * 16 : -1;
+                boff[jj] = tk < nt ? p.o_rec + recidx(tk) * p.rec_bytes + pl * NQ * p.cpr * 16 : -1;
             }
             // Q8_0: the tokens of this lane's accumulator columns 8 jj + 2 t, + 1
             int coff[NTL][2];
@@ -267,7 +291,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int tk = 8 * jj + 2 * t + h;
-                    coff[jj][h] = NDIG == 1 && tk < nt ? p.o_rec + (rbase + tk) * p.rec_bytes + RL.hdr : -1;
+                    coff[jj][h] = NDIG == 1 && tk < nt ? p.o_rec + recidx(tk) * p.rec_bytes + RL.hdr : -1;
                 }
             int acc[NM][NTL][4];
             float facc[NM][NTL][4];
@@ -281,21 +305,21 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                         facc[m][jj][q] = 0.f;
                     }
             const int nsc = p.row_bytes / GM_SCB;
-            auto ld = [&](int sc, uint4 (&b)[NM][2]) {
+            constexpr int TB = NM * GM_ROWS * GM_TSTRIDE;      // bytes of one tile
+            // the copies of step sc into tile sc % GM_STAGES (16 bytes per lane per row)
+            auto issue = [&](int sc) {
+                if (sc < nsc) {
+                    const uint32_t tb = tile_s + (sc % GM_STAGES) * TB;
 #pragma unroll
-                for (int m = 0; m < NM; ++m) {
-                    b[m][0] = ld_stream16(wa[m] + (size_t)sc * GM_SCB);
-                    b[m][1] = ld_stream16(wb[m] + (size_t)sc * GM_SCB);
+                    for (int m = 0; m < NM; ++m) {
+                        gm_cp16(tb + (m * 16 + g) * GM_TSTRIDE + 16 * t, wa[m] + (size_t)sc * GM_SCB);
+                        gm_cp16(tb + (m * 16 + g + 8) * GM_TSTRIDE + 16 * t, wb[m] + (size_t)sc * GM_SCB);
+                    }
                 }
+                gm_commit();                                   // one group per step, empty past the end
             };
-            auto step = [&](int sc, const uint4 (&b)[NM][2]) {
-                __syncwarp();                                  // the last step's ldmatrix reads are done
-#pragma unroll
-                for (int m = 0; m < NM; ++m) {
-                    *reinterpret_cast<uint4 *>(tile + (m * 16 + g) * GM_TSTRIDE + 16 * t) = b[m][0];
-                    *reinterpret_cast<uint4 *>(tile + (m * 16 + g + 8) * GM_TSTRIDE + 16 * t) = b[m][1];
-                }
-                __syncwarp();
+            auto step = [&](int sc) {
+                const uint32_t tb = tile_s + (sc % GM_STAGES) * TB;
                 // aw[m][piece][half]: word t of 16-byte piece `piece` of row g (half 0) or g + 8 (half 1)
                 uint32_t aw[NM][4][2];
 #pragma unroll
@@ -306,12 +330,32 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                         const int mi = lane >> 3, rr = lane & 7;
                         const int row = rr + 8 * (mi & 1), piece = 2 * xq + (mi >> 1);
                         uint32_t r4[4];
-                        gm_ldsm4(tile_s + (m * 16 + row) * GM_TSTRIDE + piece * 16, r4);
+                        gm_ldsm4(tb + (m * 16 + row) * GM_TSTRIDE + piece * 16, r4);
                         aw[m][2 * xq][0] = r4[0];
                         aw[m][2 * xq][1] = r4[1];
                         aw[m][2 * xq + 1][0] = r4[2];
                         aw[m][2 * xq + 1][1] = r4[3];
                     }
+                // the step's B fragments, all issued before the first mma
+                uint32_t bf[NBLK][NTL][2];
+#pragma unroll
+                for (int kb = 0; kb < NBLK; ++kb) {
+                    const int c = WB == 4 ? NBLK * sc + kb : 4 * sc + 2 * kb;   // record chunk of k = 0 .. 15
+#pragma unroll
+                    for (int jj = 0; jj < NTL; ++jj) {
+                        bf[kb][jj][0] = bf[kb][jj][1] = 0;
+                        if (boff[jj] >= 0) {
+                            if constexpr (WB == 4) {
+                                const uint2 bb = *reinterpret_cast<const uint2 *>(sm + boff[jj] + ((t >> 1) * p.cpr + c) * 16 + (t & 1) * 8);
+                                bf[kb][jj][0] = bb.x;
+                                bf[kb][jj][1] = bb.y;
+                            } else {
+                                bf[kb][jj][0] = *reinterpret_cast<const uint32_t *>(sm + boff[jj] + c * 16 + 4 * t);
+                                bf[kb][jj][1] = *reinterpret_cast<const uint32_t *>(sm + boff[jj] + (c + 1) * 16 + 4 * t);
+                            }
+                        }
+                    }
+                }
 #pragma unroll
                 for (int kb = 0; kb < NBLK; ++kb) {
                     uint32_t a[NM][4];
@@ -331,24 +375,14 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                             a[m][3] = aw[m][2 * kb + 1][1];
                         }
                     }
-                    const int c = WB == 4 ? NBLK * sc + kb : 4 * sc + 2 * kb;   // record chunk of k = 0 .. 15
+                    const int c = WB == 4 ? NBLK * sc + kb : 4 * sc + 2 * kb;
                     const int blk = WB == 4 ? c : c >> 1;                        // Q8_0 block
 #pragma unroll
                     for (int jj = 0; jj < NTL; ++jj) {
-                        uint32_t b0 = 0, b1 = 0;
-                        if (boff[jj] >= 0) {
-                            if constexpr (WB == 4) {
-                                const uint2 bb = *reinterpret_cast<const uint2 *>(sm + boff[jj] + ((t >> 1) * p.cpr + c) * 16 + (t & 1) * 8);
-                                b0 = bb.x;
-                                b1 = bb.y;
-                            } else {
-                                b0 = *reinterpret_cast<const uint32_t *>(sm + boff[jj] + c * 16 + 4 * t);
-                                b1 = *reinterpret_cast<const uint32_t *>(sm + boff[jj] + (c + 1) * 16 + 4 * t);
-                            }
-                        }
                         if constexpr (NDIG == 3) {
 #pragma unroll
-                            for (int m = 0; m < NM; ++m) gm_mma(acc[m][jj], a[m][0], a[m][1], a[m][2], a[m][3], b0, b1, WB == 4);
+                            for (int m = 0; m < NM; ++m)
+                                gm_mma(acc[m][jj], a[m][0], a[m][1], a[m][2], a[m][3], bf[kb][jj][0], bf[kb][jj][1], WB == 4);
                         } else {
                             // started from the block's offset correction, scaled by the token's d_b
                             int cr[2] = {0, 0};
@@ -362,7 +396,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
 #pragma unroll
                             for (int m = 0; m < NM; ++m) {
                                 int d4[4] = {cr[0], cr[1], cr[0], cr[1]};
-                                gm_mma(d4, a[m][0], a[m][1], a[m][2], a[m][3], b0, b1, WB == 4);
+                                gm_mma(d4, a[m][0], a[m][1], a[m][2], a[m][3], bf[kb][jj][0], bf[kb][jj][1], WB == 4);
 #pragma unroll
                                 for (int q = 0; q < 4; ++q) facc[m][jj][q] = fmaf(dq[q & 1], (float)d4[q], facc[m][jj][q]);
                             }
@@ -370,15 +404,18 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                     }
                 }
             };
-            uint4 bufA[NM][2], bufB[NM][2];
-            ld(0, bufA);
+            // the ring: GM_STAGES - 1 steps in flight ahead of the one computed
+            __syncwarp();                                      // the last unit's tile reads are done
+#pragma unroll
+            for (int q = 0; q < GM_STAGES - 1; ++q) issue(q);
 #pragma unroll 1
-            for (int sc = 0; sc < nsc; sc += 2) {
-                if (sc + 1 < nsc) ld(sc + 1, bufB);
-                step(sc, bufA);
-                if (sc + 2 < nsc) ld(sc + 2, bufA);
-                if (sc + 1 < nsc) step(sc + 1, bufB);
+            for (int sc = 0; sc < nsc; ++sc) {
+                gm_wait_groups<GM_STAGES - 2>();               // this lane's copies of step sc have landed
+                __syncwarp();                                  // ... and every lane's; tile (sc - 1) % S is free
+                issue(sc + GM_STAGES - 1);
+                step(sc);
             }
+            gm_wait_groups<0>();
             // ---- epilogue: accumulators -> the warp's tile as [m][row][column] -> outputs
             __syncwarp();
             float *stf = reinterpret_cast<float *>(tile);
@@ -403,10 +440,10 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                 for (int m = 0; m < NM; ++m) {
                     if constexpr (NDIG == 3) {
                         const int *pp = sti + (m * 16 + row) * NC + tk * 3;
-                        const int *tt = tot + (rbase + tk) * 4;
+                        const int *tt = tot + recidx(tk) * 4;
                         const int P0 = pp[0] - (WB == 4 ? tt[0] : 0), P1 = pp[1] - (WB == 4 ? tt[1] : 0),
                                   P2 = pp[2] - (WB == 4 ? tt[2] : 0);
-                        const float sg = *reinterpret_cast<const float *>(recs + (size_t)(rbase + tk) * p.rec_bytes + RL.hdr);
+                        const float sg = *reinterpret_cast<const float *>(recs + (size_t)recidx(tk) * p.rec_bytes + RL.hdr);
                         x[m] = sg * fmaf(65536.f, (float)P2, fmaf(256.f, (float)P1, (float)P0));
                     } else {
                         x[m] = stf[(m * 16 + row) * NC + tk];
@@ -458,7 +495,8 @@ static inline bool gm_plan(GmPlan &pl, int wbits, int ndig, int K, int rows, int
         const int need = ndig == 3 ? (3 * T + 7) / 8 : (T + 7) / 8;
         if (ntl > 1 && ntl - 1 >= need && !(ndig == 1 && ntl == 4 && need > 2)) continue;
         p.ms = (E < A ? E : A) + 1 + (A + T + ntok - 1) / ntok + 1;
-        p.ntile = al(nm * GM_ROWS * GM_TSTRIDE > nm * GM_ROWS * 8 * ntl * 4 ? nm * GM_ROWS * GM_TSTRIDE : nm * GM_ROWS * 8 * ntl * 4, 16);
+        const int ring = GM_STAGES * nm * GM_ROWS * GM_TSTRIDE, stage = nm * GM_ROWS * 8 * ntl * 4;
+        p.ntile = al(ring > stage ? ring : stage, 16);
         int o = 0;
         p.o_sl = o;
         o = al(o + (4 + 3 * p.ms) * 4, 16);
@@ -471,11 +509,17 @@ static inline bool gm_plan(GmPlan &pl, int wbits, int ndig, int K, int rows, int
         p.o_hmx = o;                                   // warp tiles
         o = al(o + G2_NW * p.ntile, 16);
         const int per = ntok * (p.rec_bytes + 16 + G2_NW * 4);
-        int cap = (G2_SMEM_MAX - 256 - o) / per;
-        if (cap > p.ms) cap = p.ms;
-        if (cap < 1) continue;
-        p.slot_cap = cap;
-        p.nrec = cap * ntok;
+        p.allrec = nm == 2 && T <= ntok;               // gate/up: every token's record, once
+        if (p.allrec) {
+            p.slot_cap = p.ms;
+            p.nrec = T;
+        } else {
+            int cap = (G2_SMEM_MAX - 256 - o) / per;
+            if (cap > p.ms) cap = p.ms;
+            if (cap < 1) continue;
+            p.slot_cap = cap;
+            p.nrec = cap * ntok;
+        }
         p.o_route = o;                                 // plane digit totals
         o = al(o + p.nrec * 16, 16);
         p.o_rmax = o;
