@@ -200,6 +200,17 @@ __device__ __forceinline__ void g2_tr_reduce(float (&v)[V], int lane)
     g2_tr_rec<V, LPR / 2>(v, lane);
 }
 
+// A team of consecutive warps of the CTA that works and synchronises on its
+// own (named barrier `bar`; bar 0 with every thread is __syncthreads).
+struct G2Team {
+    int tid, nthr, warp, nwarp, bar;
+    __device__ void sync() const { asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(nthr) : "memory"); }
+};
+__device__ __forceinline__ G2Team g2_cta()
+{
+    return G2Team{(int)threadIdx.x, G2_THREADS, (int)(threadIdx.x >> 5), G2_NW, 0};
+}
+
 // ---------------------------------------------------------------- record builder
 // EW consecutive values e0 .. e0 + EW - 1 of one input row as the dot sees
 // them (EW = 4, 8 or 16; e0 a multiple of EW): f32 rows (x, or h -- rounded to
@@ -265,11 +276,12 @@ __device__ __forceinline__ void g2_put_words(unsigned char *plane, int cpr, int 
 // lanes.  src(i, row) gives record i's input row (false: record i is unused).
 // rmax: n * G2_NW floats of scratch.  Ends with __syncthreads.
 template <int WB, int NDIG, bool CACHE, typename SrcFn>
-__device__ void g2_build(const G2P &p, unsigned char *recs, int n, SrcFn src, bool gateup, float *rmax)
+__device__ void g2_build(const G2P &p, unsigned char *recs, int n, SrcFn src, bool gateup, float *rmax,
+                         const G2Team tm = g2_cta())
 {
     using F = Fmt<WB>;
     constexpr int EW = F::EPC / 4, UPW = F::UPW, NQ = F::DW / 4;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = tm.tid, lane = threadIdx.x & 31, warp = tm.warp, NTH = tm.nthr;
     const int K = p.K, cpr = p.cpr, nitem = K / EW;
     const G2Rec RL = g2_rec(NDIG, K, cpr);
     const bool bf_in = gateup && p.afmt == QRX_A_BF16, rnd = !gateup && p.afmt == QRX_A_BF16;
@@ -282,14 +294,14 @@ __device__ void g2_build(const G2P &p, unsigned char *recs, int n, SrcFn src, bo
         const bool known = !gateup && p.hmax != nullptr;
         // pass 1: every row's largest magnitude; a thread's first two (row, item)
         // values stay in registers for pass 2 (item it = tid + q * threads in both)
-        const int nq = (nitem + G2_THREADS - 1) / G2_THREADS;
+        const int nq = (nitem + NTH - 1) / NTH;
         float cache[2][EW];
         for (int i = 0; i < n && !known; ++i) {
             int64_t row;
             if (!src(i, row)) continue;
             const void *rp = row_ptr(row);
             float am = 0.f;
-            for (int it = tid, q = 0; it < nitem; it += G2_THREADS, ++q) {
+            for (int it = tid, q = 0; it < nitem; it += NTH, ++q) {
                 float v[EW];
                 g2_vals<EW>(rp, bf_in, rnd, it * EW, v);
                 const int slot = i * nq + q;
@@ -303,7 +315,7 @@ __device__ void g2_build(const G2P &p, unsigned char *recs, int n, SrcFn src, bo
             am = warp_max(am);
             if (lane == 0) rmax[i * G2_NW + warp] = am;
         }
-        if (!known) __syncthreads();
+        if (!known) tm.sync();
         // pass 2: digits and chunk digit sums
         for (int i = 0; i < n; ++i) {
             int64_t row;
@@ -315,13 +327,12 @@ __device__ void g2_build(const G2P &p, unsigned char *recs, int n, SrcFn src, bo
                 am = __uint_as_float(p.hmax[row]);
                 if (rnd) am = __bfloat162float(__float2bfloat16_rn(am));
             } else {
-#pragma unroll
-                for (int w = 0; w < G2_NW; ++w) am = fmaxf(am, rmax[i * G2_NW + w]);
+                for (int w = 0; w < tm.nwarp; ++w) am = fmaxf(am, rmax[i * G2_NW + w]);
             }
             const int sh = am != 0.f ? fixed_shift(am) : 0;
             const bool fast = sh >= -126 && sh <= 127;
             const float mul = fast ? __int_as_float((sh + 127) << 23) : 0.f;
-            for (int base = warp * 32, q = 0; base < nitem; base += G2_THREADS, ++q) {
+            for (int base = warp * 32, q = 0; base < nitem; base += NTH, ++q) {
                 const int it = base + lane;
                 const bool act = it < nitem;
                 const int c = it >> 2, wi = it & 3, slot = i * nq + q;
@@ -380,7 +391,7 @@ __device__ void g2_build(const G2P &p, unsigned char *recs, int n, SrcFn src, bo
             unsigned char *rec = recs + (size_t)i * p.rec_bytes;
             float *dsc = reinterpret_cast<float *>(rec + RL.hdr);
             int *cor = reinterpret_cast<int *>(rec + RL.hdr + (RL.bytes - RL.hdr) / 2);
-            for (int base = warp * 32; base < nitem; base += G2_THREADS) {
+            for (int base = warp * 32; base < nitem; base += NTH) {
                 const int it = base + lane;
                 const bool act = it < nitem;
                 const int c = it >> 2, wi = it & 3, b = it / IPB;
@@ -449,7 +460,7 @@ __device__ void g2_build(const G2P &p, unsigned char *recs, int n, SrcFn src, bo
             }
         }
     }
-    __syncthreads();
+    tm.sync();
 }
 
 // ---------------------------------------------------------------- slot tables
@@ -491,11 +502,12 @@ struct G2RouteSm {
 
 // CTA 0 publishes the route: choice, permutation, usage, the compact slot
 // table; and zeroes the combine counters.  Every thread of the CTA calls it.
-__device__ void g2_publish(const G2P &p, const G2RouteSm &r, G2Slots sl, int A, int nu, int nslots)
+__device__ void g2_publish(const G2P &p, const G2RouteSm &r, G2Slots sl, int A, int nu, int nslots,
+                           const G2Team tm = g2_cta())
 {
-    const int tid = threadIdx.x, E = p.E;
+    const int tid = tm.tid, E = p.E, NTH = tm.nthr;
     {
-        for (int a = tid; a < A; a += G2_THREADS) {
+        for (int a = tid; a < A; a += NTH) {
             p.idx[a] = r.ridx[a];
             p.w[a] = r.rw[a];
             p.inv[a] = r.pos[a];
@@ -503,7 +515,7 @@ __device__ void g2_publish(const G2P &p, const G2RouteSm &r, G2Slots sl, int A, 
             if (r.lead[a] && p.usage)
                 atomicAdd(reinterpret_cast<unsigned long long *>(p.usage + r.ridx[a]), (unsigned long long)r.cnt[a]);
         }
-        for (int e = tid; e <= E; e += G2_THREADS) {
+        for (int e = tid; e <= E; e += NTH) {
             int less = 0, cnt = 0;
             for (int b = 0; b < A; ++b) {
                 const int f = r.ridx[b];
@@ -514,8 +526,8 @@ __device__ void g2_publish(const G2P &p, const G2RouteSm &r, G2Slots sl, int A, 
             p.offsets[e] = less;
             if (e < E) p.counts[e] = cnt;
         }
-        for (int u = tid; u < nu; u += G2_THREADS) p.union_ids[u] = sl.e[u];
-        for (int s = tid; s < nslots; s += G2_THREADS) {
+        for (int u = tid; u < nu; u += NTH) p.union_ids[u] = sl.e[u];
+        for (int s = tid; s < nslots; s += NTH) {
             p.tab_out[G2_TAB_HDR + 4 * s] = sl.e[s];
             p.tab_out[G2_TAB_HDR + 4 * s + 1] = sl.p0[s];
             p.tab_out[G2_TAB_HDR + 4 * s + 2] = sl.nt[s];
@@ -528,7 +540,7 @@ __device__ void g2_publish(const G2P &p, const G2RouteSm &r, G2Slots sl, int A, 
             p.tab_out[2] = 0;
             p.tab_out[3] = 0;
         }
-        for (int i = tid; i < p.ncnt; i += G2_THREADS) p.cnt[i] = 0;
+        for (int i = tid; i < p.ncnt; i += NTH) p.cnt[i] = 0;
     }
 }
 
@@ -692,19 +704,19 @@ __host__ __device__ inline bool g2_route1_ok(int T, int E, int G, int k)
     return T == 1 && G >= 1 && G <= 32 && E % G == 0 && (E / G) % 32 == 0 && k <= 32;
 }
 
-__device__ void g2_route1(const G2P &p, int *rsm, G2Slots sl, int *srt)
+__device__ void g2_route1(const G2P &p, int *rsm, G2Slots sl, int *srt, const G2Team tm = g2_cta())
 {
     const int E = p.E, G = p.G, Gk = p.Gk, k = p.k, gs = E / G;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = tm.tid, lane = threadIdx.x & 31, warp = tm.warp;
     G2RouteSm r(rsm, 1, E, G, Gk, k);
     float *ps = r.csc;                        // s of the pick of each rank
-    for (int e = tid; e < E; e += G2_THREADS) {
+    for (int e = tid; e < E; e += tm.nthr) {
         const float s = (float)(1.0 / (1.0 + exp(-(double)p.logits[e])));
         r.s[e] = s;
         r.sc[e] = __fadd_rn(s, p.bias[e]);
     }
-    __syncthreads();
-    for (int g = warp; g < G; g += G2_NW) {
+    tm.sync();
+    for (int g = warp; g < G; g += tm.nwarp) {
         float t1 = -INFINITY, t2 = -INFINITY;
         for (int e = g * gs + lane; e < (g + 1) * gs; e += 32) {
             const float v = r.sc[e];
@@ -720,19 +732,21 @@ __device__ void g2_route1(const G2P &p, int *rsm, G2Slots sl, int *srt)
         }
         if (lane == 0) r.gsc[g] = __fadd_rn(t1, t2);        // gs >= 32: two members at least
     }
-    __syncthreads();
-    // kept groups as a bit mask (every thread the same)
-    uint32_t kept = 0;
-    for (int g = 0; g < G; ++g) {
-        const float v = r.gsc[g];
+    tm.sync();
+    // kept groups as a bit mask (every thread the same): lane g of every warp ranks group g
+    uint32_t kept;
+    {
         int rank = 0;
-        for (int h = 0; h < G; ++h) {
-            const float u = r.gsc[h];
-            rank += (u > v) || (u == v && h < g);
+        if (lane < G) {
+            const float v = r.gsc[lane];
+            for (int h = 0; h < G; ++h) {
+                const float u = r.gsc[h];
+                rank += (u > v) || (u == v && h < lane);
+            }
         }
-        if (rank < Gk) kept |= 1u << g;
+        kept = __ballot_sync(0xffffffffu, lane < G && rank < Gk);
     }
-    for (int q = tid; q < 2 * E; q += G2_THREADS) {       // (expert, half) pairs on neighbouring lanes
+    for (int q = tid; q < 2 * E; q += tm.nthr) {       // (expert, half) pairs on neighbouring lanes
         const int e = q >> 1, half = q & 1;
         const bool mine = kept >> (e / gs) & 1u;
         int cnt = 0;
@@ -754,7 +768,7 @@ __device__ void g2_route1(const G2P &p, int *rsm, G2Slots sl, int *srt)
             ps[cnt] = r.s[e];
         }
     }
-    __syncthreads();
+    tm.sync();
     if (warp == 0) {
         const int my_e = lane < k ? r.pick[lane] : 0;
         const float my_s = lane < k ? ps[lane] : 0.f;
@@ -796,8 +810,8 @@ __device__ void g2_route1(const G2P &p, int *rsm, G2Slots sl, int *srt)
             }
         }
     }
-    __syncthreads();
-    if (blockIdx.x == 0) g2_publish(p, r, sl, k, sl.hdr[1], sl.hdr[0]);
+    tm.sync();
+    if (blockIdx.x == 0) g2_publish(p, r, sl, k, sl.hdr[1], sl.hdr[0], tm);
 }
 
 // Slot table from a permutation in memory (gate/up without fusing; down
@@ -959,18 +973,37 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gemv2(const __grid_constant__
     unsigned char *recs = sm + p.o_rec;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+    bool routed_now = false;
     if constexpr (GATEUP) {
-        // the records of every token, before the dependency wait: x is an input
-        // of the call, so this overlaps the kernels before
-        g2_build<WB, NDIG, true>(p, recs, p.T, [](int i, int64_t &row) { row = i; return true; }, true, rmax);
+        if (p.fuse && g2_route1_ok(p.T, p.E, p.G, p.k) && p.E <= G2_THREADS / 2) {
+            // one token: half the CTA makes the choice from the logits while the
+            // other half builds the token's record (x is an input of the call)
+            if (warp < G2_NW / 2) {
+                pdl_wait();            // the logits
+                g2_route1(p, reinterpret_cast<int *>(sm + p.o_route), sl, srt,
+                          G2Team{tid, G2_THREADS / 2, warp, G2_NW / 2, 1});
+            } else {
+                g2_build<WB, NDIG, true>(p, recs, p.T, [](int i, int64_t &row) { row = i; return true; }, true, rmax,
+                                         G2Team{tid - G2_THREADS / 2, G2_THREADS / 2, warp - G2_NW / 2, G2_NW / 2, 2});
+            }
+            __syncthreads();
+            pdl_trigger();
+            routed_now = true;
+        } else {
+            // the records of every token, before the dependency wait: x is an input
+            // of the call, so this overlaps the kernels before
+            g2_build<WB, NDIG, true>(p, recs, p.T, [](int i, int64_t &row) { row = i; return true; }, true, rmax);
+        }
     }
-    pdl_wait();            // gate/up: the logits or the permutation; down: h, from the kernels before
-    pdl_trigger();
-    if (GATEUP && p.fuse) {
-        if (g2_route1_ok(p.T, p.E, p.G, p.k)) g2_route1(p, reinterpret_cast<int *>(sm + p.o_route), sl, srt);
-        else g2_route(p, reinterpret_cast<int *>(sm + p.o_route), sl, srt);
-    } else {
-        g2_slots_from_perm(p, sl, srt, GATEUP);
+    if (!routed_now) {
+        pdl_wait();            // gate/up: the logits or the permutation; down: h, from the kernels before
+        pdl_trigger();
+        if (GATEUP && p.fuse) {
+            if (g2_route1_ok(p.T, p.E, p.G, p.k)) g2_route1(p, reinterpret_cast<int *>(sm + p.o_route), sl, srt);
+            else g2_route(p, reinterpret_cast<int *>(sm + p.o_route), sl, srt);
+        } else {
+            g2_slots_from_perm(p, sl, srt, GATEUP);
+        }
     }
     const int nslots = sl.hdr[0], nu = sl.hdr[1];
     uint32_t *hmx = reinterpret_cast<uint32_t *>(sm + p.o_hmx);
