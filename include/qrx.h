@@ -333,20 +333,28 @@ int qrx_expert_ffn_noalloc(const qrx_cfg *cfg, const qrx_experts *routed,
 
 /* ---- the whole layer --------------------------------------------------- */
 
-/* activation records -> route -> permute -> routed + shared FFN -> combine,
+/* route -> permute -> routed + shared FFN -> combine (README "JustVugg/colibri",
+ * section "已实现的功能": the router, the batch-union MoE, the shared expert),
  * all on `stream` with no host synchronisation.  (Capture into a CUDA graph
  * is not tested; the first call on a device also raises kernels' shared-memory
  * limits, so make one call before capturing.)
  * The kernels after the first are chained with programmatic dependent launch:
  * each may start while its predecessor drains and waits for it only where it
- * reads its output (the down kernel starts streaming its weights first).
+ * reads its output.
  * shared may be NULL.  x: the activations in cfg->afmt (f32 or bf16 [T][H];
  * Q8_0 is quantised from f32 x inside the call), 16-byte aligned.
  * topk_idx, topk_w: outputs [T][k].  out [T][H] f32, 16-byte aligned.
- * Expert FFN engine: bf16 activations, int4 experts, T >= 256 and H, I
- * multiples of 256 run gate/up and down as grouped GEMMs on the tcgen05 tensor
- * cores (bf16 x bf16 -> f32; int4 codes are exact in bf16); every other case
- * runs the HBM-streaming integer GEMV. */
+ * Expert FFN engines, by the call's shape:
+ *   T = 1: the decode GEMV; its gate/up launch also makes the selection and
+ *          the permutation from the router logits, its down launch also the
+ *          combine (three launches in all);
+ *   2 <= T <= 64 with int4 / int8 experts: the multi-token GEMV, the dot
+ *          products on tensor cores (mma.sync, 8-bit codes x 8-bit digits ->
+ *          exact int32);
+ *   bf16 activations, int4 experts, T >= 256, H and I multiples of 256:
+ *          grouped GEMMs on the tcgen05 tensor cores (bf16 x bf16 -> f32;
+ *          int4 codes are exact in bf16);
+ *   otherwise: the HBM-streaming dp4a GEMV. */
 int qrx_moe_forward(const qrx_cfg *cfg, const void *x, int32_t T, const float *W_router,
                     const float *bias, const qrx_experts *routed, const qrx_experts *shared,
                     int32_t *topk_idx, float *topk_w, float *out, void *ws,
