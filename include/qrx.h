@@ -136,7 +136,10 @@ typedef struct {
 
 /* ---- queries (host only, synchronous) ---------------------------------- */
 
-/* Check a configuration.  QRX_EINVAL for non-positive sizes or a bad enum;
+/* Check a configuration (README "JustVugg/colibri", section "已实现的功能": a
+ * DeepSeek-V3-like router over n_group groups keeping topk_group, top_k
+ * experts, routed_scaling_factor; int8 / packed int4 / packed int2 experts;
+ * f32 or Q8_0-style int8 activations).  QRX_EINVAL for non-positive sizes or a bad enum;
  * QRX_EUNSUPPORTED when: E % G != 0, Gk > G, Gk*E/G < k, k > 32, E > 1024,
  * H or I not a multiple of 64, or a row of H or I codes is not a supported
  * number of 16-byte chunks (1, 2, 4, 8, 16, 32, 64, 96, 128, 192 or 384). */
@@ -147,8 +150,12 @@ size_t qrx_workspace_bytes(const qrx_cfg *cfg, int32_t T);
 
 /* Which engine runs the expert FFN (gate/up + SwiGLU and down) of a call with
  * this configuration and T tokens (the routed, shared and whole-layer entry
- * points that take a workspace):
- *   QRX_ENGINE_GEMV  the HBM-streaming integer-digit GEMV (any format);
+ * points that take a workspace; README "JustVugg/colibri", section "已实现的功能":
+ * the kernel for a shape is chosen by measurement):
+ *   QRX_ENGINE_GEMV  the HBM-streaming integer GEMVs (any format): the
+ *                    one-token decode GEMV, the multi-token GEMV with its dot
+ *                    products on mma.sync tensor cores (2..64 tokens, int4 /
+ *                    int8), or the dp4a engine;
  *   QRX_ENGINE_TC    grouped GEMMs on the tcgen05 tensor cores: bf16
  *                    activations, int4 weights, T >= 256, H and I multiples
  *                    of 256, and a CUDA driver that provides tensor-map
@@ -248,8 +255,11 @@ int qrx_topp_prune(const qrx_cfg *cfg, int32_t *topk_idx, float *topk_w, int32_t
  * before the first call; calls on one stream accumulate in order. */
 int qrx_usage_accumulate(const qrx_cfg *cfg, const qrx_perm *perm, uint64_t *usage, void *stream);
 
-/* Routed experts' SwiGLU FFN over the batch union: for each expert of the
- * union, its gate/up rows are read once for all of its positions:
+/* Routed experts' SwiGLU FFN over the batch union (README "JustVugg/colibri",
+ * section "已实现的功能": batch-union MoE, int8 / packed int4 / packed int2
+ * dequantised on use; blog "GLM-5.2 on slow computers", section
+ * "让它变得可以忍受的那些装置": an expert shared by a batch is read once): for
+ * each expert of the union, its gate/up rows are read once for all of its positions:
  * h = silu(s_g (Q_g x)) * (s_u (Q_u x)), then y = s_d (Q_d h') where h' is h
  * (F32), h rounded to bf16 (BF16) or h re-quantised to Q8_0 (Q8_0).
  *   h_sorted: [T*k][I] f32 output (may be NULL: workspace is used)
@@ -258,8 +268,9 @@ int qrx_expert_ffn(const qrx_cfg *cfg, const qrx_experts *routed, const qrx_perm
                    const qrx_act *act, int32_t T, float *h_sorted, float *y_sorted,
                    void *ws, size_t ws_bytes, void *stream);
 
-/* Down projection alone, from a given h_sorted [T*k][I] f32 (stage
- * isolation: lets a test feed the reference's h). */
+/* Down projection alone (the second half of the expert FFN above, README
+ * "JustVugg/colibri", section "已实现的功能"), from a given h_sorted [T*k][I]
+ * f32 (stage isolation: lets a test feed the reference's h). */
 int qrx_expert_down(const qrx_cfg *cfg, const qrx_experts *routed, const qrx_perm *perm,
                     const float *h_sorted, int32_t T, float *y_sorted, void *ws,
                     size_t ws_bytes, void *stream);
@@ -291,7 +302,9 @@ int qrx_shared_ffn(const qrx_cfg *cfg, const qrx_experts *shared, const qrx_act 
                    int32_t T, float *h_sh, float *y_sh, void *ws, size_t ws_bytes,
                    void *stream);
 
-/* Weighted combine: out[t] = y_sh[t] + sum_j topk_w[t][j] * y_sorted[inv[t*k+j]]
+/* Weighted combine (README "JustVugg/colibri", section "已实现的功能": routed
+ * experts weighted by the router, plus the shared expert):
+ * out[t] = y_sh[t] + sum_j topk_w[t][j] * y_sorted[inv[t*k+j]]
  * in fixed j order.  y_sh may be NULL (no shared term).  A slot with
  * inv < 0 (dropped by adaptive top-p) contributes nothing, whatever its
  * weight.  out [T][H] f32. */
