@@ -636,3 +636,79 @@ def test_hostio_matches_device_call(glm):
     ws = qrx.workspace(c, 1)
     qrx.qrx_moe_forward_hostio(c, xh, glay.Wr, glay.bias, glay.routed[4], glay.shared[4], oh, ws)
     assert np.array_equal(oh.numpy(), out)
+
+
+# ------------------------------------------------------------------ maximum sizes
+# The largest routing the library accepts (E = 1024 experts, top-32, 32 groups of
+# 32 with 8 kept) on a small expert (H = I = 256, which the tensor-core engine also
+# takes), through qrx_moe_forward in every activation mode and every engine: the
+# one-token fused decode path (T = 1), the multi-token mma GEMV (T = 4, 33) and the
+# tensor-core engine (bf16, T = 300).
+MAX_WL = W.TINY.with_(name="max_e1024_k32", n_experts=1024, n_group=32, topk_group=8,
+                      top_k=32, inter=256)
+
+
+@pytest.fixture(scope="session")
+def max_layer(dev):
+    return GpuLayer(MAX_WL, formats=(4, 8, 2)), OracleLayer(MAX_WL)
+
+
+@pytest.mark.parametrize("T", [1, 4, 33])
+@pytest.mark.parametrize("afmt", [W.A_F32, W.A_Q8, W.A_BF16], ids=["f32", "q8", "bf16"])
+def test_max_sizes_layer(max_layer, afmt, T):
+    glay, olay = max_layer
+    wl = MAX_WL.with_(afmt=afmt, T=T)
+    res = check_layer(glay, olay, wl, activations(wl, batch=T), range(T))
+    assert res["idx"].shape == (T, 32) and (res["idx"] >= 0).all()
+    assert all(len(set(row.tolist())) == 32 for row in res["idx"])
+
+
+@pytest.mark.parametrize("bits", [8, 2])
+@pytest.mark.parametrize("T", [1, 33])
+def test_max_sizes_formats(max_layer, bits, T):
+    glay, olay = max_layer
+    wl = MAX_WL.with_(T=T)
+    check_layer(glay, olay, wl, activations(wl, batch=T), range(T), bits=bits)
+
+
+def test_max_sizes_tensor_core(max_layer):
+    glay, olay = max_layer
+    wl = MAX_WL.with_(afmt=W.A_BF16, T=300)
+    assert qrx.qrx_ffn_engine(qrx.cfg_of(wl), 300) == qrx.QRX_ENGINE_TC
+    check_layer(glay, olay, wl, activations(wl), list(range(0, 300, 13)) + [299])
+
+
+def test_max_sizes_topp(max_layer):
+    glay, olay = max_layer
+    wl = MAX_WL.with_(afmt=W.A_Q8, T=33)
+    check_layer(glay, olay, wl, activations(wl, batch=5), range(33), topp=0.6)
+
+
+# ------------------------------------------------------------------ repeat runs
+def _same_bits(a, b):
+    return all(np.array_equal(np.asarray(u).view(np.uint32), np.asarray(v).view(np.uint32))
+               for u, v in zip(a, b))
+
+
+@pytest.mark.parametrize("wl", [W.GLM_DECODE_T1, W.GLM_DECODE_T1.with_(afmt=W.A_Q8),
+                                W.GLM_VERIFY_T4_BF16, W.GLM_DECODE_T32_Q8,
+                                W.GLM_PREFILL_T2048_BF16], ids=lambda w: f"{w.name}_a{w.afmt}")
+def test_glm_repeat_runs_bit_identical(glm, wl):
+    """Three runs of the same call give the same indices, weights and output bits
+    on every engine (fused decode, mma GEMV, tensor core): no atomics decide an
+    order of floating-point additions."""
+    glay, _ = glm
+    x = activations(wl)
+    bias = cu(router_weights(wl)[1])
+    first = gpu_layer(glay, wl, x, bias=bias)
+    for _ in range(2):
+        assert _same_bits(first, gpu_layer(glay, wl, x, bias=bias))
+
+
+@pytest.mark.parametrize("T,afmt", [(1, W.A_F32), (33, W.A_Q8), (300, W.A_BF16)])
+def test_max_sizes_repeat_runs_bit_identical(max_layer, T, afmt):
+    glay, _ = max_layer
+    wl = MAX_WL.with_(afmt=afmt, T=T)
+    x = activations(wl)
+    first = gpu_layer(glay, wl, x)
+    assert _same_bits(first, gpu_layer(glay, wl, x))
