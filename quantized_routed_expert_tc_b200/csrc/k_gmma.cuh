@@ -35,6 +35,12 @@
 // block's offset correction and scaled by the token's d_b in f32).  int4
 // codes enter as offset binary (code + 8); the offset is removed through the
 // digit sums (per block for Q8_0, per row and plane for the fixed point).
+// The down projection with the fixed point skips the tile: each lane's own
+// 16 bytes of rows g and g + 8 (block 4 s + t of step s for int4, half a block
+// for int8) are its A fragments -- word j's low and high nibbles (int4), or
+// words 2 j and 2 j + 1 (int8), fill k = 4 t .. 4 t + 3 and 16 + 4 t .. of mma
+// j -- and the B fragments are the matching digit words of record chunk
+// 4 s + t; the sums are exact over all of K, so the k order is free.
 #pragma once
 #include "k_gemv2.cuh"
 
@@ -173,6 +179,12 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
     constexpr int NTOK = NDIG == 3 ? NC / 3 : NC;        // tokens per pass
     constexpr int NQ = F::DW / 4;
     constexpr int NBLK = WB == 4 ? 4 : 2;                // 32-code blocks per 64-byte step
+    // down projection with the fixed point (three planes, exact sums over all of
+    // K): the A fragments come straight from the lane's loads, in a k order the
+    // records match.  Q8_0 needs one block per mma, which the tile and ldmatrix
+    // arrange; gate/up keeps the tile ring too, which measured faster there
+    // (two matrices: twice the loads per step in flight behind the copies)
+    constexpr bool RD = NDIG == 3 && !GATEUP;
     static_assert(WB == 4 || WB == 8, "int4 or int8 weights");
     extern __shared__ __align__(128) unsigned char sm[];
     G2Slots sl(reinterpret_cast<int *>(sm + p.o_sl), p.ms);
@@ -404,18 +416,88 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                     }
                 }
             };
-            // the ring: GM_STAGES - 1 steps in flight ahead of the one computed
-            __syncwarp();                                      // the last unit's tile reads are done
+            if constexpr (RD) {
+                // fixed point: the lane's own 16 bytes of rows g and g + 8 are its A
+                // fragments (block 4 sc + t for int4, half block for int8); the
+                // records give the matching digits, one step of loads ahead
+                uint4 nx[NM][2];
+                auto load = [&](int sc) {
+                    if (sc < nsc)
 #pragma unroll
-            for (int q = 0; q < GM_STAGES - 1; ++q) issue(q);
+                        for (int m = 0; m < NM; ++m) {
+                            nx[m][0] = ld_stream16(wa[m] + (size_t)sc * GM_SCB);
+                            nx[m][1] = ld_stream16(wb[m] + (size_t)sc * GM_SCB);
+                        }
+                };
+                load(0);
 #pragma unroll 1
-            for (int sc = 0; sc < nsc; ++sc) {
-                gm_wait_groups<GM_STAGES - 2>();               // this lane's copies of step sc have landed
-                __syncwarp();                                  // ... and every lane's; tile (sc - 1) % S is free
-                issue(sc + GM_STAGES - 1);
-                step(sc);
+                for (int sc = 0; sc < nsc; ++sc) {
+                    uint32_t cw[NM][2][4];
+#pragma unroll
+                    for (int m = 0; m < NM; ++m)
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            cw[m][hf][0] = nx[m][hf].x;
+                            cw[m][hf][1] = nx[m][hf].y;
+                            cw[m][hf][2] = nx[m][hf].z;
+                            cw[m][hf][3] = nx[m][hf].w;
+                        }
+                    load(sc + 1);
+                    const int c = 4 * sc + t;                  // the record chunk of this lane's 16 bytes
+                    // mma j: k = 4 t .. 4 t + 3 <- word j's low nibbles (int4) or word 2 j
+                    // (int8); k = 16 + 4 t .. <- its high nibbles or word 2 j + 1
+                    uint32_t bf[NBLK][NTL][2];
+#pragma unroll
+                    for (int j = 0; j < NBLK; ++j)
+#pragma unroll
+                        for (int jj = 0; jj < NTL; ++jj) {
+                            bf[j][jj][0] = bf[j][jj][1] = 0;
+                            if (boff[jj] >= 0) {
+                                const int off = WB == 4 ? ((j >> 1) * p.cpr + c) * 16 + (j & 1) * 8 : c * 16 + 8 * j;
+                                const uint2 bb = *reinterpret_cast<const uint2 *>(sm + boff[jj] + off);
+                                bf[j][jj][0] = bb.x;
+                                bf[j][jj][1] = bb.y;
+                            }
+                        }
+#pragma unroll
+                    for (int j = 0; j < NBLK; ++j) {
+                        uint32_t a[NM][4];
+#pragma unroll
+                        for (int m = 0; m < NM; ++m) {
+                            if constexpr (WB == 4) {
+                                const uint32_t wg = cw[m][0][j] ^ 0x88888888u, wh = cw[m][1][j] ^ 0x88888888u;
+                                a[m][0] = wg & 0x0F0F0F0Fu;
+                                a[m][1] = wh & 0x0F0F0F0Fu;
+                                a[m][2] = (wg >> 4) & 0x0F0F0F0Fu;
+                                a[m][3] = (wh >> 4) & 0x0F0F0F0Fu;
+                            } else {
+                                a[m][0] = cw[m][0][2 * j];
+                                a[m][1] = cw[m][1][2 * j];
+                                a[m][2] = cw[m][0][2 * j + 1];
+                                a[m][3] = cw[m][1][2 * j + 1];
+                            }
+                        }
+#pragma unroll
+                        for (int jj = 0; jj < NTL; ++jj)
+#pragma unroll
+                            for (int m = 0; m < NM; ++m)
+                                gm_mma(acc[m][jj], a[m][0], a[m][1], a[m][2], a[m][3], bf[j][jj][0], bf[j][jj][1], WB == 4);
+                    }
+                }
+            } else {
+                // the ring: GM_STAGES - 1 steps in flight ahead of the one computed
+                __syncwarp();                                  // the last unit's tile reads are done
+#pragma unroll
+                for (int q = 0; q < GM_STAGES - 1; ++q) issue(q);
+#pragma unroll 1
+                for (int sc = 0; sc < nsc; ++sc) {
+                    gm_wait_groups<GM_STAGES - 2>();           // this lane's copies of step sc have landed
+                    __syncwarp();                              // ... and every lane's; tile (sc - 1) % S is free
+                    issue(sc + GM_STAGES - 1);
+                    step(sc);
+                }
+                gm_wait_groups<0>();
             }
-            gm_wait_groups<0>();
             // ---- epilogue: accumulators -> the warp's tile as [m][row][column] -> outputs
             __syncwarp();
             float *stf = reinterpret_cast<float *>(tile);
