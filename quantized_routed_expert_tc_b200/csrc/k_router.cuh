@@ -253,15 +253,30 @@ __global__ void __launch_bounds__(256) k_router_split(RouterArgs a, int nslice, 
     __syncthreads();
     if (last) {
         __threadfence();
+        // slice by slice for all 16 of the thread's outputs at once (16
+        // independent loads per slice in flight), each output still summed in
+        // slice order
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+#pragma unroll 2
+        for (int q = 0; q < nslice; ++q) {
+            const double *pq = part + q * TE;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int t = t0 + ty + 16 * i, e = e0 + tx + 16 * j;
+                    if (t < a.T && e < a.E) acc[i][j] += __ldcg(pq + (int64_t)t * a.E + e);
+                }
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int t = t0 + ty + 16 * i, e = e0 + tx + 16 * j;
-                if (t >= a.T || e >= a.E) continue;
-                double sum = 0.0;
-                for (int q = 0; q < nslice; ++q) sum += __ldcg(part + q * TE + (int64_t)t * a.E + e);
-                a.logits[(int64_t)t * a.E + e] = (float)sum;
+                if (t < a.T && e < a.E) a.logits[(int64_t)t * a.E + e] = (float)acc[i][j];
             }
     }
     pdl_wait();
