@@ -99,9 +99,10 @@ def uses_decode_gemv(wl) -> bool:
 
 
 def uses_mma_gemv(wl) -> bool:
-    """Calls of 2..64 tokens over int4 / int8 weights: the multi-token GEMV on
-    tensor cores (k_gmma)."""
-    return not uses_tensor_cores(wl) and 2 <= wl.T <= 64 and wl.wbits in (4, 8)
+    """Calls of 2..64 tokens over int4 / int8 weights, or int2 weights with f32 /
+    bf16 activations: the multi-token GEMV on tensor cores (k_gmma)."""
+    return not uses_tensor_cores(wl) and 2 <= wl.T <= 64 and (wl.wbits in (4, 8) or
+                                                               (wl.wbits == 2 and wl.afmt != 1))
 
 
 def gemv_kernel(wl) -> str:

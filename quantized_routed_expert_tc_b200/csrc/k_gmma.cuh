@@ -178,14 +178,14 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
     constexpr int NC = 8 * NTL;                          // columns per pass
     constexpr int NTOK = NDIG == 3 ? NC / 3 : NC;        // tokens per pass
     constexpr int NQ = F::DW / 4;
-    constexpr int NBLK = WB == 4 ? 4 : 2;                // 32-code blocks per 64-byte step
+    constexpr int NBLK = WB == 4 ? 4 : (WB == 2 ? 8 : 2);  // mmas per matrix and 64-byte step
     // down projection with the fixed point (three planes, exact sums over all of
     // K): the A fragments come straight from the lane's loads, in a k order the
     // records match.  Q8_0 needs one block per mma, which the tile and ldmatrix
     // arrange; gate/up keeps the tile ring too, which measured faster there
     // (two matrices: twice the loads per step in flight behind the copies)
     constexpr bool RD = NDIG == 3 && !GATEUP;
-    static_assert(WB == 4 || WB == 8, "int4 or int8 weights");
+    static_assert(WB == 4 || WB == 8 || (WB == 2 && NDIG == 3), "int4 or int8 weights, or int2 with the fixed point");
     extern __shared__ __align__(128) unsigned char sm[];
     G2Slots sl(reinterpret_cast<int *>(sm + p.o_sl), p.ms);
     int *srt = reinterpret_cast<int *>(sm + p.o_srt);
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
 
     // OFF times each record's digit total per plane (fixed point, int4), records [i0, i1)
     auto totals = [&](int i0, int i1) {
-        if constexpr (NDIG == 3 && WB == 4) {
+        if constexpr (NDIG == 3 && WB != 8) {
             for (int q = warp; q < (i1 - i0) * 3; q += G2_NW) {
                 const int i = i0 + q / 3, pl = q % 3;
                 const unsigned char *rec = recs + (size_t)i * p.rec_bytes;
@@ -352,13 +352,19 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                 uint32_t bf[NBLK][NTL][2];
 #pragma unroll
                 for (int kb = 0; kb < NBLK; ++kb) {
-                    const int c = WB == 4 ? NBLK * sc + kb : 4 * sc + 2 * kb;   // record chunk of k = 0 .. 15
+                    // record chunk of the mma's k = 0 .. 15
+                    const int c = WB == 4 ? NBLK * sc + kb : (WB == 2 ? 4 * sc + (kb >> 1) : 4 * sc + 2 * kb);
 #pragma unroll
                     for (int jj = 0; jj < NTL; ++jj) {
                         bf[kb][jj][0] = bf[kb][jj][1] = 0;
                         if (boff[jj] >= 0) {
                             if constexpr (WB == 4) {
                                 const uint2 bb = *reinterpret_cast<const uint2 *>(sm + boff[jj] + ((t >> 1) * p.cpr + c) * 16 + (t & 1) * 8);
+                                bf[kb][jj][0] = bb.x;
+                                bf[kb][jj][1] = bb.y;
+                            } else if constexpr (WB == 2) {
+                                // digit words 4 t + 2 (kb & 1) and the next: piece t, 8 bytes in
+                                const uint2 bb = *reinterpret_cast<const uint2 *>(sm + boff[jj] + (t * p.cpr + c) * 16 + (kb & 1) * 8);
                                 bf[kb][jj][0] = bb.x;
                                 bf[kb][jj][1] = bb.y;
                             } else {
@@ -373,7 +379,16 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                     uint32_t a[NM][4];
 #pragma unroll
                     for (int m = 0; m < NM; ++m) {
-                        if constexpr (WB == 4) {
+                        if constexpr (WB == 2) {
+                            // word t of piece kb / 2, fields flipped to offset binary (code + 2):
+                            // byte b of field pair (kb & 1) is codes 16 t + 4 b + 2 (kb & 1) and + 1
+                            const int sh = 4 * (kb & 1);
+                            const uint32_t wg = aw[m][kb >> 1][0] ^ 0xAAAAAAAAu, wh = aw[m][kb >> 1][1] ^ 0xAAAAAAAAu;
+                            a[m][0] = (wg >> sh) & 0x03030303u;
+                            a[m][1] = (wh >> sh) & 0x03030303u;
+                            a[m][2] = (wg >> (sh + 2)) & 0x03030303u;
+                            a[m][3] = (wh >> (sh + 2)) & 0x03030303u;
+                        } else if constexpr (WB == 4) {
                             // two's-complement nibbles flipped to offset binary (code + 8)
                             const uint32_t wg = aw[m][kb][0] ^ 0x88888888u, wh = aw[m][kb][1] ^ 0x88888888u;
                             a[m][0] = wg & 0x0F0F0F0Fu;                    // codes 8t + 0, 2, 4, 6 of row g
@@ -394,7 +409,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                         if constexpr (NDIG == 3) {
 #pragma unroll
                             for (int m = 0; m < NM; ++m)
-                                gm_mma(acc[m][jj], a[m][0], a[m][1], a[m][2], a[m][3], bf[kb][jj][0], bf[kb][jj][1], WB == 4);
+                                gm_mma(acc[m][jj], a[m][0], a[m][1], a[m][2], a[m][3], bf[kb][jj][0], bf[kb][jj][1], WB != 8);
                         } else {
                             // started from the block's offset correction, scaled by the token's d_b
                             int cr[2] = {0, 0};
@@ -408,7 +423,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
 #pragma unroll
                             for (int m = 0; m < NM; ++m) {
                                 int d4[4] = {cr[0], cr[1], cr[0], cr[1]};
-                                gm_mma(d4, a[m][0], a[m][1], a[m][2], a[m][3], bf[kb][jj][0], bf[kb][jj][1], WB == 4);
+                                gm_mma(d4, a[m][0], a[m][1], a[m][2], a[m][3], bf[kb][jj][0], bf[kb][jj][1], WB != 8);
 #pragma unroll
                                 for (int q = 0; q < 4; ++q) facc[m][jj][q] = fmaf(dq[q & 1], (float)d4[q], facc[m][jj][q]);
                             }
@@ -453,7 +468,8 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                         for (int jj = 0; jj < NTL; ++jj) {
                             bf[j][jj][0] = bf[j][jj][1] = 0;
                             if (boff[jj] >= 0) {
-                                const int off = WB == 4 ? ((j >> 1) * p.cpr + c) * 16 + (j & 1) * 8 : c * 16 + 8 * j;
+                                // int4: digit words 2 j, 2 j + 1; int2: 4 (j / 2) + 2 (j & 1) and the next
+                                const int off = WB != 8 ? ((j >> 1) * p.cpr + c) * 16 + (j & 1) * 8 : c * 16 + 8 * j;
                                 const uint2 bb = *reinterpret_cast<const uint2 *>(sm + boff[jj] + off);
                                 bf[j][jj][0] = bb.x;
                                 bf[j][jj][1] = bb.y;
@@ -464,7 +480,14 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                         uint32_t a[NM][4];
 #pragma unroll
                         for (int m = 0; m < NM; ++m) {
-                            if constexpr (WB == 4) {
+                            if constexpr (WB == 2) {
+                                const int sh = 4 * (j & 1);
+                                const uint32_t wg = cw[m][0][j >> 1] ^ 0xAAAAAAAAu, wh = cw[m][1][j >> 1] ^ 0xAAAAAAAAu;
+                                a[m][0] = (wg >> sh) & 0x03030303u;
+                                a[m][1] = (wh >> sh) & 0x03030303u;
+                                a[m][2] = (wg >> (sh + 2)) & 0x03030303u;
+                                a[m][3] = (wh >> (sh + 2)) & 0x03030303u;
+                            } else if constexpr (WB == 4) {
                                 const uint32_t wg = cw[m][0][j] ^ 0x88888888u, wh = cw[m][1][j] ^ 0x88888888u;
                                 a[m][0] = wg & 0x0F0F0F0Fu;
                                 a[m][1] = wh & 0x0F0F0F0Fu;
@@ -481,7 +504,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                         for (int jj = 0; jj < NTL; ++jj)
 #pragma unroll
                             for (int m = 0; m < NM; ++m)
-                                gm_mma(acc[m][jj], a[m][0], a[m][1], a[m][2], a[m][3], bf[j][jj][0], bf[j][jj][1], WB == 4);
+                                gm_mma(acc[m][jj], a[m][0], a[m][1], a[m][2], a[m][3], bf[j][jj][0], bf[j][jj][1], WB != 8);
                     }
                 }
             } else {
@@ -523,8 +546,8 @@ __global__ void __launch_bounds__(G2_THREADS, 1) k_gmma(const __grid_constant__ 
                     if constexpr (NDIG == 3) {
                         const int *pp = sti + (m * 16 + row) * NC + tk * 3;
                         const int *tt = tot + recidx(tk) * 4;
-                        const int P0 = pp[0] - (WB == 4 ? tt[0] : 0), P1 = pp[1] - (WB == 4 ? tt[1] : 0),
-                                  P2 = pp[2] - (WB == 4 ? tt[2] : 0);
+                        const int P0 = pp[0] - (WB != 8 ? tt[0] : 0), P1 = pp[1] - (WB != 8 ? tt[1] : 0),
+                                  P2 = pp[2] - (WB != 8 ? tt[2] : 0);
                         const float sg = *reinterpret_cast<const float *>(recs + (size_t)recidx(tk) * p.rec_bytes + RL.hdr);
                         x[m] = sg * fmaf(65536.f, (float)P2, fmaf(256.f, (float)P1, (float)P0));
                     } else {
@@ -559,7 +582,9 @@ static inline bool gm_plan(GmPlan &pl, int wbits, int ndig, int K, int rows, int
 {
     G2P &p = pl.p;
     p = G2P{};
-    if ((wbits != 4 && wbits != 8) || T < 1 || T > 64 || rows < 1 || E < 1 || k < 1 || k > 32) return false;
+    if ((wbits != 4 && wbits != 8 && !(wbits == 2 && ndig == 3)) || T < 1 || T > 64 || rows < 1 || E < 1 || k < 1 ||
+        k > 32)
+        return false;
     p.K = K;
     p.rows = rows;
     p.row_bytes = K * wbits / 8;
@@ -639,6 +664,7 @@ static cudaError_t gm_dispatch(const GmPlan &pl, int wbits, int ndig, int grid, 
     if (wbits == WB && ndig == ND && pl.ntl == NTL) return gm_go<WB, ND, NTL, GU>(pl.p, grid, st);
     QRX_GM(4, 3, 1) QRX_GM(4, 3, 2) QRX_GM(4, 3, 3) QRX_GM(4, 1, 1) QRX_GM(4, 1, 2) QRX_GM(4, 1, 4)
     QRX_GM(8, 3, 1) QRX_GM(8, 3, 2) QRX_GM(8, 3, 3) QRX_GM(8, 1, 1) QRX_GM(8, 1, 2) QRX_GM(8, 1, 4)
+    QRX_GM(2, 3, 1) QRX_GM(2, 3, 2) QRX_GM(2, 3, 3)
 #undef QRX_GM
     return cudaErrorInvalidValue;
 }
