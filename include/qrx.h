@@ -155,7 +155,8 @@ size_t qrx_workspace_bytes(const qrx_cfg *cfg, int32_t T);
  *   QRX_ENGINE_GEMV  the HBM-streaming integer GEMVs (any format): the
  *                    one-token decode GEMV, the multi-token GEMV with its dot
  *                    products on mma.sync tensor cores (2..64 tokens, int4 /
- *                    int8), or the dp4a engine;
+ *                    int8, or int2 with f32 / bf16 activations), or the dp4a
+ *                    engine;
  *   QRX_ENGINE_TC    grouped GEMMs on the tcgen05 tensor cores: bf16
  *                    activations, int4 weights, T >= 256, H and I multiples
  *                    of 256, and a CUDA driver that provides tensor-map
@@ -361,9 +362,9 @@ int qrx_expert_ffn_noalloc(const qrx_cfg *cfg, const qrx_experts *routed,
  *   T = 1: the decode GEMV; its gate/up launch also makes the selection and
  *          the permutation from the router logits, its down launch also the
  *          combine (three launches in all);
- *   2 <= T <= 64 with int4 / int8 experts: the multi-token GEMV, the dot
- *          products on tensor cores (mma.sync, 8-bit codes x 8-bit digits ->
- *          exact int32);
+ *   2 <= T <= 64 with int4 / int8 experts (int2: with f32 / bf16
+ *          activations): the multi-token GEMV, the dot products on tensor
+ *          cores (mma.sync, 8-bit codes x 8-bit digits -> exact int32);
  *   bf16 activations, int4 experts, T >= 256, H and I multiples of 256:
  *          grouped GEMMs on the tcgen05 tensor cores (bf16 x bf16 -> f32;
  *          int4 codes are exact in bf16);
