@@ -671,6 +671,15 @@ def test_max_sizes_formats(max_layer, bits, T):
     check_layer(glay, olay, wl, activations(wl, batch=T), range(T), bits=bits)
 
 
+@pytest.mark.parametrize("T", [4, 33])
+@pytest.mark.parametrize("afmt", [W.A_F32, W.A_BF16], ids=["f32", "bf16"])
+def test_max_sizes_int2_multi_token(max_layer, afmt, T):
+    """int2 weights with fixed-point activations on the multi-token mma GEMV."""
+    glay, olay = max_layer
+    wl = MAX_WL.with_(afmt=afmt, T=T)
+    check_layer(glay, olay, wl, activations(wl, batch=T + 7), range(T), bits=2)
+
+
 def test_max_sizes_tensor_core(max_layer):
     glay, olay = max_layer
     wl = MAX_WL.with_(afmt=W.A_BF16, T=300)
